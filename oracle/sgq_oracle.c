@@ -1,0 +1,332 @@
+/*
+ * sgq_oracle.c -- the CPU oracle for the activation-sparse int4 GEMV.
+ *
+ * TEST INFRASTRUCTURE ONLY: a plain, slow, obviously correct fp64 restatement
+ * of the hot path, used to check the CUDA library and to time a CPU baseline.
+ * It shares no code with the CUDA library and the library never calls it.
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -shared -fPIC.
+ *
+ * Sources, by page and section:
+ *   [P1] "Enabling Dynamic Sparsity in Quantized LLM Inference", Abstract.
+ *   [P5] "SVD Contextual Sparsity Predictors for Fast LLM Inference", Abstract.
+ *
+ * Every floating-point step is a single IEEE double operation (no contraction),
+ * so results do not depend on the compiler.
+ */
+#include "sgq_oracle.h"
+
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+
+/* ------------------------------------------------------------------------- */
+/* Number formats.                                                           */
+/* ------------------------------------------------------------------------- */
+
+/* Round a >= 0 (finite) to the nearest number that has p significant bits and
+ * an exponent no lower than emin (values below 2^emin share the quantum of the
+ * lowest normal binade, i.e. they become subnormals). Ties go to even. */
+static double round_to_grid(double a, int p, int emin)
+{
+    if (a == 0.0)
+        return 0.0;
+    int e;
+    frexp(a, &e);            /* a in [2^(e-1), 2^e) */
+    int E = e - 1;
+    if (E < emin)
+        E = emin;
+    double quantum = ldexp(1.0, E - (p - 1));
+    return nearbyint(a / quantum) * quantum; /* a / quantum is exact */
+}
+
+/* Encode a value that is already on the grid of a format with p significant
+ * bits, minimum normal exponent emin and exponent bias 'bias'. */
+static uint32_t encode_on_grid(double a, int p, int emin, int bias)
+{
+    if (a == 0.0)
+        return 0;
+    if (a < ldexp(1.0, emin))          /* subnormal: a = m * 2^(emin-p+1) */
+        return (uint32_t)(a / ldexp(1.0, emin - (p - 1)));
+    int e;
+    double f = frexp(a, &e);           /* a = f * 2^e, f in [0.5, 1) */
+    uint32_t m = (uint32_t)(f * ldexp(1.0, p)) - (1u << (p - 1));
+    return ((uint32_t)(e - 1 + bias) << (p - 1)) | m;
+}
+
+double oracle_half_to_double(uint16_t h)
+{
+    int sign = h >> 15;
+    int e = (h >> 10) & 0x1f;
+    int m = h & 0x3ff;
+    double v;
+    if (e == 0)
+        v = ldexp((double)m, -24);                 /* subnormal */
+    else if (e == 31)
+        v = m ? NAN : INFINITY;
+    else
+        v = ldexp((double)(1024 + m), e - 15 - 10);
+    return sign ? -v : v;
+}
+
+uint16_t oracle_double_to_half(double v)
+{
+    if (isnan(v))
+        return 0x7e00;
+    uint16_t sign = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (isinf(a))
+        return sign | 0x7c00;
+    a = round_to_grid(a, 11, -14);
+    if (a >= 65536.0)                             /* rounded past the largest finite */
+        return sign | 0x7c00;
+    return sign | (uint16_t)encode_on_grid(a, 11, -14, 15);
+}
+
+double oracle_bf16_to_double(uint16_t b)
+{
+    int sign = b >> 15;
+    int e = (b >> 7) & 0xff;
+    int m = b & 0x7f;
+    double v;
+    if (e == 0)
+        v = ldexp((double)m, -133);                /* subnormal */
+    else if (e == 255)
+        v = m ? NAN : INFINITY;
+    else
+        v = ldexp((double)(128 + m), e - 127 - 7);
+    return sign ? -v : v;
+}
+
+uint16_t oracle_double_to_bf16(double v)
+{
+    if (isnan(v))
+        return 0x7fc0;
+    uint16_t sign = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (isinf(a))
+        return sign | 0x7f80;
+    a = round_to_grid(a, 8, -126);
+    if (a >= ldexp(1.0, 128))
+        return sign | 0x7f80;
+    return sign | (uint16_t)encode_on_grid(a, 8, -126, 127);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Group-wise asymmetric int4 quantization ([P1] Abstract: group-wise low-bit  */
+/* quantization is the dominant way to fit the weights).                     */
+/* Readings (the page fixes none of these): 4 bits, asymmetric, one group =   */
+/* g consecutive input channels of one output row; the range always contains */
+/* 0; scale s = fp16(range / 15); zero z = rint(-lo / s) clamped to [0, 15],  */
+/* stored as an integer-valued fp16; code q = clamp(rint(w / s) + z, 0, 15);  */
+/* rint rounds half to even; a group whose scale is 0 gets s = 1, z = 0.      */
+/* ------------------------------------------------------------------------- */
+
+/* Clamp to [0, 15]; a zero (including -0, from -lo when lo = +0) becomes +0,
+ * since the zero point and the codes are unsigned integers. */
+static double clamp15(double v)
+{
+    if (v <= 0.0)
+        return 0.0;
+    if (v > 15.0)
+        return 15.0;
+    return v;
+}
+
+int oracle_quantize(const uint16_t *W, int N, int K, int g,
+                    uint8_t *q, uint16_t *s, uint16_t *z)
+{
+    if (N <= 0 || K <= 0 || g <= 0 || K % g != 0)
+        return -2;
+    int G = K / g;
+    for (int n = 0; n < N; ++n) {
+        for (int grp = 0; grp < G; ++grp) {
+            const uint16_t *wrow = W + (size_t)n * K + (size_t)grp * g;
+            double lo = 0.0, hi = 0.0;
+            for (int j = 0; j < g; ++j) {
+                double w = oracle_half_to_double(wrow[j]);
+                if (!isfinite(w))
+                    return -1;
+                if (w < lo)
+                    lo = w;
+                if (w > hi)
+                    hi = w;
+            }
+            uint16_t s_bits = oracle_double_to_half((hi - lo) / 15.0);
+            double sv = oracle_half_to_double(s_bits);
+            double zv;
+            if (sv == 0.0) {
+                s_bits = 0x3c00; /* 1.0 */
+                sv = 1.0;
+                zv = 0.0;
+            } else {
+                zv = clamp15(nearbyint(-lo / sv));
+            }
+            s[(size_t)n * G + grp] = s_bits;
+            z[(size_t)n * G + grp] = oracle_double_to_half(zv);
+            for (int j = 0; j < g; ++j) {
+                double w = oracle_half_to_double(wrow[j]);
+                double c = clamp15(nearbyint(w / sv) + zv);
+                q[(size_t)n * K + (size_t)grp * g + j] = (uint8_t)c;
+            }
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Packed layout, version 1 (the library's own format; the page names a      */
+/* sparsity-aware layout for memory locality but does not give it).          */
+/* Channel-major: row k of qweight holds the codes of input channel k for    */
+/* all N outputs, so skipping channel k skips one run of N/2 bytes.          */
+/*   qweight[k][b] = q[2b][k] | q[2b+1][k] << 4                              */
+/*   sz[grp][n][0] = s[n][grp],  sz[grp][n][1] = z[n][grp]                   */
+/* ------------------------------------------------------------------------- */
+
+int oracle_pack_layout(const uint8_t *q, const uint16_t *s, const uint16_t *z,
+                       int N, int K, int g, uint8_t *qweight, uint16_t *sz)
+{
+    if (N <= 0 || K <= 0 || g <= 0 || K % g != 0 || N % 2 != 0)
+        return -2;
+    int G = K / g;
+    for (int k = 0; k < K; ++k)
+        for (int b = 0; b < N / 2; ++b) {
+            uint8_t lo = q[(size_t)(2 * b) * K + k];
+            uint8_t hi = q[(size_t)(2 * b + 1) * K + k];
+            qweight[(size_t)k * (N / 2) + b] = (uint8_t)(lo | (hi << 4));
+        }
+    for (int grp = 0; grp < G; ++grp)
+        for (int n = 0; n < N; ++n) {
+            sz[((size_t)grp * N + n) * 2 + 0] = s[(size_t)n * G + grp];
+            sz[((size_t)grp * N + n) * 2 + 1] = z[(size_t)n * G + grp];
+        }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Active set ([P1] Abstract: dynamic sparsity, runtime gathering of the     */
+/* sparse indices; [P5] Abstract: ReGLU neurons that are zero are skipped).  */
+/* Readings: channel k is active when |x[k]| > t (strict), so t = 0 keeps    */
+/* exactly the nonzero channels; NaN is never active; indices ascend; for a  */
+/* batch the active set is the union over rows.                              */
+/* ------------------------------------------------------------------------- */
+
+int oracle_select(const uint16_t *x, int B, int K, const float *t,
+                  int32_t *idx, int32_t *count)
+{
+    if (B <= 0 || K <= 0)
+        return -2;
+    int32_t c = 0;
+    for (int k = 0; k < K; ++k) {
+        int active = 0;
+        for (int b = 0; b < B; ++b) {
+            double a = fabs(oracle_bf16_to_double(x[(size_t)b * K + k]));
+            if (a > (double)t[b])
+                active = 1;
+        }
+        if (active)
+            idx[c++] = k;
+    }
+    *count = c;
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* The sparse GEMV: y = W_deq[:, S] x[S] with W_deq[n][k] = s (q - z) of the  */
+/* group of k ([P1] Abstract: a GEMV over the quantized weights restricted   */
+/* to the active channels). Every row of a batch uses the same active set.   */
+/* ------------------------------------------------------------------------- */
+
+int oracle_gemv(const uint8_t *q, const uint16_t *s, const uint16_t *z,
+                int N, int K, int g, const uint16_t *x, int B,
+                const int32_t *idx, int count,
+                double *y, double *sumabs, uint16_t *y_bf16)
+{
+    if (N <= 0 || K <= 0 || g <= 0 || K % g != 0 || B <= 0 || count < 0 || count > K)
+        return -2;
+    int G = K / g;
+    for (int i = 0; i < count; ++i)
+        if (idx[i] < 0 || idx[i] >= K)
+            return -3;
+    for (int b = 0; b < B; ++b) {
+        for (int n = 0; n < N; ++n) {
+            double acc = 0.0, acc_abs = 0.0;
+            for (int i = 0; i < count; ++i) {
+                int k = idx[i];
+                int grp = k / g;
+                double sv = oracle_half_to_double(s[(size_t)n * G + grp]);
+                double zv = oracle_half_to_double(z[(size_t)n * G + grp]);
+                double w = sv * ((double)q[(size_t)n * K + k] - zv);
+                double p = w * oracle_bf16_to_double(x[(size_t)b * K + k]);
+                acc += p;
+                acc_abs += fabs(p);
+            }
+            size_t o = (size_t)b * N + n;
+            if (y)
+                y[o] = acc;
+            if (sumabs)
+                sumabs[o] = acc_abs;
+            if (y_bf16)
+                y_bf16[o] = oracle_double_to_bf16(acc);
+        }
+    }
+    return 0;
+}
+
+int oracle_gemv_dense(const uint8_t *q, const uint16_t *s, const uint16_t *z,
+                      int N, int K, int g, const uint16_t *x, int B,
+                      double *y, double *sumabs, uint16_t *y_bf16)
+{
+    if (N <= 0 || K <= 0 || g <= 0 || K % g != 0 || B <= 0)
+        return -2;
+    int G = K / g;
+    for (int b = 0; b < B; ++b) {
+        for (int n = 0; n < N; ++n) {
+            double acc = 0.0, acc_abs = 0.0;
+            for (int k = 0; k < K; ++k) {
+                int grp = k / g;
+                double sv = oracle_half_to_double(s[(size_t)n * G + grp]);
+                double zv = oracle_half_to_double(z[(size_t)n * G + grp]);
+                double w = sv * ((double)q[(size_t)n * K + k] - zv);
+                double p = w * oracle_bf16_to_double(x[(size_t)b * K + k]);
+                acc += p;
+                acc_abs += fabs(p);
+            }
+            size_t o = (size_t)b * N + n;
+            if (y)
+                y[o] = acc;
+            if (sumabs)
+                sumabs[o] = acc_abs;
+            if (y_bf16)
+                y_bf16[o] = oracle_double_to_bf16(acc);
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Gated activation between the up/gate and down projections of an FFN       */
+/* ([P5] Abstract: ReGLU FFNs, whose ReLU zeros are the skipped neurons).    */
+/* h = act(gate) * up; SiLU(v) = v / (1 + e^-v); ReLU(v) = v if v > 0 else 0. */
+/* ------------------------------------------------------------------------- */
+
+int oracle_glu(const uint16_t *gate, const uint16_t *up, int64_t n, int act,
+               double *h, uint16_t *h_bf16)
+{
+    if (n < 0 || (act != 0 && act != 1))
+        return -2;
+    for (int64_t i = 0; i < n; ++i) {
+        double gv = oracle_bf16_to_double(gate[i]);
+        double uv = oracle_bf16_to_double(up[i]);
+        double a;
+        if (act == 0)
+            a = gv / (1.0 + exp(-gv));
+        else
+            a = (gv > 0.0) ? gv : 0.0;
+        double hv = a * uv;
+        if (h)
+            h[i] = hv;
+        if (h_bf16)
+            h_bf16[i] = oracle_double_to_bf16(hv);
+    }
+    return 0;
+}
