@@ -1,0 +1,268 @@
+// api.cu -- the extern "C" entry points of libsgq (declared in include/sgq.h).
+// Host-side argument checks, then one launch on the caller's stream. Nothing
+// here allocates, frees or synchronises.
+#include "sgq_launch.h"
+
+#include <cuda_runtime.h>
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+constexpr int kMaxDevices = 64;
+int g_num_sms[kMaxDevices];      // 0 = not queried yet
+int g_device_ok[kMaxDevices];    // 0 = unknown, 1 = sm_10x, -1 = other
+
+int fail_cuda(cudaError_t e)
+{
+    g_last_cuda_error = (int)e;
+    return SGQ_ERR_CUDA;
+}
+
+// SM count of the current device (cached), or a negative SGQ_ERR_*.
+int current_device_sms()
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return fail_cuda(e);
+    if (dev < 0 || dev >= kMaxDevices)
+        return SGQ_ERR_DEVICE;
+    if (g_device_ok[dev] == 0) {
+        int major = 0, sms = 0;
+        if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) !=
+            cudaSuccess)
+            return fail_cuda(e);
+        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) !=
+            cudaSuccess)
+            return fail_cuda(e);
+        g_num_sms[dev] = sms;
+        g_device_ok[dev] = (major == 10) ? 1 : -1;
+    }
+    if (g_device_ok[dev] != 1)
+        return SGQ_ERR_DEVICE;
+    return g_num_sms[dev];
+}
+
+bool aligned16(const void *p)
+{
+    return ((uintptr_t)p & 15u) == 0;
+}
+
+bool group_ok(int group)
+{
+    return group == 32 || group == 64 || group == 128;
+}
+
+int check_weights(int N, int K, int group)
+{
+    if (!group_ok(group))
+        return SGQ_ERR_GROUP;
+    if (N <= 0 || K <= 0 || N % 32 != 0 || K % group != 0)
+        return SGQ_ERR_SHAPE;
+    if ((long long)N * K > (1LL << 40))
+        return SGQ_ERR_SHAPE;
+    return SGQ_OK;
+}
+
+int run_gemv(sgq::GemvProblem &p, size_t ws_bytes, void *workspace, void *stream)
+{
+    int rc = check_weights(p.N, p.K, p.group);
+    if (rc)
+        return rc;
+    if (p.B < 1 || p.B > SGQ_MAX_BATCH)
+        return SGQ_ERR_BATCH;
+    if (!p.qweight || !p.sz || !p.x || !p.y || !workspace)
+        return SGQ_ERR_NULL;
+    if (p.source == sgq::ROWS_LIST && (!p.idx || !p.count))
+        return SGQ_ERR_NULL;
+    if (!aligned16(p.qweight) || !aligned16(p.sz) || !aligned16(p.x) || !aligned16(p.y) ||
+        !aligned16(workspace) || (p.y_f32 && !aligned16(p.y_f32)))
+        return SGQ_ERR_ALIGN;
+    if (p.source == sgq::ROWS_THRESH && (p.B != 1 || p.K % 8 != 0))
+        return SGQ_ERR_SHAPE;
+    if (ws_bytes < sgq::gemv_workspace_bytes(p.N, p.B))
+        return SGQ_ERR_WORKSPACE;
+    const int sms = current_device_sms();
+    if (sms < 0)
+        return sms;
+    p.ws_acc = static_cast<float *>(workspace);
+    cudaError_t e = sgq::launch_gemv(p, sms, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+        return fail_cuda(e);
+    return SGQ_OK;
+}
+
+} // namespace
+
+extern "C" {
+
+int sgq_layout_version(void)
+{
+    return SGQ_LAYOUT_VERSION;
+}
+
+int sgq_last_cuda_error(void)
+{
+    return g_last_cuda_error;
+}
+
+const char *sgq_status_string(int code)
+{
+    switch (code) {
+    case SGQ_OK: return "ok";
+    case SGQ_ERR_NULL: return "a required pointer is NULL";
+    case SGQ_ERR_SHAPE: return "shape out of range or not divisible as required";
+    case SGQ_ERR_GROUP: return "group size must be 32, 64 or 128";
+    case SGQ_ERR_ALIGN: return "a device pointer is not 16-byte aligned";
+    case SGQ_ERR_BATCH: return "batch must be between 1 and 16";
+    case SGQ_ERR_WORKSPACE: return "workspace smaller than sgq_gemv_workspace_bytes";
+    case SGQ_ERR_ACT: return "unknown activation";
+    case SGQ_ERR_CUDA: return "a CUDA call failed (see sgq_last_cuda_error)";
+    case SGQ_ERR_DEVICE: return "the current device is not compute capability 10.x (B200)";
+    default: return "unknown sgq status";
+    }
+}
+
+int sgq_packed_sizes(int N, int K, int group, size_t *qweight_bytes, size_t *sz_bytes)
+{
+    int rc = check_weights(N, K, group);
+    if (rc)
+        return rc;
+    if (!qweight_bytes || !sz_bytes)
+        return SGQ_ERR_NULL;
+    *qweight_bytes = (size_t)K * (N / 2);
+    *sz_bytes = (size_t)(K / group) * N * 4;
+    return SGQ_OK;
+}
+
+int sgq_pack(const void *W, int N, int K, int group, void *qweight, void *sz, int32_t *status,
+             void *stream)
+{
+    int rc = check_weights(N, K, group);
+    if (rc)
+        return rc;
+    if (!W || !qweight || !sz)
+        return SGQ_ERR_NULL;
+    if (!aligned16(W) || !aligned16(qweight) || !aligned16(sz))
+        return SGQ_ERR_ALIGN;
+    int sms = current_device_sms();
+    if (sms < 0)
+        return sms;
+    cudaError_t e = sgq::launch_pack(static_cast<const uint16_t *>(W), N, K, group,
+                                     static_cast<uint8_t *>(qweight),
+                                     static_cast<uint32_t *>(sz), status,
+                                     static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SGQ_OK : fail_cuda(e);
+}
+
+int sgq_select(const void *x, int B, int K, const float *t_host, int32_t *idx, int32_t *count,
+               void *stream)
+{
+    if (B < 1 || B > SGQ_MAX_BATCH)
+        return SGQ_ERR_BATCH;
+    if (K <= 0 || K % 8 != 0)
+        return SGQ_ERR_SHAPE;
+    if (!x || !t_host || !idx || !count)
+        return SGQ_ERR_NULL;
+    if (!aligned16(x) || !aligned16(idx))
+        return SGQ_ERR_ALIGN;
+    int sms = current_device_sms();
+    if (sms < 0)
+        return sms;
+    sgq::Thresholds th{};
+    for (int b = 0; b < B; ++b)
+        th.t[b] = t_host[b];
+    cudaError_t e = sgq::launch_select(static_cast<const uint16_t *>(x), B, K, th, idx, count,
+                                       static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SGQ_OK : fail_cuda(e);
+}
+
+size_t sgq_gemv_workspace_bytes(int N, int K, int B)
+{
+    (void)K;
+    if (N <= 0 || B < 1 || B > SGQ_MAX_BATCH)
+        return 0;
+    return sgq::gemv_workspace_bytes(N, B);
+}
+
+int sgq_gemv(const void *qweight, const void *sz, int N, int K, int group, const void *x, int B,
+             const int32_t *idx, const int32_t *count, void *y, float *y_f32, void *workspace,
+             size_t ws_bytes, int32_t *status, void *stream)
+{
+    sgq::GemvProblem p{};
+    p.qweight = static_cast<const uint8_t *>(qweight);
+    p.sz = static_cast<const uint32_t *>(sz);
+    p.x = static_cast<const uint16_t *>(x);
+    p.idx = idx;
+    p.count = count;
+    p.y = static_cast<uint16_t *>(y);
+    p.y_f32 = y_f32;
+    p.status = status;
+    p.N = N;
+    p.K = K;
+    p.group = group;
+    p.B = B;
+    p.source = sgq::ROWS_LIST;
+    return run_gemv(p, ws_bytes, workspace, stream);
+}
+
+int sgq_gemv_thresh(const void *qweight, const void *sz, int N, int K, int group, const void *x,
+                    float t, void *y, float *y_f32, void *workspace, size_t ws_bytes,
+                    int32_t *status, void *stream)
+{
+    sgq::GemvProblem p{};
+    p.qweight = static_cast<const uint8_t *>(qweight);
+    p.sz = static_cast<const uint32_t *>(sz);
+    p.x = static_cast<const uint16_t *>(x);
+    p.y = static_cast<uint16_t *>(y);
+    p.y_f32 = y_f32;
+    p.status = status;
+    p.N = N;
+    p.K = K;
+    p.group = group;
+    p.B = 1;
+    p.t = t;
+    p.source = sgq::ROWS_THRESH;
+    return run_gemv(p, ws_bytes, workspace, stream);
+}
+
+int sgq_gemv_dense(const void *qweight, const void *sz, int N, int K, int group, const void *x,
+                   int B, void *y, float *y_f32, void *workspace, size_t ws_bytes,
+                   int32_t *status, void *stream)
+{
+    sgq::GemvProblem p{};
+    p.qweight = static_cast<const uint8_t *>(qweight);
+    p.sz = static_cast<const uint32_t *>(sz);
+    p.x = static_cast<const uint16_t *>(x);
+    p.y = static_cast<uint16_t *>(y);
+    p.y_f32 = y_f32;
+    p.status = status;
+    p.N = N;
+    p.K = K;
+    p.group = group;
+    p.B = B;
+    p.source = sgq::ROWS_DENSE;
+    return run_gemv(p, ws_bytes, workspace, stream);
+}
+
+int sgq_glu(const void *gate, const void *up, void *h, int B, int I, int act, void *stream)
+{
+    if (act != SGQ_ACT_SILU && act != SGQ_ACT_RELU)
+        return SGQ_ERR_ACT;
+    if (B < 1 || I <= 0 || ((long long)B * I) % 8 != 0)
+        return SGQ_ERR_SHAPE;
+    if (!gate || !up || !h)
+        return SGQ_ERR_NULL;
+    if (!aligned16(gate) || !aligned16(up) || !aligned16(h))
+        return SGQ_ERR_ALIGN;
+    int sms = current_device_sms();
+    if (sms < 0)
+        return sms;
+    cudaError_t e = sgq::launch_glu(static_cast<const uint16_t *>(gate),
+                                    static_cast<const uint16_t *>(up), static_cast<uint16_t *>(h),
+                                    (long long)B * I, act, sms, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SGQ_OK : fail_cuda(e);
+}
+
+} // extern "C"

@@ -1,0 +1,862 @@
+// gemv.cu -- the activation-sparse GEMV over group-wise int4 weights.
+//
+//   y[b][n] = sum_{k in S} s[g(k)][n] * (q[k][n] - z[g(k)][n]) * x[b][k]
+//
+// Method: "Enabling Dynamic Sparsity in Quantized LLM Inference", Abstract: a
+// GEMV that works on the quantized layout and reads only the weights of the
+// active input channels, gathered at run time. Layout version 1 keeps each
+// channel's codes as one contiguous run (N/2 bytes), so an inactive channel
+// costs no memory traffic at all.
+//
+// The path is HBM-bound (batch 1..16, no dense contraction, no tensor cores),
+// and at these sizes the whole GEMV is about one latency-bandwidth product of
+// HBM, so the kernel's job is to have nearly all of its bytes in flight early
+// and to keep the arithmetic under the memory time:
+//  * Outputs are cut into tiles (1024 outputs = 512 bytes of a packed row for
+//    B = 1; 256 outputs for B > 1); the rows (active channels) of each tile into
+//    k_splits shares so that n_tiles * k_splits CTAs cover the SMs.
+//  * Scale/zero of the CTA's groups are prefetched first; in the threshold
+//    path (select fused into the prologue) their span is known from the CTA's
+//    channel slice, before x is read.
+//  * Each warp takes a contiguous slice of the CTA's rows; every lane streams
+//    its own 16-byte (B = 1) or 4-byte (B > 1) column of each row through a
+//    per-lane ring in shared memory with cp.async, up to 16 rows ahead. A lane
+//    reads back only bytes it copied itself: no barrier, only its own groups.
+//  * B = 1: codes are summed per group without dequantizing
+//    (sum s (q - z) x = s (sum q x - z sum x)). One AND turns a code into an
+//    fp32 operand (the masked bits read as the subnormal q * 2^(p-149)); pairs
+//    of codes go through one packed f32x2 FMA with x scaled by a per-warp power
+//    of two so every product is exact and normal. Scale and zero are applied
+//    once per (group, output) in a fold.
+//  * B > 1: each code is dequantized exactly (one LOP3, one FMA, one add) and
+//    multiplied into B accumulators with packed f32x2 FMAs.
+//  * Split-K: each warp leaves its partial tile in its own (drained) ring
+//    region; after one barrier the CTA sums the warps' tiles (no shared
+//    atomics: many-way float atomics on the same addresses serialize) and adds
+//    the result into an fp32 workspace with vector reductions, then exits. A
+//    second tiny kernel, chained with programmatic dependent launch, turns the
+//    workspace into bf16 y and re-zeroes it once the GEMV grid has completed.
+//  * Programmatic dependent launch: a GEMV lets the next kernel in the stream
+//    launch early and itself waits for the previous one before it reads x,
+//    idx or count or writes anything; only the packed weights are read before.
+#include "sgq_device.cuh"
+#include "sgq_launch.h"
+
+#include <algorithm>
+
+namespace sgq {
+
+namespace {
+
+constexpr int kTileN1 = 1024;            // B = 1: outputs per tile, 32 per lane
+constexpr int kRowBytes1 = kTileN1 / 2;  // bytes of one packed row per tile
+constexpr int kTileNB = 256;             // B > 1: outputs per tile, 8 per lane
+constexpr int kRowBytesB = kTileNB / 2;
+
+struct KParams {
+    GemvProblem p;
+    int n_tiles;
+    int k_splits;
+    int rows_cap;  // capacity of the per-CTA row arrays
+    int span_cap;  // groups of scale/zero staged in shared memory per CTA
+    int lg;        // log2(group)
+};
+
+__device__ __forceinline__ int warp_max_exponent(float m)
+{
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1)
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, d));
+    if (!(m > 0.0f) || isinf(m))
+        return INT32_MIN; // all zero (or non-finite): no scaling
+    return ilogbf(m);
+}
+
+// Channel slice [c0, c1) of split s when channels are dealt out in runs of 8.
+__device__ __forceinline__ void channel_slice(const KParams &kp, int split, int &c0, int &c1)
+{
+    const int K8 = kp.p.K / 8;
+    c0 = (int)((long long)K8 * split / kp.k_splits) * 8;
+    c1 = (int)((long long)K8 * (split + 1) / kp.k_splits) * 8;
+}
+
+// ---------------------------------------------------------------------------
+// Row lists: fill ridx[0..nr) (and rx = x for ROWS_THRESH) for this CTA and
+// return nr. Entries outside [0, K) become -1 (their x is 0; they read row 0).
+// Must be called by all threads; ends with a barrier.
+// ---------------------------------------------------------------------------
+template <int SRC, int NT>
+__device__ int build_rows(const KParams &kp, int split, int32_t *ridx, float *rx, int *scan)
+{
+    const GemvProblem &p = kp.p;
+    const int tid = threadIdx.x;
+    if (SRC == ROWS_LIST) {
+        const int c = __ldg(p.count);
+        const int a = c < 0 ? 0 : (c > p.K ? p.K : c);
+        if (a != c && tid == 0 && blockIdx.x == 0)
+            set_status(p.status, SGQ_STATUS_BAD_COUNT);
+        const int r0 = (int)((long long)a * split / kp.k_splits);
+        const int r1 = (int)((long long)a * (split + 1) / kp.k_splits);
+        for (int j = tid; j < r1 - r0; j += NT) {
+            int k = __ldg(p.idx + r0 + j);
+            if ((unsigned)k >= (unsigned)p.K) {
+                set_status(p.status, SGQ_STATUS_BAD_INDEX);
+                k = -1;
+            }
+            ridx[j] = k;
+        }
+        __syncthreads();
+        return r1 - r0;
+    } else if (SRC == ROWS_DENSE) {
+        const int r0 = (int)((long long)p.K * split / kp.k_splits);
+        const int r1 = (int)((long long)p.K * (split + 1) / kp.k_splits);
+        for (int j = tid; j < r1 - r0; j += NT)
+            ridx[j] = r0 + j;
+        __syncthreads();
+        return r1 - r0;
+    } else {
+        // Threshold this CTA's channel slice: each warp takes runs of 32
+        // channels, one per lane; a ballot gives each run's active channels,
+        // a count per run and a prefix over runs give the ascending positions.
+        int c0, c1;
+        channel_slice(kp, split, c0, c1);
+        const int lane = tid & 31, warp = tid >> 5;
+        const int runs = (c1 - c0 + 31) / 32;
+        uint32_t mask[4];
+        float xv[4];
+        // Runs of this warp: warp, warp + NT/32, ... (the launcher keeps
+        // runs <= 4 * NT / 32).
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int q = warp + u * (NT / 32);
+            const int c = c0 + q * 32 + lane;
+            float v = 0.f;
+            bool act = false;
+            if (q < runs && c < c1) {
+                v = bf16_bits_to_float(__ldg(p.x + c));
+                act = fabsf(v) > p.t;
+            }
+            mask[u] = __ballot_sync(0xffffffffu, act);
+            xv[u] = v;
+            if (lane == 0 && q < runs)
+                scan[q] = __popc(mask[u]);
+        }
+        __syncthreads();
+        int total = 0;
+        for (int q = 0; q < runs; ++q)
+            total += scan[q];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int q = warp + u * (NT / 32);
+            if (q < runs && ((mask[u] >> lane) & 1u)) {
+                int pos = __popc(mask[u] & ((1u << lane) - 1u));
+                for (int r = 0; r < q; ++r)
+                    pos += scan[r];
+                ridx[pos] = c0 + q * 32 + lane;
+                rx[pos] = xv[u];
+            }
+        }
+        __syncthreads();
+        return total;
+    }
+}
+
+// Split-K epilogue, a second (tiny) kernel launched right behind the GEMV with
+// programmatic dependent launch: it waits until the GEMV grid has completed
+// (so every partial sum has been added into the workspace), converts the fp32
+// sums to bf16 y, writes the optional fp32 copy and re-zeroes the workspace.
+// Doing this in a kernel of its own keeps memory fences and tickets out of the
+// GEMV's CTAs, which just add their partials and exit.
+__global__ void __launch_bounds__(256) finalize_kernel(GemvProblem p)
+{
+    grid_launch_dependents();
+    grid_dependency_wait();
+    const int quads = p.N / 4;
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < p.B * quads;
+         e += gridDim.x * blockDim.x) {
+        const size_t o = (size_t)(e / quads) * p.N + (size_t)(e % quads) * 4;
+        float *wp = p.ws_acc + o;
+        const float4 v = ld_cg_v4(wp);
+        st_cg_v4(wp, make_float4(0.f, 0.f, 0.f, 0.f));
+        uint2 yb;
+        yb.x = (uint32_t)float_to_bf16_bits(v.x) | ((uint32_t)float_to_bf16_bits(v.y) << 16);
+        yb.y = (uint32_t)float_to_bf16_bits(v.z) | ((uint32_t)float_to_bf16_bits(v.w) << 16);
+        *reinterpret_cast<uint2 *>(p.y + o) = yb;
+        if (p.y_f32)
+            *reinterpret_cast<float4 *>(p.y_f32 + o) = v;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// B = 1
+// ---------------------------------------------------------------------------
+
+constexpr int kWarps1 = 8;
+constexpr int kThreads1 = kWarps1 * 32;
+constexpr int kStages1 = 24; // rows in flight per warp
+
+struct Smem1 {
+    size_t ring, szs, ridx, rx, scan, total;
+};
+
+// Each warp's ring region (kStages1 * 512 B = 12 KB) holds, once the warp has
+// consumed all of its rows, its partial tile (1024 floats = 4 KB).
+__host__ __device__ inline Smem1 smem1_layout(int span_cap, int rows_cap)
+{
+    Smem1 s;
+    s.ring = 0;
+    s.szs = s.ring + (size_t)kWarps1 * kStages1 * kRowBytes1;
+    s.ridx = s.szs + (size_t)span_cap * kTileN1 * 4;
+    s.rx = s.ridx + (size_t)rows_cap * 4;
+    s.scan = s.rx + (size_t)rows_cap * 4;
+    s.total = s.scan + (size_t)((rows_cap + 31) / 32 + 4) * 4;
+    return s;
+}
+
+__device__ __forceinline__ uint64_t pack2(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ float2 unpack2(uint64_t v)
+{
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+    return r;
+}
+
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint64_t ffma2p(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+// One packed 32-bit word (codes of 8 consecutive outputs) times x' into the
+// four pair accumulators of those outputs. Each code is isolated with one AND;
+// the masked register read as fp32 is the subnormal q * 2^(p - 149), exact.
+// Codes 5..7 are taken from word >> 12, so every code sits at bit offset
+// p in {0, 4, 8, 12, 16}: pairs (0,4) (8,12) (16,8) (12,16).
+__device__ __forceinline__ void mac_word(uint32_t w, uint64_t xb, uint64_t &a0, uint64_t &a1,
+                                         uint64_t &a2, uint64_t &a3)
+{
+    asm("{\n\t"
+        ".reg .b32 h, c0, c1, c2, c3, c4, c5, c6, c7;\n\t"
+        ".reg .b64 p0, p1, p2, p3;\n\t"
+        "shr.b32 h, %4, 12;\n\t"
+        "and.b32 c0, %4, 0x0000000F;\n\t"
+        "and.b32 c1, %4, 0x000000F0;\n\t"
+        "and.b32 c2, %4, 0x00000F00;\n\t"
+        "and.b32 c3, %4, 0x0000F000;\n\t"
+        "and.b32 c4, %4, 0x000F0000;\n\t"
+        "and.b32 c5, h, 0x00000F00;\n\t"
+        "and.b32 c6, h, 0x0000F000;\n\t"
+        "and.b32 c7, h, 0x000F0000;\n\t"
+        "mov.b64 p0, {c0, c1};\n\t"
+        "mov.b64 p1, {c2, c3};\n\t"
+        "mov.b64 p2, {c4, c5};\n\t"
+        "mov.b64 p3, {c6, c7};\n\t"
+        "fma.rn.f32x2 %0, p0, %5, %0;\n\t"
+        "fma.rn.f32x2 %1, p1, %5, %1;\n\t"
+        "fma.rn.f32x2 %2, p2, %5, %2;\n\t"
+        "fma.rn.f32x2 %3, p3, %5, %3;\n\t"
+        "}"
+        : "+l"(a0), "+l"(a1), "+l"(a2), "+l"(a3)
+        : "r"(w), "l"(xb));
+}
+
+// 2^(85 - p) for the two codes of pair m % 4 (see mac_word): turns
+// sum q x' 2^(p - 149) into 2^-64 sum q x'.
+__device__ __forceinline__ uint64_t fold_scale(int m4)
+{
+    const int p0 = (m4 == 0) ? 0 : (m4 == 1) ? 8 : (m4 == 2) ? 16 : 12;
+    const int p1 = (m4 == 0) ? 4 : (m4 == 1) ? 12 : (m4 == 2) ? 8 : 16;
+    return pack2(pow2f(85 - p0), pow2f(85 - p1));
+}
+
+__device__ __forceinline__ float half_lo(uint32_t w)
+{
+    return __half2float(__ushort_as_half((uint16_t)(w & 0xffffu)));
+}
+
+__device__ __forceinline__ float half_hi(uint32_t w)
+{
+    return __half2float(__ushort_as_half((uint16_t)(w >> 16)));
+}
+
+// Float4 slot of outputs 32l + 4c .. 32l + 4c + 3 (lane l, chunk c) inside a
+// warp's partial tile: the chunk index is XOR-ed with l & 7 so that a warp's
+// 128-bit stores (fixed c) and the readers' 128-bit loads (fixed l) are free
+// of bank conflicts.
+__device__ __forceinline__ int part_chunk(int l, int c)
+{
+    return 8 * l + (c ^ (l & 7));
+}
+
+template <int SRC>
+__global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
+{
+    extern __shared__ __align__(16) uint8_t smem[];
+    const GemvProblem &p = kp.p;
+    const Smem1 L = smem1_layout(kp.span_cap, kp.rows_cap);
+    uint8_t *ring = smem + L.ring;
+    const uint32_t *szs = reinterpret_cast<const uint32_t *>(smem + L.szs);
+    int32_t *ridx = reinterpret_cast<int32_t *>(smem + L.ridx);
+    float *rx = reinterpret_cast<float *>(smem + L.rx);
+    int *scan = reinterpret_cast<int *>(smem + L.scan);
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tile = blockIdx.x % kp.n_tiles;
+    const int split = blockIdx.x / kp.n_tiles;
+    const int n0 = tile * kTileN1;
+    const int lg = kp.lg;
+    const size_t row_stride = (size_t)(p.N / 2);
+    const bool lane_ok = (n0 + lane * 32) < p.N;
+
+    grid_launch_dependents();
+
+    // Scale/zero staging. With a fixed channel slice (threshold / dense) the
+    // groups are known now and are fetched before waiting on the previous
+    // kernel; with an index list they follow the list.
+    int G0 = 0, span = 0;
+    auto stage_sz = [&]() {
+        for (int c = tid; c < span * (kTileN1 / 4); c += kThreads1) {
+            const int r = c / (kTileN1 / 4), o = (c % (kTileN1 / 4)) * 4;
+            if (n0 + o < p.N)
+                cp_async16(smem + L.szs + ((size_t)r * kTileN1 + o) * 4,
+                           p.sz + (size_t)(G0 + r) * p.N + n0 + o);
+        }
+        cp_async_commit();
+    };
+    if (SRC != ROWS_LIST) {
+        int c0, c1;
+        if (SRC == ROWS_THRESH) {
+            channel_slice(kp, split, c0, c1);
+        } else {
+            c0 = (int)((long long)p.K * split / kp.k_splits);
+            c1 = (int)((long long)p.K * (split + 1) / kp.k_splits);
+        }
+        if (c1 > c0) {
+            G0 = c0 >> lg;
+            span = min(((c1 - 1) >> lg) - G0 + 1, kp.span_cap);
+        }
+        stage_sz();
+    }
+
+    grid_dependency_wait(); // x, idx, count may come from the previous kernel
+
+    const int nr = build_rows<SRC, kThreads1>(kp, split, ridx, rx, scan);
+
+    if (SRC == ROWS_LIST) {
+        if (nr > 0) {
+            const int kf = max(ridx[0], 0), kl = max(ridx[nr - 1], 0);
+            G0 = kf >> lg;
+            span = min(max((kl >> lg) - G0 + 1, 1), kp.span_cap);
+        }
+        stage_sz();
+    }
+
+    // This warp's contiguous slice of the CTA's rows.
+    const int wa = (int)((long long)nr * warp / kWarps1);
+    const int n = (int)((long long)nr * (warp + 1) / kWarps1) - wa;
+
+    // Ring prologue. Lanes past N read column 0 (valid memory, result unused);
+    // invalid rows read row 0 and have x = 0.
+    const uint8_t *wcol = p.qweight + (lane_ok ? ((size_t)n0 / 2 + lane * 16) : 0);
+    uint8_t *myring = ring + (size_t)warp * kStages1 * kRowBytes1 + lane * 16;
+#pragma unroll
+    for (int s = 0; s < kStages1; ++s) {
+        if (s < n)
+            cp_async16(myring + s * kRowBytes1, wcol + (size_t)max(ridx[wa + s], 0) * row_stride);
+        cp_async_commit();
+    }
+
+    // x of this warp's rows, scaled by 2^S so that every product
+    // q * x' * 2^(p-149) is a normal fp32 (exact); |x'| < 2^91.
+    if (SRC != ROWS_THRESH) {
+        for (int j = lane; j < n; j += 32) {
+            const int k = ridx[wa + j];
+            rx[wa + j] = (k >= 0) ? bf16_bits_to_float(__ldg(p.x + k)) : 0.f;
+        }
+        __syncwarp();
+    }
+    float m = 0.f;
+    for (int j = lane; j < n; j += 32)
+        m = fmaxf(m, fabsf(rx[wa + j]));
+    const int e = warp_max_exponent(m);
+    const int S = (e == INT32_MIN) ? 0 : 90 - e;
+    {
+        const float fa = pow2f(S - S / 2), fb = pow2f(S / 2);
+        for (int j = lane; j < n; j += 32)
+            rx[wa + j] = (rx[wa + j] * fa) * fb;
+    }
+    __syncwarp();
+
+    // Pair accumulators: accg = this group's sum of q x' 2^(p-149);
+    // acc = folded result in units of 2^(S-64).
+    uint64_t accg[16], acc[16];
+#pragma unroll
+    for (int m2 = 0; m2 < 16; ++m2) {
+        accg[m2] = 0ull;
+        acc[m2] = 0ull;
+    }
+    float Xg = 0.f;
+    int curG = (n > 0) ? (max(ridx[wa], 0) >> lg) : 0;
+
+    //   acc += s * (2^(85-p) accg - z * 2^-64 sum x')
+    auto fold = [&](int G) {
+        const bool staged = (G >= G0) && (G < G0 + span);
+        const uint32_t *src = staged ? (szs + (size_t)(G - G0) * kTileN1 + lane * 32)
+                                     : (p.sz + (size_t)G * p.N + n0 + (lane_ok ? lane * 32 : 0));
+        const float nx = -Xg * pow2f(-64);
+        const uint64_t nx2 = pack2(nx, nx);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const uint4 w4 = staged ? *reinterpret_cast<const uint4 *>(src + 4 * c)
+                                    : __ldg(reinterpret_cast<const uint4 *>(src + 4 * c));
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int m2 = 2 * c + h;
+                const uint32_t wa0 = h ? w4.z : w4.x, wa1 = h ? w4.w : w4.y;
+                uint64_t t = fmul2(accg[m2], fold_scale(m2 & 3));
+                t = ffma2p(pack2(half_hi(wa0), half_hi(wa1)), nx2, t);
+                acc[m2] = ffma2p(pack2(half_lo(wa0), half_lo(wa1)), t, acc[m2]);
+                accg[m2] = 0ull;
+            }
+        }
+        Xg = 0.f;
+    };
+
+    // The staged scale/zero (the oldest cp.async group) must be complete and
+    // visible to every warp before the first fold.
+    cp_async_wait<kStages1>();
+    __syncthreads();
+
+    // Two rows per iteration (more independent work per warp); a group change
+    // between the two takes the slower path that folds in between.
+    int i = 0, slot = 0;
+    for (; i + 1 < n; i += 2) {
+        cp_async_wait<kStages1 - 2>(); // rows i and i + 1 have landed
+        const int slot1 = (slot + 1 == kStages1) ? 0 : slot + 1;
+        const uint4 v0 = *reinterpret_cast<const uint4 *>(myring + slot * kRowBytes1);
+        const uint4 v1 = *reinterpret_cast<const uint4 *>(myring + slot1 * kRowBytes1);
+        const int G0r = max(ridx[wa + i], 0) >> lg;
+        const int G1r = max(ridx[wa + i + 1], 0) >> lg;
+        const float x0 = rx[wa + i], x1 = rx[wa + i + 1];
+        if (G0r != curG) {
+            fold(curG);
+            curG = G0r;
+        }
+        const uint64_t xb0 = pack2(x0, x0);
+        mac_word(v0.x, xb0, accg[0], accg[1], accg[2], accg[3]);
+        mac_word(v0.y, xb0, accg[4], accg[5], accg[6], accg[7]);
+        mac_word(v0.z, xb0, accg[8], accg[9], accg[10], accg[11]);
+        mac_word(v0.w, xb0, accg[12], accg[13], accg[14], accg[15]);
+        Xg += x0;
+        if (G1r != curG) {
+            fold(curG);
+            curG = G1r;
+        }
+        const uint64_t xb1 = pack2(x1, x1);
+        mac_word(v1.x, xb1, accg[0], accg[1], accg[2], accg[3]);
+        mac_word(v1.y, xb1, accg[4], accg[5], accg[6], accg[7]);
+        mac_word(v1.z, xb1, accg[8], accg[9], accg[10], accg[11]);
+        mac_word(v1.w, xb1, accg[12], accg[13], accg[14], accg[15]);
+        Xg += x1;
+        if (i + kStages1 < n)
+            cp_async16(myring + slot * kRowBytes1,
+                       wcol + (size_t)max(ridx[wa + i + kStages1], 0) * row_stride);
+        cp_async_commit();
+        if (i + 1 + kStages1 < n)
+            cp_async16(myring + slot1 * kRowBytes1,
+                       wcol + (size_t)max(ridx[wa + i + 1 + kStages1], 0) * row_stride);
+        cp_async_commit();
+        slot = (slot1 + 1 == kStages1) ? 0 : slot1 + 1;
+    }
+    if (i < n) {
+        cp_async_wait<kStages1 - 1>();
+        const uint4 v = *reinterpret_cast<const uint4 *>(myring + slot * kRowBytes1);
+        const int G = max(ridx[wa + i], 0) >> lg;
+        const float xs = rx[wa + i];
+        if (G != curG) {
+            fold(curG);
+            curG = G;
+        }
+        const uint64_t xb = pack2(xs, xs);
+        mac_word(v.x, xb, accg[0], accg[1], accg[2], accg[3]);
+        mac_word(v.y, xb, accg[4], accg[5], accg[6], accg[7]);
+        mac_word(v.z, xb, accg[8], accg[9], accg[10], accg[11]);
+        mac_word(v.w, xb, accg[12], accg[13], accg[14], accg[15]);
+        Xg += xs;
+    }
+    if (n > 0)
+        fold(curG);
+
+    // This warp's partial tile, in real units (x 2^(64-S), two exact
+    // factors), into its own ring region: every cp.async of this warp has
+    // landed and been read, so nothing else touches that region any more.
+    cp_async_wait_all();
+    __syncwarp();
+    {
+        float4 *part = reinterpret_cast<float4 *>(ring + (size_t)warp * kStages1 * kRowBytes1);
+        const int E = 64 - S;
+        const uint64_t f1 = pack2(pow2f(E / 2), pow2f(E / 2));
+        const uint64_t f2 = pack2(pow2f(E - E / 2), pow2f(E - E / 2));
+        const bool live = lane_ok && n > 0;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const float2 lo = unpack2(fmul2(fmul2(acc[2 * c], f1), f2));
+            const float2 hi = unpack2(fmul2(fmul2(acc[2 * c + 1], f1), f2));
+            part[part_chunk(lane, c)] =
+                live ? make_float4(lo.x, lo.y, hi.x, hi.y) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+    __syncthreads();
+    if (tid < kTileN1 / 4) {
+        const int l = tid >> 3, c = tid & 7;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < kWarps1; ++w) {
+            const float4 u = reinterpret_cast<const float4 *>(
+                ring + (size_t)w * kStages1 * kRowBytes1)[part_chunk(l, c)];
+            v.x += u.x;
+            v.y += u.y;
+            v.z += u.z;
+            v.w += u.w;
+        }
+        if (n0 + 4 * tid < p.N)
+            red_add_v4(p.ws_acc + n0 + 4 * tid, v);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 1 < B <= 16
+// ---------------------------------------------------------------------------
+
+constexpr int kWarpsB = 8;
+constexpr int kThreadsB = kWarpsB * 32;
+constexpr int kStagesB = 32; // 8 warps * 32 * 128 B = 32 KB ring
+
+struct SmemB {
+    size_t ring, szs, red, ridx, rx, scan, total;
+};
+
+__host__ __device__ inline SmemB smemB_layout(int span_cap, int rows_cap, int BT)
+{
+    SmemB s;
+    s.ring = 0;
+    s.szs = s.ring + (size_t)kWarpsB * kStagesB * kRowBytesB;
+    s.red = s.szs + (size_t)span_cap * kTileNB * 4;
+    s.ridx = s.red + (size_t)BT * kTileNB * 4;
+    s.rx = s.ridx + (size_t)rows_cap * 4;
+    s.scan = s.rx + (size_t)rows_cap * BT * 4;
+    s.total = s.scan + 64;
+    return s;
+}
+
+__host__ __device__ constexpr int code_pos(int j)
+{
+    // Bit offset of code j (0..7) of a packed word inside the register it is
+    // extracted from: codes 0..4 from the word itself, 5..7 from word >> 12.
+    return (j < 5) ? 4 * j : 4 * j - 12;
+}
+
+__host__ __device__ constexpr uint32_t code_mask(int j)
+{
+    return 0xFu << code_pos(j);
+}
+
+template <int BT, int SRC>
+__global__ void __launch_bounds__(kThreadsB, 1) gemv_bn_kernel(const KParams kp)
+{
+    extern __shared__ __align__(16) uint8_t smem[];
+    const GemvProblem &p = kp.p;
+    const SmemB L = smemB_layout(kp.span_cap, kp.rows_cap, BT);
+    uint8_t *ring = smem + L.ring;
+    const uint32_t *szs = reinterpret_cast<const uint32_t *>(smem + L.szs);
+    float *red = reinterpret_cast<float *>(smem + L.red);
+    int32_t *ridx = reinterpret_cast<int32_t *>(smem + L.ridx);
+    float *rx = reinterpret_cast<float *>(smem + L.rx);
+    int *scan = reinterpret_cast<int *>(smem + L.scan);
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tile = blockIdx.x % kp.n_tiles;
+    const int split = blockIdx.x / kp.n_tiles;
+    const int n0 = tile * kTileNB;
+    const int lg = kp.lg;
+    const int B = p.B;
+    const size_t row_stride = (size_t)(p.N / 2);
+    const bool lane_ok = (n0 + lane * 8) < p.N;
+
+    grid_launch_dependents();
+    grid_dependency_wait();
+    for (int i = tid; i < BT * kTileNB; i += kThreadsB)
+        red[i] = 0.f;
+
+    const int nr = build_rows<SRC, kThreadsB>(kp, split, ridx, rx, scan);
+
+    const int wa = (int)((long long)nr * warp / kWarpsB);
+    const int n = (int)((long long)nr * (warp + 1) / kWarpsB) - wa;
+
+    int G0 = 0, span = 0;
+    if (nr > 0) {
+        const int kf = max(ridx[0], 0), kl = max(ridx[nr - 1], 0);
+        G0 = kf >> lg;
+        span = min(max((kl >> lg) - G0 + 1, 1), kp.span_cap);
+    }
+    // 256 outputs * 4 bytes = 64 chunks of 16 bytes per group.
+    for (int c = tid; c < span * (kTileNB / 4); c += kThreadsB) {
+        const int r = c / (kTileNB / 4), o = (c % (kTileNB / 4)) * 4;
+        if (n0 + o < p.N)
+            cp_async16(smem + L.szs + ((size_t)r * kTileNB + o) * 4,
+                       p.sz + (size_t)(G0 + r) * p.N + n0 + o);
+    }
+    cp_async_commit();
+
+    const uint8_t *wcol = p.qweight + (lane_ok ? ((size_t)n0 / 2 + lane * 4) : 0);
+    uint8_t *myring = ring + (size_t)warp * kStagesB * kRowBytesB + lane * 4;
+#pragma unroll
+    for (int s = 0; s < kStagesB; ++s) {
+        if (s < n)
+            cp_async4(myring + s * kRowBytesB, wcol + (size_t)max(ridx[wa + s], 0) * row_stride);
+        cp_async_commit();
+    }
+
+    // x of every batch row for this warp's rows: rx[j * BT + b].
+    for (int e2 = lane; e2 < n * BT; e2 += 32) {
+        const int j = e2 / BT, b = e2 % BT;
+        const int k = ridx[wa + j];
+        rx[(size_t)(wa + j) * BT + b] =
+            (k >= 0 && b < B) ? bf16_bits_to_float(__ldg(p.x + (size_t)b * p.K + k)) : 0.f;
+    }
+    __syncwarp();
+
+    float2 acc[BT][4];
+#pragma unroll
+    for (int b = 0; b < BT; ++b)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            acc[b][j] = make_float2(0.f, 0.f);
+    // Per-group constants of the 8 outputs: sp = s 2^-p, cb = -2^(23-p) s, zs = z s,
+    // so that fma(2^23 + q 2^p, sp, cb) - zs = (q - z) s exactly.
+    float sp[8], cb[8], zs[8];
+    int curG = -1;
+
+    auto load_group = [&](int G) {
+        const bool staged = (G >= G0) && (G < G0 + span);
+        const uint32_t *src = staged ? (szs + (size_t)(G - G0) * kTileNB + lane * 8)
+                                     : (p.sz + (size_t)G * p.N + n0 + (lane_ok ? lane * 8 : 0));
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            uint4 v4 = staged ? *reinterpret_cast<const uint4 *>(src + 4 * c)
+                              : __ldg(reinterpret_cast<const uint4 *>(src + 4 * c));
+            const uint32_t w4[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int j = 4 * c + u;
+                const float s = half_lo(w4[u]);
+                const float z = half_hi(w4[u]);
+                sp[j] = s * pow2f(-code_pos(j));
+                cb[j] = -(s * pow2f(23 - code_pos(j)));
+                zs[j] = z * s;
+            }
+        }
+    };
+
+    cp_async_wait<kStagesB>();
+    __syncthreads();
+
+    for (int i = 0; i < n; ++i) {
+        cp_async_wait<kStagesB - 1>();
+        const int slot = i % kStagesB;
+        const uint32_t word = *reinterpret_cast<const uint32_t *>(myring + slot * kRowBytesB);
+        const int k = max(ridx[wa + i], 0);
+        const int G = k >> lg;
+        if (G != curG) {
+            load_group(G);
+            curG = G;
+        }
+        const uint32_t hi = word >> 12;
+        float w[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const uint32_t src = (j < 5) ? word : hi;
+            const float v = __uint_as_float((src & code_mask(j)) | 0x4B000000u);
+            w[j] = fmaf(v, sp[j], cb[j]) - zs[j];
+        }
+        const float *xr = rx + (size_t)(wa + i) * BT;
+#pragma unroll
+        for (int b = 0; b < BT; ++b) {
+            const float xv = xr[b];
+            const float2 xb = make_float2(xv, xv);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                acc[b][j] = ffma2(make_float2(w[2 * j], w[2 * j + 1]), xb, acc[b][j]);
+        }
+        const int nxt = i + kStagesB;
+        if (nxt < n)
+            cp_async4(myring + slot * kRowBytesB, wcol + (size_t)max(ridx[wa + nxt], 0) * row_stride);
+        cp_async_commit();
+    }
+
+    if (lane_ok && n > 0) {
+#pragma unroll
+        for (int b = 0; b < BT; ++b)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                // rotate by lane inside the 8 outputs of a lane to spread banks
+                atomicAdd(red + b * kTileNB + lane * 8 + ((2 * j + lane) & 7), acc[b][j].x);
+                atomicAdd(red + b * kTileNB + lane * 8 + ((2 * j + 1 + lane) & 7), acc[b][j].y);
+            }
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    for (int e2 = tid; e2 < B * (kTileNB / 4); e2 += kThreadsB) {
+        const int b = e2 / (kTileNB / 4), o = (e2 % (kTileNB / 4)) * 4;
+        const int l = o >> 3;
+        const float *rb = red + b * kTileNB + (l << 3);
+        const float4 v = make_float4(rb[(o + l) & 7], rb[(o + 1 + l) & 7], rb[(o + 2 + l) & 7],
+                                     rb[(o + 3 + l) & 7]);
+        if (n0 + o < p.N)
+            red_add_v4(p.ws_acc + (size_t)b * p.N + n0 + o, v);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host-side configuration
+// ---------------------------------------------------------------------------
+
+constexpr size_t kMaxSmem = 227 * 1024;
+
+int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+template <typename Kern, typename Arg>
+cudaError_t launch_pdl(Kern kern, int grid, int block, size_t smem, cudaStream_t stream,
+                       const Arg &arg)
+{
+    if (smem > 48 * 1024) {
+        cudaError_t err = cudaFuncSetAttribute(
+            kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (err != cudaSuccess)
+            return err;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, arg);
+}
+
+// The GEMV grid, then the split-K epilogue grid behind it.
+template <typename Kern>
+cudaError_t launch_gemv_and_finalize(Kern kern, int grid, int block, size_t smem,
+                                     cudaStream_t stream, const KParams &kp)
+{
+    cudaError_t err = launch_pdl(kern, grid, block, smem, stream, kp);
+    if (err != cudaSuccess)
+        return err;
+    const int quads = kp.p.B * (kp.p.N / 4);
+    const int fgrid = std::max(1, std::min(ceil_div(quads, 256), 148));
+    return launch_pdl(finalize_kernel, fgrid, 256, 0, stream, kp.p);
+}
+
+template <int SRC>
+cudaError_t launch_b1(KParams kp, int num_sms, cudaStream_t stream)
+{
+    const GemvProblem &p = kp.p;
+    kp.n_tiles = ceil_div(p.N, kTileN1);
+    kp.k_splits = std::max(1, num_sms / kp.n_tiles);
+    const int G = p.K >> kp.lg;
+    Smem1 L;
+    for (;;) {
+        kp.rows_cap = ceil_div(p.K, kp.k_splits) + 8;
+        kp.span_cap = std::min(G, ceil_div(p.K, (long long)kp.k_splits << kp.lg) + 2);
+        L = smem1_layout(kp.span_cap, kp.rows_cap);
+        // the threshold path handles at most 4 runs of 32 channels per warp
+        const bool runs_ok = (SRC != ROWS_THRESH) || (kp.rows_cap <= 4 * kThreads1);
+        if ((L.total <= kMaxSmem && runs_ok) || kp.k_splits >= p.K / 8)
+            break;
+        kp.k_splits *= 2;
+    }
+    if (L.total > kMaxSmem || (SRC == ROWS_THRESH && kp.rows_cap > 4 * kThreads1))
+        return cudaErrorInvalidConfiguration;
+    return launch_gemv_and_finalize(gemv_b1_kernel<SRC>, kp.n_tiles * kp.k_splits, kThreads1,
+                                    L.total, stream, kp);
+}
+
+template <int BT, int SRC>
+cudaError_t launch_bn_t(KParams kp, int num_sms, cudaStream_t stream)
+{
+    const GemvProblem &p = kp.p;
+    kp.n_tiles = ceil_div(p.N, kTileNB);
+    kp.k_splits = std::max(1, num_sms / kp.n_tiles);
+    const int G = p.K >> kp.lg;
+    SmemB L;
+    for (;;) {
+        kp.rows_cap = ceil_div(p.K, kp.k_splits) + 8;
+        kp.span_cap = std::min(G, ceil_div(p.K, (long long)kp.k_splits << kp.lg) + 2);
+        L = smemB_layout(kp.span_cap, kp.rows_cap, BT);
+        if (L.total <= kMaxSmem || kp.k_splits >= p.K / 8)
+            break;
+        kp.k_splits *= 2;
+    }
+    if (L.total > kMaxSmem)
+        return cudaErrorInvalidConfiguration;
+    return launch_gemv_and_finalize(gemv_bn_kernel<BT, SRC>, kp.n_tiles * kp.k_splits,
+                                    kThreadsB, L.total, stream, kp);
+}
+
+template <int SRC>
+cudaError_t launch_bn(KParams kp, int num_sms, cudaStream_t stream)
+{
+    const int B = kp.p.B;
+    if (B <= 2)
+        return launch_bn_t<2, SRC>(kp, num_sms, stream);
+    if (B <= 4)
+        return launch_bn_t<4, SRC>(kp, num_sms, stream);
+    if (B <= 8)
+        return launch_bn_t<8, SRC>(kp, num_sms, stream);
+    return launch_bn_t<16, SRC>(kp, num_sms, stream);
+}
+
+} // namespace
+
+size_t gemv_workspace_bytes(int N, int B)
+{
+    const size_t acc = (size_t)B * N * sizeof(float);
+    return (acc + 255) / 256 * 256;
+}
+
+cudaError_t launch_gemv(const GemvProblem &p, int num_sms, cudaStream_t stream)
+{
+    KParams kp{};
+    kp.p = p;
+    kp.lg = __builtin_ctz((unsigned)p.group);
+    if (p.B == 1) {
+        switch (p.source) {
+        case ROWS_LIST: return launch_b1<ROWS_LIST>(kp, num_sms, stream);
+        case ROWS_DENSE: return launch_b1<ROWS_DENSE>(kp, num_sms, stream);
+        default: return launch_b1<ROWS_THRESH>(kp, num_sms, stream);
+        }
+    }
+    if (p.source == ROWS_DENSE)
+        return launch_bn<ROWS_DENSE>(kp, num_sms, stream);
+    return launch_bn<ROWS_LIST>(kp, num_sms, stream);
+}
+
+} // namespace sgq

@@ -1,0 +1,49 @@
+// sgq_launch.h -- internal host-side launchers behind the C ABI (not exported).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/sgq.h"
+
+namespace sgq {
+
+struct Thresholds {
+    float t[SGQ_MAX_BATCH];
+};
+
+// Where the rows (active input channels) of a GEMV come from.
+enum RowSource : int {
+    ROWS_LIST = 0,   // device list idx[0..*count)
+    ROWS_DENSE = 1,  // every channel
+    ROWS_THRESH = 2, // |x[k]| > t, found by each CTA for its own channel slice
+};
+
+struct GemvProblem {
+    const uint8_t *qweight;
+    const uint32_t *sz;
+    const uint16_t *x;
+    const int32_t *idx;
+    const int32_t *count;
+    uint16_t *y;
+    float *y_f32;
+    float *ws_acc;
+    int32_t *status;
+    int N, K, group, B;
+    float t;
+    int source;
+};
+
+// Bytes of workspace (partial sums + tile counters) for N outputs, B rows.
+size_t gemv_workspace_bytes(int N, int B);
+
+cudaError_t launch_pack(const uint16_t *W, int N, int K, int g, uint8_t *qweight, uint32_t *sz,
+                        int32_t *status, cudaStream_t stream);
+cudaError_t launch_select(const uint16_t *x, int B, int K, const Thresholds &th, int32_t *idx,
+                          int32_t *count, cudaStream_t stream);
+cudaError_t launch_gemv(const GemvProblem &p, int num_sms, cudaStream_t stream);
+cudaError_t launch_glu(const uint16_t *gate, const uint16_t *up, uint16_t *h, long long n,
+                       int act, int num_sms, cudaStream_t stream);
+
+} // namespace sgq

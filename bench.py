@@ -1,0 +1,557 @@
+#!/usr/bin/env python3
+"""Benchmark of the activation-sparse int4 GEMV on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--path auto|list|thresh] [--sparsity 0.5] [--sweep]
+
+Workload: the Llama-3-8B FFN down_proj GEMV (K = 14336 input channels,
+N = 4096 outputs), int4 asymmetric weights in groups of 128 along K with fp16
+scale and zero, batch 1, x = SiLU(g) * u with g, u ~ N(0, 1) in bf16, and a
+magnitude threshold at the 50th percentile of |x| (50% activation sparsity).
+All inputs are synthetic and seeded; weights ~ N(0, 0.02).
+
+A step is one pass of the hot path over one activation vector: gathering the
+active channels and the sparse GEMV over them (select + gemv, or the fused
+threshold-GEMV). Steps cycle through R copies of the packed weights whose total
+size is more than 4x the L2 cache, so every step reads its weights from HBM.
+The K timed steps run as CUDA-graph replays on one stream, timed with CUDA
+events, bracketed by a barrier and a device synchronize.
+
+Metric: HBM GB/s on active bytes (and us per GEMV). Active bytes per GEMV are
+the weight bytes of the active channels (a*N/2), the scale/zero bytes of the
+groups they touch (4*N per group), the index and activation bytes (6*a) and
+the output (2*N).
+
+Multi-GPU: the path does not shard across GPUs in this workload (one GEMV per
+step); `--gpus N` under torchrun runs N independent replicas, each timing its
+own steps, and reports the units of all ranks over the slowest rank's time
+(weak scaling).
+
+`--impl reference` times the CPU oracle (the plain fp64 C restatement under
+oracle/) on the machine's host cores on a bounded sample of the same workload; it
+is a deliberately slow reference arm, not a target.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from activation_sparse_quantized_b200 import sgq                     # noqa: E402
+from activation_sparse_quantized_b200 import workloads as wl         # noqa: E402
+
+METRIC = "µs/GEMV and HBM GB/s on active bytes, int4 sparse GEMV, 8B FFN, 50% sparsity"
+UNIT = "GB/s"
+WORKLOAD = ("Llama-3-8B FFN down_proj GEMV: K=14336, N=4096, int4 asymmetric group 128 "
+            "(fp16 scale+zero), x = SiLU(g)*u bf16, batch 1, 50% magnitude sparsity")
+
+
+# ---------------------------------------------------------------------------
+# process / device plumbing
+# ---------------------------------------------------------------------------
+
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self, backend="nccl"):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", self.local)
+                                    if backend == "nccl" else None)
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, v: float) -> float:
+        if not self.pg:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def sum(self, v: float) -> float:
+        if not self.pg:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.SUM)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock"}
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.err = str(e)
+
+    def _sample(self):
+        self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+        try:
+            r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            r = self.nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        self.reasons |= int(r)
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._sample()
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self._thread.join()
+            self._sample()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def source_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "activation_sparse_quantized_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, src_hash: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)[kernel]
+        if d.get("source_hash") == src_hash:
+            return float(d["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+# ---------------------------------------------------------------------------
+# the workload
+# ---------------------------------------------------------------------------
+
+N, K, GROUP = wl.LLAMA8B_DOWN["N"], wl.LLAMA8B_DOWN["K"], wl.LLAMA8B_DOWN["group"]
+
+
+def active_bytes(a: int, touched_groups: int, n: int = N, B: int = 1) -> int:
+    return a * n // 2 + touched_groups * n * 4 + a * (4 + 2 * B) + 2 * B * n
+
+
+class Replica:
+    """R packed weight copies (> 4x L2 in total) and R activation vectors."""
+
+    def __init__(self, sparsity: float, seed: int = 0):
+        self.sparsity = sparsity
+        W = wl.weight(N, K, seed)
+        qw0, sz0 = sgq.alloc_packed(N, K, GROUP)
+        sgq.sgq_pack(W.cuda(), N, K, GROUP, qw0, sz0)
+        l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+        per = qw0.numel() + sz0.numel() * 4
+        self.R = max(2, int(math.ceil(4 * l2 / per)) + 1)
+        self.qw = [qw0] + [qw0.clone() for _ in range(self.R - 1)]
+        self.sz = [sz0] + [sz0.clone() for _ in range(self.R - 1)]
+        self.bytes_resident = self.R * per
+        self.l2 = l2
+        self.x_host = [wl.x_silu_gated(1, K, 1000 + r) for r in range(self.R)]
+        self.x = [x.cuda() for x in self.x_host]
+        self.t = [wl.percentile_threshold(x[0], sparsity) for x in self.x_host]
+        # per-copy index lists (for timing the GEMV kernel alone) and byte counts
+        self.idx, self.cnt, self.abytes, self.active = [], [], [], []
+        for r in range(self.R):
+            idx, cnt = sgq.alloc_select(K)
+            sgq.sgq_select(self.x[r], 1, K, [self.t[r]], idx, cnt)
+            a = int(cnt.item())
+            groups = int(np.unique(idx[:a].cpu().numpy() // GROUP).size)
+            self.idx.append(idx)
+            self.cnt.append(cnt)
+            self.active.append(a)
+            self.abytes.append(active_bytes(a, groups))
+        self.y = torch.empty(1, N, dtype=torch.bfloat16, device="cuda")
+        self.ws = sgq.alloc_workspace(N, K, 1)
+        self.sidx, self.scnt = sgq.alloc_select(K)
+
+    def step(self, r: int, path: str):
+        """One pass of the hot path on copy r (kernels launched: 2 or 1)."""
+        if path == "list":
+            sgq.sgq_select(self.x[r], 1, K, [self.t[r]], self.sidx, self.scnt)
+            sgq.sgq_gemv(self.qw[r], self.sz[r], N, K, GROUP, self.x[r], 1, self.sidx,
+                         self.scnt, self.y, None, self.ws)
+        else:
+            sgq.sgq_gemv_thresh(self.qw[r], self.sz[r], N, K, GROUP, self.x[r], self.t[r],
+                                self.y, None, self.ws)
+
+    def kernel_only(self, r: int, which: str):
+        if which == "gemv":
+            sgq.sgq_gemv(self.qw[r], self.sz[r], N, K, GROUP, self.x[r], 1, self.idx[r],
+                         self.cnt[r], self.y, None, self.ws)
+        elif which == "dense":
+            sgq.sgq_gemv_dense(self.qw[r], self.sz[r], N, K, GROUP, self.x[r], 1, self.y, None,
+                               self.ws)
+        elif which == "thresh":
+            sgq.sgq_gemv_thresh(self.qw[r], self.sz[r], N, K, GROUP, self.x[r], self.t[r],
+                                self.y, None, self.ws)
+        elif which == "select":
+            sgq.sgq_select(self.x[r], 1, K, [self.t[r]], self.sidx, self.scnt)
+
+
+class GraphRunner:
+    """Runs exactly n calls of fn(i) as replays of captured CUDA graphs."""
+
+    def __init__(self, fn, period: int, stream):
+        self.fn, self.period, self.stream = fn, period, stream
+        self.graphs = {}
+
+    def _graph(self, length: int, offset: int):
+        key = (length, offset)
+        if key not in self.graphs:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(self.stream):
+                with torch.cuda.graph(g, stream=self.stream):
+                    for i in range(length):
+                        self.fn(offset + i)
+            self.graphs[key] = g
+        return self.graphs[key]
+
+    def prepare(self, n: int):
+        full, rem = divmod(n, self.period)
+        if full:
+            self._graph(self.period, 0)
+        if rem:
+            self._graph(rem, 0)
+
+    def run(self, n: int):
+        full, rem = divmod(n, self.period)
+        for _ in range(full):
+            self._graph(self.period, 0).replay()
+        if rem:
+            self._graph(rem, 0).replay()
+
+
+def time_calls(fn, n: int, period: int, dist: Dist | None = None, warm: int = 3):
+    """Device time (ms) of exactly n calls of fn(i), via CUDA graphs."""
+    stream = torch.cuda.Stream()
+    gr = GraphRunner(fn, period, stream)
+    gr.prepare(n)
+    gr.prepare(max(warm, 1))
+    with torch.cuda.stream(stream):
+        gr.run(max(warm, 1))
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        gr.run(n)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    return e0.elapsed_time(e1)
+
+
+# ---------------------------------------------------------------------------
+# arms
+# ---------------------------------------------------------------------------
+
+def run_ours(args, dist: Dist):
+    torch.cuda.set_device(dist.local)
+    sgq.load()
+    rep = Replica(args.sparsity)
+    R = rep.R
+    path = args.path
+    if path == "auto":
+        path = "thresh"
+    kernels_per_step = 2 if path == "list" else 1
+    period = R * max(1, 64 // R)
+
+    # warm-up (untimed) then exactly K timed steps
+    stream = torch.cuda.Stream()
+    runner = GraphRunner(lambda i: rep.step(i % R, path), period, stream)
+    runner.prepare(args.steps)
+    runner.prepare(args.warmup)
+    with torch.cuda.stream(stream):
+        runner.run(args.warmup)
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dist.local) as clk:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            runner.run(args.steps)
+            e1.record(stream)
+        torch.cuda.synchronize()
+    dist.barrier()
+    ms_local = e0.elapsed_time(e1)
+    ms = dist.max(ms_local)
+    step_bytes = sum(rep.abytes[i % R] for i in range(args.steps))
+    total_bytes = dist.sum(step_bytes)
+    value = total_bytes / (ms * 1e-3) / 1e9
+    us_per_gemv = ms * 1e3 / args.steps
+
+    # the dominant kernel alone, same rotation, for the roofline
+    dom = "thresh" if path == "thresh" else "gemv"
+    nk = max(args.steps, 2 * R)
+    kms = time_calls(lambda i: rep.kernel_only(i % R, dom), nk, period)
+    k_us = kms * 1e3 / nk
+    k_bytes = sum(rep.abytes[i % R] for i in range(nk)) / nk
+    if dom == "thresh":   # reads all of x, no index list
+        k_bytes = k_bytes - 6 * np.mean(rep.active) + 2 * K
+    peak, peak_kind = measured_peak()
+    achieved = k_bytes / (k_us * 1e-6) / 1e9
+    src = source_hash("gemv.cu", "sgq_device.cuh")
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                "traffic": profiled_traffic(dom, src), "kernel": f"sgq_{dom}",
+                "kernel_us": round(k_us, 3), "algorithmic_bytes": int(k_bytes),
+                "frac_of_8TBps": round(achieved / 8000.0, 4)}
+
+    # comparison points on the same rotation: dense int4 GEMV, select alone
+    dense_ms = time_calls(lambda i: rep.kernel_only(i % R, "dense"), 2 * period, period)
+    sel_ms = time_calls(lambda i: rep.kernel_only(i % R, "select"), 2 * period, period)
+
+    e2e = run_e2e(rep, path, min(args.steps, 2000), args.warmup, dist)
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded; weights N(0,0.02), x = SiLU(g)*u)",
+        "config": {"workload": WORKLOAD, "K": K, "N": N, "group": GROUP, "batch": 1,
+                   "sparsity": args.sparsity, "active_channels": int(np.mean(rep.active)),
+                   "path": "select+gemv" if path == "list" else "gemv_thresh (select fused)",
+                   "l2": f"inputs larger than L2: {R} rotating weight copies, "
+                         f"{rep.bytes_resident / 1e6:.0f} MB vs L2 {rep.l2 / 1e6:.0f} MB",
+                   "parallelism": f"replicas x{dist.world}" if dist.world > 1 else "single GPU"},
+        "us_per_gemv": round(us_per_gemv, 3),
+        "active_bytes_per_gemv": int(np.mean(rep.abytes)),
+        "roofline": roofline,
+        "dense_int4_gemv_us": round(dense_ms * 1e3 / (2 * period), 3),
+        "select_us": round(sel_ms * 1e3 / (2 * period), 3),
+        "e2e": e2e,
+        "gpu_launches": args.steps * kernels_per_step,
+        "clocks": clk.summary(),
+    }
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    return line
+
+
+def run_e2e(rep: Replica, path: str, steps: int, warmup: int, dist: Dist):
+    """The same metric through the public API with host buffers: every step
+    copies x from pinned host memory, runs the path, and reads y back."""
+    xs = [x.pin_memory() for x in rep.x_host]
+    yh = torch.empty(1, N, dtype=torch.bfloat16).pin_memory()
+    xd = torch.empty(1, K, dtype=torch.bfloat16, device="cuda")
+    R = rep.R
+
+    def one(i):
+        r = i % R
+        xd.copy_(xs[r], non_blocking=True)
+        if path == "list":
+            sgq.sgq_select(xd, 1, K, [rep.t[r]], rep.sidx, rep.scnt)
+            sgq.sgq_gemv(rep.qw[r], rep.sz[r], N, K, GROUP, xd, 1, rep.sidx, rep.scnt, rep.y,
+                         None, rep.ws)
+        else:
+            sgq.sgq_gemv_thresh(rep.qw[r], rep.sz[r], N, K, GROUP, xd, rep.t[r], rep.y, None,
+                                rep.ws)
+        yh.copy_(rep.y, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+        return float(yh[0, 0])
+
+    for i in range(max(3, warmup)):
+        one(i)
+    torch.cuda.synchronize()
+    dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        one(i)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = dist.max(e0.elapsed_time(e1))
+    b = dist.sum(sum(rep.abytes[i % R] for i in range(steps)))
+    return {"value": round(b / (ms * 1e-3) / 1e9, 1), "unit": UNIT,
+            "us_per_gemv": round(ms * 1e3 / steps, 3), "steps": steps,
+            "h2d_bytes_per_step": 2 * K, "d2h_bytes_per_step": 2 * N}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timings (cpu_baseline leg and the reference arm)
+# ---------------------------------------------------------------------------
+
+class OracleSample:
+    """The oracle's select + GEMV on the benchmark workload (setup untimed)."""
+
+    def __init__(self, sparsity: float):
+        import oracle
+        self.o = oracle
+        self.W = wl.weight(N, K, 0)
+        self.x = wl.x_silu_gated(1, K, 1000)
+        self.t = [wl.percentile_threshold(self.x[0], sparsity)]
+        wb = self.W.view(torch.int16).numpy().view(np.uint16)
+        self.q, self.s, self.z = oracle.quantize(wb, GROUP)
+        self.xb = wl.bits(self.x)
+        idx = oracle.select(self.xb, self.t)
+        self.a = int(idx.size)
+        self.groups = int(np.unique(idx // GROUP).size)
+
+    def run(self, rows: np.ndarray):
+        """select + GEMV for the given outputs; returns the active bytes covered."""
+        idx = self.o.select(self.xb, self.t)
+        self.o.gemv(self.q[rows], self.s[rows], self.z[rows], GROUP, self.xb, idx)
+        n = len(rows)
+        return active_bytes(self.a, self.groups, n=n)
+
+
+def cpu_cores_used():
+    return 1   # the oracle is single-threaded C
+
+
+def cpu_baseline(seconds: float):
+    smp = OracleSample(0.5)
+    rows = np.arange(N)
+    done, t0 = 0, time.perf_counter()
+    reps = 0
+    while True:
+        done += smp.run(rows)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or reps >= 50:
+            break
+    return {"value": round(done / el / 1e9, 3), "unit": UNIT, "cores": cpu_cores_used(),
+            "kind": "oracle",
+            "sample": f"{reps} full GEMVs (select + fp64 GEMV, all {N} outputs) in {el:.1f} s, "
+                      f"host has {len(os.sched_getaffinity(0))} cores"}
+
+
+def run_reference(args, dist: Dist):
+    """The reference arm: the CPU oracle as it stands, on a bounded sample of
+    the workload per step (a slice of the outputs), K steps after W warm-up."""
+    smp = OracleSample(args.sparsity)
+    budget = max(60.0, 0.0) / max(args.steps + args.warmup, 1)
+    t0 = time.perf_counter()
+    smp.run(np.arange(8))
+    per_row = (time.perf_counter() - t0) / 8
+    nrows = int(max(1, min(N, budget / max(per_row, 1e-9))))
+    rng = np.random.default_rng(0)
+    for _ in range(args.warmup):
+        smp.run(np.sort(rng.choice(N, nrows, replace=False)))
+    done = 0
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        done += smp.run(np.sort(rng.choice(N, nrows, replace=False)))
+    el = time.perf_counter() - t0
+    value = done / el / 1e9
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT,
+            "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": el * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "K": K, "N": N, "group": GROUP, "batch": 1,
+                       "sparsity": args.sparsity,
+                       "path": "CPU oracle: select + fp64 GEMV (plain C, one thread)"},
+            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cpu_cores_used(),
+                             "kind": "oracle",
+                             "sample": f"each step: {nrows} of {N} outputs of the GEMV"},
+            "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--path", choices=["auto", "list", "thresh"], default="auto")
+    ap.add_argument("--sparsity", type=float, default=0.5)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    dist = Dist()
+    if dist.world != args.gpus and dist.world > 1:
+        args.gpus = dist.world
+    if args.impl == "reference":
+        if dist.rank == 0:
+            print(json.dumps(run_reference(args, dist)), flush=True)
+        return 0
+    dist.init("nccl")
+    try:
+        line = run_ours(args, dist)
+        if dist.rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        dist.close()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,186 @@
+/*
+ * sgq.h -- C ABI of libsgq: activation-sparse GEMV over group-wise int4 weights
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The operation ("Enabling Dynamic Sparsity in Quantized LLM Inference",
+ * Abstract): weights are quantized group-wise to low-bit codes, the input
+ * activation of a decode step is dynamically sparse, the active channel
+ * indices are gathered at run time, and a GEMV reads only the weights of the
+ * active channels:
+ *
+ *     y[b][n] = sum over k in S of  s[g(k)][n] * (q[k][n] - z[g(k)][n]) * x[b][k]
+ *     S       = { k : |x[b][k]| > t[b] for some row b }          (strict)
+ *
+ * With t = 0, S is the set of nonzero channels, which is how a ReGLU FFN skips
+ * its zero neurons ("SVD Contextual Sparsity Predictors for Fast LLM
+ * Inference", Abstract).
+ *
+ * Conventions for every call:
+ *  - Pointers named *_host are host memory; every other pointer is device
+ *    memory owned by the caller (the library allocates nothing, frees nothing
+ *    and never synchronises the stream or the device).
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream); all work
+ *    is enqueued asynchronously on it, in call order.
+ *  - Element types: fp16 and bf16 are passed as 16-bit IEEE / bfloat16 bit
+ *    patterns; all arrays are dense and row-major as stated.
+ *  - Device pointers must be 16-byte aligned.
+ *  - Return value: SGQ_OK (0) or a negative SGQ_ERR_* code. Argument errors are
+ *    detected on the host before anything is enqueued. SGQ_ERR_CUDA means a
+ *    launch failed; sgq_last_cuda_error() returns the cudaError_t.
+ *  - Faults found on the device (non-finite weights, indices out of range) are
+ *    OR-ed as SGQ_STATUS_* bits into an optional caller-owned int32 `status`
+ *    word in device memory (NULL = not reported). The offending work is
+ *    skipped, never performed out of bounds.
+ *  - Only one GPU is used: the current device of the calling thread.
+ */
+#ifndef SGQ_H
+#define SGQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SGQ_LAYOUT_VERSION 1
+#define SGQ_MAX_BATCH 16
+
+/* Return codes. */
+#define SGQ_OK              0
+#define SGQ_ERR_NULL       -1  /* a required pointer is NULL                     */
+#define SGQ_ERR_SHAPE      -2  /* N, K, B or a size out of range / indivisible   */
+#define SGQ_ERR_GROUP      -3  /* group size not 32, 64 or 128                   */
+#define SGQ_ERR_ALIGN      -4  /* a device pointer is not 16-byte aligned        */
+#define SGQ_ERR_BATCH      -5  /* B < 1 or B > SGQ_MAX_BATCH                     */
+#define SGQ_ERR_WORKSPACE  -6  /* workspace smaller than sgq_gemv_workspace_bytes */
+#define SGQ_ERR_ACT        -7  /* unknown activation                             */
+#define SGQ_ERR_CUDA       -8  /* a CUDA runtime call or launch failed           */
+#define SGQ_ERR_DEVICE     -9  /* current device is not compute capability 10.x  */
+
+/* Device status bits (OR-ed into the optional `status` word). */
+#define SGQ_STATUS_NONFINITE_W  1  /* sgq_pack: W holds NaN or Inf (that group packed as zeros) */
+#define SGQ_STATUS_BAD_INDEX    2  /* sgq_gemv: an index outside [0, K) was skipped             */
+#define SGQ_STATUS_BAD_COUNT    4  /* sgq_gemv: *count outside [0, K]; clamped                  */
+
+/* Activations for sgq_glu. */
+#define SGQ_ACT_SILU 0
+#define SGQ_ACT_RELU 1
+
+/*
+ * Sizes of the packed buffers for an N x K weight with the given group size.
+ *   qweight_bytes = K * N / 2          (uint8, layout below)
+ *   sz_bytes      = (K / group) * N * 4 (two fp16 per group and output)
+ * Requires N % 32 == 0, K % group == 0, group in {32, 64, 128}.
+ */
+int sgq_packed_sizes(int N, int K, int group, size_t *qweight_bytes, size_t *sz_bytes);
+
+/*
+ * Group-wise asymmetric int4 quantization of W and packing into the
+ * channel-major layout, version 1 (the abstract's group-wise quantization; the
+ * layout is this library's own: it keeps each input channel's codes
+ * contiguous so that skipping a channel skips one contiguous run of bytes).
+ *
+ *   W       fp16 [N][K] (torch.nn.Linear weight layout), read only.
+ *   qweight uint8 [K][N/2]: byte b of row k = q[2b][k] | q[2b+1][k] << 4.
+ *   sz      [K/group][N] pairs of fp16 (scale, zero), scale first.
+ * Per output n and group of `group` consecutive k: lo = min(0, min w),
+ * hi = max(0, max w), s = fp16(RN((hi - lo) / 15)), z = clamp(rint(-lo/s), 0, 15),
+ * q = clamp(rint(w / s) + z, 0, 15) in fp64 arithmetic, rint = half to even;
+ * a group with s == 0 gets s = 1, z = 0. A group holding NaN/Inf is packed as
+ * s = 1, z = 0, q = 0 and sets SGQ_STATUS_NONFINITE_W.
+ * Offline step; not tuned for speed.
+ */
+int sgq_pack(const void *W, int N, int K, int group, void *qweight, void *sz,
+             int32_t *status, void *stream);
+
+/*
+ * Runtime gathering of the active channels (the abstract's "compact runtime
+ * mechanism that gathers sparse indices").
+ *
+ *   x       bf16 [B][K]; t_host: B floats (host memory, read during the call).
+ *   idx     int32 [K] capacity; receives the ascending, unique active channels
+ *           k with |x[b][k]| > t[b] for at least one b (NaN never active).
+ *   count   int32 device scalar; receives |S|.
+ * Requires 1 <= B <= 16, K % 8 == 0. t < 0 selects every channel.
+ */
+int sgq_select(const void *x, int B, int K, const float *t_host,
+               int32_t *idx, int32_t *count, void *stream);
+
+/*
+ * Workspace for sgq_gemv / sgq_gemv_thresh / sgq_gemv_dense: B*N floats of
+ * split-K partial sums. It must be zero-filled once when it is allocated;
+ * every call leaves it zero-filled again. Calls that may run concurrently
+ * (different streams) must not share a workspace.
+ *
+ * Each GEMV call enqueues two kernels with programmatic dependent launch: the
+ * GEMV (which reads the packed weights before the previous kernel in the
+ * stream has finished, and x, idx, count only after) and a small epilogue that
+ * writes y. Do not write the packed weights in the kernel that immediately
+ * precedes a GEMV call in the same stream without a full stream dependency.
+ */
+size_t sgq_gemv_workspace_bytes(int N, int K, int B);
+
+/*
+ * The activation-sparse GEMV: y[b][n] = sum over i < *count of
+ * s (q - z) of (n, idx[i]) times x[b][idx[i]] (bf16 output, round to nearest
+ * even; fp32 accumulation). Every batch row uses the same active list
+ * (normally the union from sgq_select); rows are not masked inside it.
+ *
+ *   qweight, sz  packed by sgq_pack (layout version 1) for this N, K, group.
+ *   x            bf16 [B][K].
+ *   idx, count   device list and device count (as written by sgq_select).
+ *                Indices should ascend (any order in [0, K) is correct, only
+ *                slower); an index outside [0, K) is skipped and flagged.
+ *   y            bf16 [B][N] output.
+ *   y_f32        optional fp32 [B][N] copy of y before the bf16 rounding
+ *                (NULL = not written).
+ *   workspace    see sgq_gemv_workspace_bytes.
+ * The grid is fixed by (N, K, B, SM count), not by *count: nothing is read
+ * back to the host.
+ */
+int sgq_gemv(const void *qweight, const void *sz, int N, int K, int group,
+             const void *x, int B, const int32_t *idx, const int32_t *count,
+             void *y, float *y_f32, void *workspace, size_t ws_bytes,
+             int32_t *status, void *stream);
+
+/*
+ * Threshold and GEMV in one launch: the same result as sgq_select(x, t) followed
+ * by sgq_gemv on its output, with the selection done by each CTA for its own
+ * slice of channels (no index list in memory). B == 1 only.
+ */
+int sgq_gemv_thresh(const void *qweight, const void *sz, int N, int K, int group,
+                    const void *x, float t, void *y, float *y_f32,
+                    void *workspace, size_t ws_bytes, int32_t *status, void *stream);
+
+/*
+ * The dense int4 GEMV over the same packed weights (every channel active): the
+ * dense quantized inference that the abstract compares against.
+ */
+int sgq_gemv_dense(const void *qweight, const void *sz, int N, int K, int group,
+                   const void *x, int B, void *y, float *y_f32,
+                   void *workspace, size_t ws_bytes, int32_t *status, void *stream);
+
+/*
+ * Gated FFN activation h = act(gate) * up, elementwise over [B][I] bf16
+ * (fp32 arithmetic, bf16 round-to-nearest-even output). act = SGQ_ACT_SILU
+ * (v / (1 + e^-v)) or SGQ_ACT_RELU (v if v > 0 else 0, the ReGLU of the SVD
+ * predictor page, whose zeros sgq_select with t = 0 then skips).
+ * Requires (B * I) % 8 == 0.
+ */
+int sgq_glu(const void *gate, const void *up, void *h, int B, int I, int act, void *stream);
+
+/* Text for a return code (static string). */
+const char *sgq_status_string(int code);
+
+/* cudaError_t of the last SGQ_ERR_CUDA on this thread (0 if none). */
+int sgq_last_cuda_error(void);
+
+/* SGQ_LAYOUT_VERSION of the packed format this build reads and writes. */
+int sgq_layout_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SGQ_H */
