@@ -95,6 +95,11 @@ int run_gemv(sgq::GemvProblem &p, size_t ws_bytes, void *workspace, void *stream
 
 } // namespace
 
+int sgq::record_cuda_error(cudaError_t e)
+{
+    return fail_cuda(e);
+}
+
 extern "C" {
 
 int sgq_layout_version(void)
@@ -120,6 +125,7 @@ const char *sgq_status_string(int code)
     case SGQ_ERR_ACT: return "unknown activation";
     case SGQ_ERR_CUDA: return "a CUDA call failed (see sgq_last_cuda_error)";
     case SGQ_ERR_DEVICE: return "the current device is not compute capability 10.x (B200)";
+    case SGQ_ERR_TOO_LARGE: return "N exceeds SGQ_NOALLOC_MAX_N, the fixed scratch of sgq_gemv_thresh_noalloc";
     default: return "unknown sgq status";
     }
 }

@@ -43,6 +43,9 @@ cudaError_t launch_pack(const uint16_t *W, int N, int K, int g, uint8_t *qweight
 cudaError_t launch_select(const uint16_t *x, int B, int K, const Thresholds &th, int32_t *idx,
                           int32_t *count, cudaStream_t stream);
 cudaError_t launch_gemv(const GemvProblem &p, int num_sms, cudaStream_t stream);
+// Records e as the last CUDA error of this thread; returns SGQ_ERR_CUDA.
+int record_cuda_error(cudaError_t e);
+
 cudaError_t launch_glu(const uint16_t *gate, const uint16_t *up, uint16_t *h, long long n,
                        int act, int num_sms, cudaStream_t stream);
 

@@ -25,11 +25,12 @@ SGQ_STATUS_NONFINITE_W = 1
 SGQ_STATUS_BAD_INDEX = 2
 SGQ_STATUS_BAD_COUNT = 4
 SGQ_MAX_BATCH = 16
+SGQ_NOALLOC_MAX_N = 65536
 
 EXPORTS = (
     "sgq_packed_sizes", "sgq_pack", "sgq_select", "sgq_gemv_workspace_bytes", "sgq_gemv",
     "sgq_gemv_thresh", "sgq_gemv_dense", "sgq_glu", "sgq_status_string", "sgq_last_cuda_error",
-    "sgq_layout_version",
+    "sgq_layout_version", "sgq_gemv_thresh_noalloc",
 )
 
 
@@ -75,6 +76,7 @@ def _declare(lib):
         "sgq_gemv": ([P, P, I, I, I, P, I, P, P, P, P, P, Z, P, P], I),
         "sgq_gemv_thresh": ([P, P, I, I, I, P, F, P, P, P, Z, P, P], I),
         "sgq_gemv_dense": ([P, P, I, I, I, P, I, P, P, P, Z, P, P], I),
+        "sgq_gemv_thresh_noalloc": ([P, P, I, I, I, P, F, P, P, P, P], I),
         "sgq_glu": ([P, P, P, I, I, I, P], I),
         "sgq_status_string": ([I], ctypes.c_char_p),
         "sgq_last_cuda_error": ([], I),
@@ -145,6 +147,14 @@ def sgq_gemv_thresh(qweight, sz, N, K, group, x, t, y, y_f32, workspace, status=
         _ptr(qweight), _ptr(sz), N, K, group, _ptr(x), float(t), _ptr(y), _ptr(y_f32),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status),
         _stream(stream)))
+
+
+def sgq_gemv_thresh_noalloc(qweight, sz, N, K, group, x, t, y, y_f32, status=None, stream=None):
+    """sgq_gemv_thresh with the library's fixed scratch instead of a workspace
+    (for callers that cannot allocate); N <= SGQ_NOALLOC_MAX_N."""
+    _check("sgq_gemv_thresh_noalloc", load().sgq_gemv_thresh_noalloc(
+        _ptr(qweight), _ptr(sz), N, K, group, _ptr(x), float(t), _ptr(y), _ptr(y_f32),
+        _ptr(status), _stream(stream)))
 
 
 def sgq_gemv_dense(qweight, sz, N, K, group, x, B, y, y_f32, workspace, status=None,

@@ -57,6 +57,7 @@ extern "C" {
 #define SGQ_ERR_ACT        -7  /* unknown activation                             */
 #define SGQ_ERR_CUDA       -8  /* a CUDA runtime call or launch failed           */
 #define SGQ_ERR_DEVICE     -9  /* current device is not compute capability 10.x  */
+#define SGQ_ERR_TOO_LARGE -10  /* N above SGQ_NOALLOC_MAX_N (no-allocation entry)  */
 
 /* Device status bits (OR-ed into the optional `status` word). */
 #define SGQ_STATUS_NONFINITE_W  1  /* sgq_pack: W holds NaN or Inf (that group packed as zeros) */
@@ -169,6 +170,25 @@ int sgq_gemv_dense(const void *qweight, const void *sz, int N, int K, int group,
  * Requires (B * I) % 8 == 0.
  */
 int sgq_glu(const void *gate, const void *up, void *h, int B, int I, int act, void *stream);
+
+/*
+ * sgq_gemv_thresh without a workspace argument, for callers that cannot
+ * allocate device memory (no cudaMalloc available to them, or none allowed
+ * during the call). The pages have no counterpart of this entry point; it is a
+ * deployment convenience of this library.
+ *
+ * The split-K scratch is a fixed array of SGQ_NOALLOC_MAX_N floats compiled
+ * into the library (held on every GPU that loads it until the process exits).
+ * N > SGQ_NOALLOC_MAX_N returns SGQ_ERR_TOO_LARGE. The first call on a device
+ * looks up the array's device address and clears it (synchronously), so make
+ * that first call before any stream capture. Every call leaves the array at
+ * zero again; calls that overlap on the GPU share the array and race. Nothing
+ * is allocated or freed. Other arguments as sgq_gemv_thresh.
+ */
+#define SGQ_NOALLOC_MAX_N 65536
+int sgq_gemv_thresh_noalloc(const void *qweight, const void *sz, int N, int K, int group,
+                            const void *x, float t, void *y, float *y_f32, int32_t *status,
+                            void *stream);
 
 /* Text for a return code (static string). */
 const char *sgq_status_string(int code);
