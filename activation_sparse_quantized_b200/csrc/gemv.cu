@@ -193,20 +193,39 @@ __global__ void __launch_bounds__(256) finalize_kernel(GemvProblem p)
 
 constexpr int kWarps1 = 8;
 constexpr int kThreads1 = kWarps1 * 32;
-constexpr int kStages1 = 24; // rows in flight per warp
+constexpr int kStages1 = 32; // rows in flight per warp (power of two)
+
+// Accumulator pairs of a lane (32 outputs = 4 packed words w0..w3): an LDS.128
+// leaves (w0, w1) and (w2, w3) in aligned register pairs, so one 64-bit AND
+// takes code j of two words at once. Pair m (0..15) holds outputs
+// (16 (m / 8) + m % 8, 16 (m / 8) + m % 8 + 8) of the lane; both of its codes
+// sit at the same bit offset p(m % 8) of their register.
+__host__ __device__ constexpr int pair_pos(int j)
+{
+    return (j < 5) ? 4 * j : 4 * j - 12; // codes 5..7 come from word >> 12
+}
+
+__host__ __device__ constexpr int pair_out(int m, int h)
+{
+    return 16 * (m / 8) + (m % 8) + 8 * h; // output of half h (0, 1) of pair m
+}
 
 struct Smem1 {
-    size_t ring, szs, ridx, rx, scan, total;
+    size_t ring, szs, rx2, ridx, rx, scan, total;
 };
 
-// Each warp's ring region (kStages1 * 512 B = 12 KB) holds, once the warp has
-// consumed all of its rows, its partial tile (1024 floats = 4 KB).
+// ring: each warp's kStages1 rows of 512 B (16 KB), which also holds the warp's
+// partial tile once the warp is done. szs: the (s, z) fp16 pairs of the staged
+// groups, 1024 words per group, lane l's 8 chunks of 4 words swizzled as
+// part_chunk(l, c). rx2: x' = x 2^S of each row duplicated as an (x', x')
+// pair. ridx: the CTA's rows (channels). rx: x of each row.
 __host__ __device__ inline Smem1 smem1_layout(int span_cap, int rows_cap)
 {
     Smem1 s;
     s.ring = 0;
     s.szs = s.ring + (size_t)kWarps1 * kStages1 * kRowBytes1;
-    s.ridx = s.szs + (size_t)span_cap * kTileN1 * 4;
+    s.rx2 = s.szs + (size_t)span_cap * kTileN1 * 4;
+    s.ridx = s.rx2 + (size_t)rows_cap * 8;
     s.rx = s.ridx + (size_t)rows_cap * 4;
     s.scan = s.rx + (size_t)rows_cap * 4;
     s.total = s.scan + (size_t)((rows_cap + 31) / 32 + 4) * 4;
@@ -241,46 +260,46 @@ __device__ __forceinline__ uint64_t ffma2p(uint64_t a, uint64_t b, uint64_t c)
     return d;
 }
 
-// One packed 32-bit word (codes of 8 consecutive outputs) times x' into the
-// four pair accumulators of those outputs. Each code is isolated with one AND;
-// the masked register read as fp32 is the subnormal q * 2^(p - 149), exact.
-// Codes 5..7 are taken from word >> 12, so every code sits at bit offset
-// p in {0, 4, 8, 12, 16}: pairs (0,4) (8,12) (16,8) (12,16).
-__device__ __forceinline__ void mac_word(uint32_t w, uint64_t xb, uint64_t &a0, uint64_t &a1,
-                                         uint64_t &a2, uint64_t &a3)
+// Two packed words (codes of outputs 16t .. 16t + 15 of the lane) times x'
+// into the 8 pair accumulators a[0..7]. A masked register read as fp32 is the
+// subnormal q * 2^(p - 149): exact, one AND per code (the logic pipe is the
+// busy one, so word >> 12 is taken as mul.hi(word, 2^20) on the FMA pipe).
+__device__ __forceinline__ void mac_2words(uint32_t w0, uint32_t w1, uint64_t xb, uint64_t *a)
 {
     asm("{\n\t"
-        ".reg .b32 h, c0, c1, c2, c3, c4, c5, c6, c7;\n\t"
-        ".reg .b64 p0, p1, p2, p3;\n\t"
-        "shr.b32 h, %4, 12;\n\t"
-        "and.b32 c0, %4, 0x0000000F;\n\t"
-        "and.b32 c1, %4, 0x000000F0;\n\t"
-        "and.b32 c2, %4, 0x00000F00;\n\t"
-        "and.b32 c3, %4, 0x0000F000;\n\t"
-        "and.b32 c4, %4, 0x000F0000;\n\t"
-        "and.b32 c5, h, 0x00000F00;\n\t"
-        "and.b32 c6, h, 0x0000F000;\n\t"
-        "and.b32 c7, h, 0x000F0000;\n\t"
-        "mov.b64 p0, {c0, c1};\n\t"
-        "mov.b64 p1, {c2, c3};\n\t"
-        "mov.b64 p2, {c4, c5};\n\t"
-        "mov.b64 p3, {c6, c7};\n\t"
-        "fma.rn.f32x2 %0, p0, %5, %0;\n\t"
-        "fma.rn.f32x2 %1, p1, %5, %1;\n\t"
-        "fma.rn.f32x2 %2, p2, %5, %2;\n\t"
-        "fma.rn.f32x2 %3, p3, %5, %3;\n\t"
+        ".reg .b64 w, h, p;\n\t"
+        ".reg .b32 h0, h1;\n\t"
+        "mov.b64 w, {%8, %9};\n\t"
+        "mul.hi.u32 h0, %8, 1048576;\n\t"
+        "mul.hi.u32 h1, %9, 1048576;\n\t"
+        "mov.b64 h, {h0, h1};\n\t"
+        "and.b64 p, w, 0x0000000F0000000F;\n\t"
+        "fma.rn.f32x2 %0, p, %10, %0;\n\t"
+        "and.b64 p, w, 0x000000F0000000F0;\n\t"
+        "fma.rn.f32x2 %1, p, %10, %1;\n\t"
+        "and.b64 p, w, 0x00000F0000000F00;\n\t"
+        "fma.rn.f32x2 %2, p, %10, %2;\n\t"
+        "and.b64 p, w, 0x0000F0000000F000;\n\t"
+        "fma.rn.f32x2 %3, p, %10, %3;\n\t"
+        "and.b64 p, w, 0x000F0000000F0000;\n\t"
+        "fma.rn.f32x2 %4, p, %10, %4;\n\t"
+        "and.b64 p, h, 0x00000F0000000F00;\n\t"
+        "fma.rn.f32x2 %5, p, %10, %5;\n\t"
+        "and.b64 p, h, 0x0000F0000000F000;\n\t"
+        "fma.rn.f32x2 %6, p, %10, %6;\n\t"
+        "and.b64 p, h, 0x000F0000000F0000;\n\t"
+        "fma.rn.f32x2 %7, p, %10, %7;\n\t"
         "}"
-        : "+l"(a0), "+l"(a1), "+l"(a2), "+l"(a3)
-        : "r"(w), "l"(xb));
+        : "+l"(a[0]), "+l"(a[1]), "+l"(a[2]), "+l"(a[3]), "+l"(a[4]), "+l"(a[5]), "+l"(a[6]),
+          "+l"(a[7])
+        : "r"(w0), "r"(w1), "l"(xb));
 }
 
-// 2^(85 - p) for the two codes of pair m % 4 (see mac_word): turns
-// sum q x' 2^(p - 149) into 2^-64 sum q x'.
-__device__ __forceinline__ uint64_t fold_scale(int m4)
+// One row (16 bytes = 4 words of this lane) into the 16 pair accumulators.
+__device__ __forceinline__ void mac_row(const uint4 &v, uint64_t xb, uint64_t *accg)
 {
-    const int p0 = (m4 == 0) ? 0 : (m4 == 1) ? 8 : (m4 == 2) ? 16 : 12;
-    const int p1 = (m4 == 0) ? 4 : (m4 == 1) ? 12 : (m4 == 2) ? 8 : 16;
-    return pack2(pow2f(85 - p0), pow2f(85 - p1));
+    mac_2words(v.x, v.y, xb, accg);
+    mac_2words(v.z, v.w, xb, accg + 8);
 }
 
 __device__ __forceinline__ float half_lo(uint32_t w)
@@ -309,9 +328,10 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
     const GemvProblem &p = kp.p;
     const Smem1 L = smem1_layout(kp.span_cap, kp.rows_cap);
     uint8_t *ring = smem + L.ring;
-    const uint32_t *szs = reinterpret_cast<const uint32_t *>(smem + L.szs);
+    const uint4 *szs = reinterpret_cast<const uint4 *>(smem + L.szs);
     int32_t *ridx = reinterpret_cast<int32_t *>(smem + L.ridx);
     float *rx = reinterpret_cast<float *>(smem + L.rx);
+    uint64_t *rx2 = reinterpret_cast<uint64_t *>(smem + L.rx2);
     int *scan = reinterpret_cast<int *>(smem + L.scan);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -324,16 +344,17 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
 
     grid_launch_dependents();
 
-    // Scale/zero staging. With a fixed channel slice (threshold / dense) the
-    // groups are known now and are fetched before waiting on the previous
-    // kernel; with an index list they follow the list.
+    // Scale/zero of the CTA's groups, staged asynchronously (the oldest
+    // cp.async group of every thread). With a fixed channel slice (threshold /
+    // dense) the groups are known now, so the copies start before waiting on
+    // the previous kernel; with an index list they follow the list.
     int G0 = 0, span = 0;
     auto stage_sz = [&]() {
         for (int c = tid; c < span * (kTileN1 / 4); c += kThreads1) {
-            const int r = c / (kTileN1 / 4), o = (c % (kTileN1 / 4)) * 4;
-            if (n0 + o < p.N)
-                cp_async16(smem + L.szs + ((size_t)r * kTileN1 + o) * 4,
-                           p.sz + (size_t)(G0 + r) * p.N + n0 + o);
+            const int g = c >> 8, q = c & 255; // q: chunk of 4 outputs in the tile
+            if (n0 + 4 * q < p.N)
+                cp_async16(smem + L.szs + ((size_t)g * 256 + part_chunk(q >> 3, q & 7)) * 16,
+                           p.sz + (size_t)(G0 + g) * p.N + n0 + 4 * q);
         }
         cp_async_commit();
     };
@@ -354,7 +375,8 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
 
     grid_dependency_wait(); // x, idx, count may come from the previous kernel
 
-    const int nr = build_rows<SRC, kThreads1>(kp, split, ridx, rx, scan);
+    // Rows; invalid list entries become row 0 with x = 0 (below).
+    const int nr = build_rows<SRC, kThreads1>(kp, split, ridx, rx, scan); // ends with a barrier
 
     if (SRC == ROWS_LIST) {
         if (nr > 0) {
@@ -362,15 +384,14 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
             G0 = kf >> lg;
             span = min(max((kl >> lg) - G0 + 1, 1), kp.span_cap);
         }
-        stage_sz();
+        stage_sz(); // stays the oldest cp.async group
     }
 
     // This warp's contiguous slice of the CTA's rows.
     const int wa = (int)((long long)nr * warp / kWarps1);
     const int n = (int)((long long)nr * (warp + 1) / kWarps1) - wa;
 
-    // Ring prologue. Lanes past N read column 0 (valid memory, result unused);
-    // invalid rows read row 0 and have x = 0.
+    // Ring prologue. Lanes past N read column 0 (valid memory, result unused).
     const uint8_t *wcol = p.qweight + (lane_ok ? ((size_t)n0 / 2 + lane * 16) : 0);
     uint8_t *myring = ring + (size_t)warp * kStages1 * kRowBytes1 + lane * 16;
 #pragma unroll
@@ -380,15 +401,21 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
         cp_async_commit();
     }
 
-    // x of this warp's rows, scaled by 2^S so that every product
-    // q * x' * 2^(p-149) is a normal fp32 (exact); |x'| < 2^91.
+    // x of this warp's rows (list / dense paths, after the weights are in
+    // flight), and the rows made >= 0 (an invalid list entry reads row 0 with
+    // x = 0).
     if (SRC != ROWS_THRESH) {
         for (int j = lane; j < n; j += 32) {
             const int k = ridx[wa + j];
             rx[wa + j] = (k >= 0) ? bf16_bits_to_float(__ldg(p.x + k)) : 0.f;
+            ridx[wa + j] = max(k, 0);
         }
         __syncwarp();
     }
+
+    // Scale x by 2^S so that every product q * x' * 2^(p-149) is a normal fp32
+    // (exact); |x'| < 2^91. Stored as (x', x') pairs, the b operand of the
+    // packed FMAs.
     float m = 0.f;
     for (int j = lane; j < n; j += 32)
         m = fmaxf(m, fabsf(rx[wa + j]));
@@ -396,10 +423,16 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
     const int S = (e == INT32_MIN) ? 0 : 90 - e;
     {
         const float fa = pow2f(S - S / 2), fb = pow2f(S / 2);
-        for (int j = lane; j < n; j += 32)
-            rx[wa + j] = (rx[wa + j] * fa) * fb;
+        for (int j = lane; j < n; j += 32) {
+            const float xs = (rx[wa + j] * fa) * fb;
+            rx2[wa + j] = pack2(xs, xs);
+        }
     }
     __syncwarp();
+    // The staged scale/zero (every thread's oldest cp.async group) have landed
+    // and are visible to every warp before the first fold.
+    cp_async_wait<kStages1>();
+    __syncthreads();
 
     // Pair accumulators: accg = this group's sum of q x' 2^(p-149);
     // acc = folded result in units of 2^(S-64).
@@ -409,97 +442,98 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
         accg[m2] = 0ull;
         acc[m2] = 0ull;
     }
-    float Xg = 0.f;
-    int curG = (n > 0) ? (max(ridx[wa], 0) >> lg) : 0;
 
     //   acc += s * (2^(85-p) accg - z * 2^-64 sum x')
-    auto fold = [&](int G) {
-        const bool staged = (G >= G0) && (G < G0 + span);
-        const uint32_t *src = staged ? (szs + (size_t)(G - G0) * kTileN1 + lane * 32)
-                                     : (p.sz + (size_t)G * p.N + n0 + (lane_ok ? lane * 32 : 0));
+    auto fold = [&](int G, float Xg) {
         const float nx = -Xg * pow2f(-64);
         const uint64_t nx2 = pack2(nx, nx);
+        const bool staged = (G >= G0) && (G < G0 + span);
+        uint32_t w[32]; // (s, z) of this lane's 32 outputs
+        if (staged) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const uint4 w4 = staged ? *reinterpret_cast<const uint4 *>(src + 4 * c)
-                                    : __ldg(reinterpret_cast<const uint4 *>(src + 4 * c));
+            for (int c = 0; c < 8; ++c) {
+                const uint4 v = szs[(G - G0) * 256 + part_chunk(lane, c)];
+                w[4 * c] = v.x;
+                w[4 * c + 1] = v.y;
+                w[4 * c + 2] = v.z;
+                w[4 * c + 3] = v.w;
+            }
+        } else {
+            const uint4 *g4 = reinterpret_cast<const uint4 *>(
+                p.sz + (size_t)G * p.N + n0 + (lane_ok ? lane * 32 : 0));
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int m2 = 2 * c + h;
-                const uint32_t wa0 = h ? w4.z : w4.x, wa1 = h ? w4.w : w4.y;
-                uint64_t t = fmul2(accg[m2], fold_scale(m2 & 3));
-                t = ffma2p(pack2(half_hi(wa0), half_hi(wa1)), nx2, t);
-                acc[m2] = ffma2p(pack2(half_lo(wa0), half_lo(wa1)), t, acc[m2]);
-                accg[m2] = 0ull;
+            for (int c = 0; c < 8; ++c) {
+                const uint4 v = __ldg(g4 + c);
+                w[4 * c] = v.x;
+                w[4 * c + 1] = v.y;
+                w[4 * c + 2] = v.z;
+                w[4 * c + 3] = v.w;
             }
         }
-        Xg = 0.f;
+#pragma unroll
+        for (int m2 = 0; m2 < 16; ++m2) {
+            const uint32_t a = w[pair_out(m2, 0)], b = w[pair_out(m2, 1)];
+            const float c = pow2f(85 - pair_pos(m2 & 7));
+            uint64_t t = fmul2(accg[m2], pack2(c, c));
+            t = ffma2p(pack2(half_hi(a), half_hi(b)), nx2, t);
+            acc[m2] = ffma2p(pack2(half_lo(a), half_lo(b)), t, acc[m2]);
+            accg[m2] = 0ull;
+        }
     };
 
-    // The staged scale/zero (the oldest cp.async group) must be complete and
-    // visible to every warp before the first fold.
-    cp_async_wait<kStages1>();
-    __syncthreads();
+    // Runs of rows of one group: the run end comes from one ballot per 32
+    // rows, and sum x' of the run from one warp reduction, so the per-row work
+    // is the ring read, the codes and the refill only.
+    int i = 0;
+    while (i < n) {
+        const int G = ridx[wa + i] >> lg;
+        int i1 = i;
+        float Xg = 0.f;
+        for (;;) {
+            const int j = i1 + lane;
+            const bool in = (j < n) && ((ridx[wa + j] >> lg) == G);
+            const uint32_t bal = __ballot_sync(0xffffffffu, in);
+            const int len = (bal == 0xffffffffu) ? 32 : (__ffs(~bal) - 1);
+            if (lane < len)
+                Xg += unpack2(rx2[wa + j]).x;
+            i1 += len;
+            if (len < 32)
+                break;
+        }
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1)
+            Xg += __shfl_xor_sync(0xffffffffu, Xg, d);
 
-    // Two rows per iteration (more independent work per warp); a group change
-    // between the two takes the slower path that folds in between.
-    int i = 0, slot = 0;
-    for (; i + 1 < n; i += 2) {
-        cp_async_wait<kStages1 - 2>(); // rows i and i + 1 have landed
-        const int slot1 = (slot + 1 == kStages1) ? 0 : slot + 1;
-        const uint4 v0 = *reinterpret_cast<const uint4 *>(myring + slot * kRowBytes1);
-        const uint4 v1 = *reinterpret_cast<const uint4 *>(myring + slot1 * kRowBytes1);
-        const int G0r = max(ridx[wa + i], 0) >> lg;
-        const int G1r = max(ridx[wa + i + 1], 0) >> lg;
-        const float x0 = rx[wa + i], x1 = rx[wa + i + 1];
-        if (G0r != curG) {
-            fold(curG);
-            curG = G0r;
+        for (; i + 1 < i1; i += 2) {
+            cp_async_wait<kStages1 - 2>(); // rows i and i + 1 have landed
+            const int slot = i & (kStages1 - 1), slot1 = (i + 1) & (kStages1 - 1);
+            const uint4 v0 = *reinterpret_cast<const uint4 *>(myring + slot * kRowBytes1);
+            const uint4 v1 = *reinterpret_cast<const uint4 *>(myring + slot1 * kRowBytes1);
+            mac_row(v0, rx2[wa + i], accg);
+            mac_row(v1, rx2[wa + i + 1], accg);
+            if (i + kStages1 < n)
+                cp_async16(myring + slot * kRowBytes1,
+                           wcol + (size_t)ridx[wa + i + kStages1] * row_stride);
+            cp_async_commit();
+            if (i + 1 + kStages1 < n)
+                cp_async16(myring + slot1 * kRowBytes1,
+                           wcol + (size_t)ridx[wa + i + 1 + kStages1] * row_stride);
+            cp_async_commit();
         }
-        const uint64_t xb0 = pack2(x0, x0);
-        mac_word(v0.x, xb0, accg[0], accg[1], accg[2], accg[3]);
-        mac_word(v0.y, xb0, accg[4], accg[5], accg[6], accg[7]);
-        mac_word(v0.z, xb0, accg[8], accg[9], accg[10], accg[11]);
-        mac_word(v0.w, xb0, accg[12], accg[13], accg[14], accg[15]);
-        Xg += x0;
-        if (G1r != curG) {
-            fold(curG);
-            curG = G1r;
+        if (i < i1) {
+            // The last row of an odd-length run.
+            cp_async_wait<kStages1 - 1>();
+            const int slot = i & (kStages1 - 1);
+            const uint4 v = *reinterpret_cast<const uint4 *>(myring + slot * kRowBytes1);
+            mac_row(v, rx2[wa + i], accg);
+            if (i + kStages1 < n)
+                cp_async16(myring + slot * kRowBytes1,
+                           wcol + (size_t)ridx[wa + i + kStages1] * row_stride);
+            cp_async_commit();
+            ++i;
         }
-        const uint64_t xb1 = pack2(x1, x1);
-        mac_word(v1.x, xb1, accg[0], accg[1], accg[2], accg[3]);
-        mac_word(v1.y, xb1, accg[4], accg[5], accg[6], accg[7]);
-        mac_word(v1.z, xb1, accg[8], accg[9], accg[10], accg[11]);
-        mac_word(v1.w, xb1, accg[12], accg[13], accg[14], accg[15]);
-        Xg += x1;
-        if (i + kStages1 < n)
-            cp_async16(myring + slot * kRowBytes1,
-                       wcol + (size_t)max(ridx[wa + i + kStages1], 0) * row_stride);
-        cp_async_commit();
-        if (i + 1 + kStages1 < n)
-            cp_async16(myring + slot1 * kRowBytes1,
-                       wcol + (size_t)max(ridx[wa + i + 1 + kStages1], 0) * row_stride);
-        cp_async_commit();
-        slot = (slot1 + 1 == kStages1) ? 0 : slot1 + 1;
+        fold(G, Xg);
     }
-    if (i < n) {
-        cp_async_wait<kStages1 - 1>();
-        const uint4 v = *reinterpret_cast<const uint4 *>(myring + slot * kRowBytes1);
-        const int G = max(ridx[wa + i], 0) >> lg;
-        const float xs = rx[wa + i];
-        if (G != curG) {
-            fold(curG);
-            curG = G;
-        }
-        const uint64_t xb = pack2(xs, xs);
-        mac_word(v.x, xb, accg[0], accg[1], accg[2], accg[3]);
-        mac_word(v.y, xb, accg[4], accg[5], accg[6], accg[7]);
-        mac_word(v.z, xb, accg[8], accg[9], accg[10], accg[11]);
-        mac_word(v.w, xb, accg[12], accg[13], accg[14], accg[15]);
-        Xg += xs;
-    }
-    if (n > 0)
-        fold(curG);
 
     // This warp's partial tile, in real units (x 2^(64-S), two exact
     // factors), into its own ring region: every cp.async of this warp has
@@ -509,16 +543,20 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
     {
         float4 *part = reinterpret_cast<float4 *>(ring + (size_t)warp * kStages1 * kRowBytes1);
         const int E = 64 - S;
-        const uint64_t f1 = pack2(pow2f(E / 2), pow2f(E / 2));
-        const uint64_t f2 = pack2(pow2f(E - E / 2), pow2f(E - E / 2));
+        const float f1 = pow2f(E / 2), f2 = pow2f(E - E / 2);
         const bool live = lane_ok && n > 0;
+        float out[32];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const float2 lo = unpack2(fmul2(fmul2(acc[2 * c], f1), f2));
-            const float2 hi = unpack2(fmul2(fmul2(acc[2 * c + 1], f1), f2));
-            part[part_chunk(lane, c)] =
-                live ? make_float4(lo.x, lo.y, hi.x, hi.y) : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int m2 = 0; m2 < 16; ++m2) {
+            const float2 v = unpack2(acc[m2]);
+            out[pair_out(m2, 0)] = (v.x * f1) * f2;
+            out[pair_out(m2, 1)] = (v.y * f1) * f2;
         }
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+            part[part_chunk(lane, c)] = live ? make_float4(out[4 * c], out[4 * c + 1],
+                                                           out[4 * c + 2], out[4 * c + 3])
+                                             : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();
     if (tid < kTileN1 / 4) {
