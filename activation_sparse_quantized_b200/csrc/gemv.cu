@@ -193,7 +193,7 @@ __global__ void __launch_bounds__(256) finalize_kernel(GemvProblem p)
 
 constexpr int kWarps1 = 8;
 constexpr int kThreads1 = kWarps1 * 32;
-constexpr int kStages1 = 32; // rows in flight per warp (power of two)
+constexpr int kStages1 = 8; // rows in flight per warp (power of two); deeper rings measured slower
 
 // Accumulator pairs of a lane (32 outputs = 4 packed words w0..w3): an LDS.128
 // leaves (w0, w1) and (w2, w3) in aligned register pairs, so one 64-bit AND
@@ -214,7 +214,7 @@ struct Smem1 {
     size_t ring, szs, rx2, ridx, rx, scan, total;
 };
 
-// ring: each warp's kStages1 rows of 512 B (16 KB), which also holds the warp's
+// ring: each warp's kStages1 rows of 512 B (4 KB), which also holds the warp's
 // partial tile once the warp is done. szs: the (s, z) fp16 pairs of the staged
 // groups, 1024 words per group, lane l's 8 chunks of 4 words swizzled as
 // part_chunk(l, c). rx2: x' = x 2^S of each row duplicated as an (x', x')
