@@ -195,111 +195,77 @@ constexpr int kWarps1 = 8;
 constexpr int kThreads1 = kWarps1 * 32;
 constexpr int kStages1 = 8; // rows in flight per warp (power of two); deeper rings measured slower
 
-// Accumulator pairs of a lane (32 outputs = 4 packed words w0..w3): an LDS.128
-// leaves (w0, w1) and (w2, w3) in aligned register pairs, so one 64-bit AND
-// takes code j of two words at once. Pair m (0..15) holds outputs
-// (16 (m / 8) + m % 8, 16 (m / 8) + m % 8 + 8) of the lane; both of its codes
-// sit at the same bit offset p(m % 8) of their register.
-__host__ __device__ constexpr int pair_pos(int j)
+// Output o (0..31) of a lane is code o % 8 of packed word o / 8. One 32-bit AND
+// takes two codes of a word at once, one into each fp16 half: the masked half
+// reads as the fp16 subnormal q * 2^-24 (codes 0, 2, 4, 6 of the word, the
+// latter two after word >> 8) or q * 2^-20 (codes 1, 3, 5, 7, taken from bits
+// 4..7 of the half). A mixed-precision FMA (fp16 operands, fp32 accumulator)
+// multiplies it by x' in fp16: the product is exact and normal in fp32.
+__host__ __device__ constexpr int code_shift(int o)
 {
-    return (j < 5) ? 4 * j : 4 * j - 12; // codes 5..7 come from word >> 12
-}
-
-__host__ __device__ constexpr int pair_out(int m, int h)
-{
-    return 16 * (m / 8) + (m % 8) + 8 * h; // output of half h (0, 1) of pair m
+    return (o & 1) ? 20 : 24; // accumulator of output o holds sum q x' 2^-code_shift
 }
 
 struct Smem1 {
-    size_t ring, szs, rx2, ridx, rx, scan, total;
+    size_t ring, szs, rxh, ridx, rx, scan, total;
 };
 
 // ring: each warp's kStages1 rows of 512 B (4 KB), which also holds the warp's
 // partial tile once the warp is done. szs: the (s, z) fp16 pairs of the staged
 // groups, 1024 words per group, lane l's 8 chunks of 4 words swizzled as
-// part_chunk(l, c). rx2: x' = x 2^S of each row duplicated as an (x', x')
-// pair. ridx: the CTA's rows (channels). rx: x of each row.
+// part_chunk(l, c). ridx: the CTA's rows (channels). rx: x of each row. rxh:
+// x' = x 2^S of each row as fp16.
 __host__ __device__ inline Smem1 smem1_layout(int span_cap, int rows_cap)
 {
     Smem1 s;
     s.ring = 0;
     s.szs = s.ring + (size_t)kWarps1 * kStages1 * kRowBytes1;
-    s.rx2 = s.szs + (size_t)span_cap * kTileN1 * 4;
-    s.ridx = s.rx2 + (size_t)rows_cap * 8;
+    s.ridx = s.szs + (size_t)span_cap * kTileN1 * 4;
     s.rx = s.ridx + (size_t)rows_cap * 4;
     s.scan = s.rx + (size_t)rows_cap * 4;
-    s.total = s.scan + (size_t)((rows_cap + 31) / 32 + 4) * 4;
+    s.rxh = s.scan + (size_t)((rows_cap + 31) / 32 + 4) * 4;
+    s.total = s.rxh + ((size_t)rows_cap * 2 + 15) / 16 * 16;
     return s;
 }
 
-__device__ __forceinline__ uint64_t pack2(float lo, float hi)
-{
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-
-__device__ __forceinline__ float2 unpack2(uint64_t v)
-{
-    float2 r;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
-    return r;
-}
-
-__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b)
-{
-    uint64_t d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-
-__device__ __forceinline__ uint64_t ffma2p(uint64_t a, uint64_t b, uint64_t c)
-{
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-
-// Two packed words (codes of outputs 16t .. 16t + 15 of the lane) times x'
-// into the 8 pair accumulators a[0..7]. A masked register read as fp32 is the
-// subnormal q * 2^(p - 149): exact, one AND per code (the logic pipe is the
-// busy one, so word >> 12 is taken as mul.hi(word, 2^20) on the FMA pipe).
-__device__ __forceinline__ void mac_2words(uint32_t w0, uint32_t w1, uint64_t xb, uint64_t *a)
+// One packed word (codes of outputs 8t .. 8t + 7 of the lane) times x' into
+// a[0..7]: word >> 8 by mul.hi on the FMA pipe, four ANDs on the logic pipe,
+// eight mixed-precision FMAs.
+__device__ __forceinline__ void mac_word(uint32_t w, uint16_t xh, float *a)
 {
     asm("{\n\t"
-        ".reg .b64 w, h, p;\n\t"
-        ".reg .b32 h0, h1;\n\t"
-        "mov.b64 w, {%8, %9};\n\t"
-        "mul.hi.u32 h0, %8, 1048576;\n\t"
-        "mul.hi.u32 h1, %9, 1048576;\n\t"
-        "mov.b64 h, {h0, h1};\n\t"
-        "and.b64 p, w, 0x0000000F0000000F;\n\t"
-        "fma.rn.f32x2 %0, p, %10, %0;\n\t"
-        "and.b64 p, w, 0x000000F0000000F0;\n\t"
-        "fma.rn.f32x2 %1, p, %10, %1;\n\t"
-        "and.b64 p, w, 0x00000F0000000F00;\n\t"
-        "fma.rn.f32x2 %2, p, %10, %2;\n\t"
-        "and.b64 p, w, 0x0000F0000000F000;\n\t"
-        "fma.rn.f32x2 %3, p, %10, %3;\n\t"
-        "and.b64 p, w, 0x000F0000000F0000;\n\t"
-        "fma.rn.f32x2 %4, p, %10, %4;\n\t"
-        "and.b64 p, h, 0x00000F0000000F00;\n\t"
-        "fma.rn.f32x2 %5, p, %10, %5;\n\t"
-        "and.b64 p, h, 0x0000F0000000F000;\n\t"
-        "fma.rn.f32x2 %6, p, %10, %6;\n\t"
-        "and.b64 p, h, 0x000F0000000F0000;\n\t"
-        "fma.rn.f32x2 %7, p, %10, %7;\n\t"
+        ".reg .b32 h, p;\n\t"
+        ".reg .f16 lo, hi;\n\t"
+        "mul.hi.u32 h, %8, 16777216;\n\t"
+        "and.b32 p, %8, 0x000F000F;\n\t"
+        "mov.b32 {lo, hi}, p;\n\t"
+        "fma.rn.f32.f16 %0, lo, %9, %0;\n\t"
+        "fma.rn.f32.f16 %4, hi, %9, %4;\n\t"
+        "and.b32 p, %8, 0x00F000F0;\n\t"
+        "mov.b32 {lo, hi}, p;\n\t"
+        "fma.rn.f32.f16 %1, lo, %9, %1;\n\t"
+        "fma.rn.f32.f16 %5, hi, %9, %5;\n\t"
+        "and.b32 p, h, 0x000F000F;\n\t"
+        "mov.b32 {lo, hi}, p;\n\t"
+        "fma.rn.f32.f16 %2, lo, %9, %2;\n\t"
+        "fma.rn.f32.f16 %6, hi, %9, %6;\n\t"
+        "and.b32 p, h, 0x00F000F0;\n\t"
+        "mov.b32 {lo, hi}, p;\n\t"
+        "fma.rn.f32.f16 %3, lo, %9, %3;\n\t"
+        "fma.rn.f32.f16 %7, hi, %9, %7;\n\t"
         "}"
-        : "+l"(a[0]), "+l"(a[1]), "+l"(a[2]), "+l"(a[3]), "+l"(a[4]), "+l"(a[5]), "+l"(a[6]),
-          "+l"(a[7])
-        : "r"(w0), "r"(w1), "l"(xb));
+        : "+f"(a[0]), "+f"(a[1]), "+f"(a[2]), "+f"(a[3]), "+f"(a[4]), "+f"(a[5]), "+f"(a[6]),
+          "+f"(a[7])
+        : "r"(w), "h"(xh));
 }
 
-// One row (16 bytes = 4 words of this lane) into the 16 pair accumulators.
-__device__ __forceinline__ void mac_row(const uint4 &v, uint64_t xb, uint64_t *accg)
+// One row (16 bytes = 4 words of this lane) into the 32 group accumulators.
+__device__ __forceinline__ void mac_row(const uint4 &v, uint16_t xh, float *accg)
 {
-    mac_2words(v.x, v.y, xb, accg);
-    mac_2words(v.z, v.w, xb, accg + 8);
+    mac_word(v.x, xh, accg);
+    mac_word(v.y, xh, accg + 8);
+    mac_word(v.z, xh, accg + 16);
+    mac_word(v.w, xh, accg + 24);
 }
 
 __device__ __forceinline__ float half_lo(uint32_t w)
@@ -331,7 +297,7 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
     const uint4 *szs = reinterpret_cast<const uint4 *>(smem + L.szs);
     int32_t *ridx = reinterpret_cast<int32_t *>(smem + L.ridx);
     float *rx = reinterpret_cast<float *>(smem + L.rx);
-    uint64_t *rx2 = reinterpret_cast<uint64_t *>(smem + L.rx2);
+    uint16_t *rxh = reinterpret_cast<uint16_t *>(smem + L.rxh);
     int *scan = reinterpret_cast<int *>(smem + L.scan);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -413,20 +379,19 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
         __syncwarp();
     }
 
-    // Scale x by 2^S so that every product q * x' * 2^(p-149) is a normal fp32
-    // (exact); |x'| < 2^91. Stored as (x', x') pairs, the b operand of the
-    // packed FMAs.
+    // x' = x 2^S in fp16 with 2^14 <= max |x'| < 2^15 over the warp's rows:
+    // exact for every |x| >= 2^-28 max |x| (fp16 normals); smaller x round on
+    // the fp16 subnormal grid, an error below 2^-39 max |x'|. Each product
+    // q 2^-24 x' (or q 2^-20 x') is then exact in fp32.
     float m = 0.f;
     for (int j = lane; j < n; j += 32)
         m = fmaxf(m, fabsf(rx[wa + j]));
     const int e = warp_max_exponent(m);
-    const int S = (e == INT32_MIN) ? 0 : 90 - e;
+    const int S = (e == INT32_MIN) ? 0 : 14 - e;
     {
         const float fa = pow2f(S - S / 2), fb = pow2f(S / 2);
-        for (int j = lane; j < n; j += 32) {
-            const float xs = (rx[wa + j] * fa) * fb;
-            rx2[wa + j] = pack2(xs, xs);
-        }
+        for (int j = lane; j < n; j += 32)
+            rxh[wa + j] = __half_as_ushort(__float2half_rn((rx[wa + j] * fa) * fb));
     }
     __syncwarp();
     // The staged scale/zero (every thread's oldest cp.async group) have landed
@@ -434,19 +399,17 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
     cp_async_wait<kStages1>();
     __syncthreads();
 
-    // Pair accumulators: accg = this group's sum of q x' 2^(p-149);
-    // acc = folded result in units of 2^(S-64).
-    uint64_t accg[16], acc[16];
+    // accg[o] = this group's sum of q x' 2^-code_shift(o); acc[o] = folded
+    // result in units of 2^-S.
+    float accg[32], acc[32];
 #pragma unroll
-    for (int m2 = 0; m2 < 16; ++m2) {
-        accg[m2] = 0ull;
-        acc[m2] = 0ull;
+    for (int o = 0; o < 32; ++o) {
+        accg[o] = 0.f;
+        acc[o] = 0.f;
     }
 
-    //   acc += s * (2^(85-p) accg - z * 2^-64 sum x')
+    //   acc += s * (2^code_shift accg - z * sum x')
     auto fold = [&](int G, float Xg) {
-        const float nx = -Xg * pow2f(-64);
-        const uint64_t nx2 = pack2(nx, nx);
         const bool staged = (G >= G0) && (G < G0 + span);
         uint32_t w[32]; // (s, z) of this lane's 32 outputs
         if (staged) {
@@ -471,13 +434,10 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
             }
         }
 #pragma unroll
-        for (int m2 = 0; m2 < 16; ++m2) {
-            const uint32_t a = w[pair_out(m2, 0)], b = w[pair_out(m2, 1)];
-            const float c = pow2f(85 - pair_pos(m2 & 7));
-            uint64_t t = fmul2(accg[m2], pack2(c, c));
-            t = ffma2p(pack2(half_hi(a), half_hi(b)), nx2, t);
-            acc[m2] = ffma2p(pack2(half_lo(a), half_lo(b)), t, acc[m2]);
-            accg[m2] = 0ull;
+        for (int o = 0; o < 32; ++o) {
+            const float t = accg[o] * pow2f(code_shift(o));
+            acc[o] = fmaf(half_lo(w[o]), fmaf(-half_hi(w[o]), Xg, t), acc[o]);
+            accg[o] = 0.f;
         }
     };
 
@@ -495,7 +455,7 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
             const uint32_t bal = __ballot_sync(0xffffffffu, in);
             const int len = (bal == 0xffffffffu) ? 32 : (__ffs(~bal) - 1);
             if (lane < len)
-                Xg += unpack2(rx2[wa + j]).x;
+                Xg += __half2float(__ushort_as_half(rxh[wa + j]));
             i1 += len;
             if (len < 32)
                 break;
@@ -509,8 +469,8 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
             const int slot = i & (kStages1 - 1), slot1 = (i + 1) & (kStages1 - 1);
             const uint4 v0 = *reinterpret_cast<const uint4 *>(myring + slot * kRowBytes1);
             const uint4 v1 = *reinterpret_cast<const uint4 *>(myring + slot1 * kRowBytes1);
-            mac_row(v0, rx2[wa + i], accg);
-            mac_row(v1, rx2[wa + i + 1], accg);
+            mac_row(v0, rxh[wa + i], accg);
+            mac_row(v1, rxh[wa + i + 1], accg);
             if (i + kStages1 < n)
                 cp_async16(myring + slot * kRowBytes1,
                            wcol + (size_t)ridx[wa + i + kStages1] * row_stride);
@@ -525,7 +485,7 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
             cp_async_wait<kStages1 - 1>();
             const int slot = i & (kStages1 - 1);
             const uint4 v = *reinterpret_cast<const uint4 *>(myring + slot * kRowBytes1);
-            mac_row(v, rx2[wa + i], accg);
+            mac_row(v, rxh[wa + i], accg);
             if (i + kStages1 < n)
                 cp_async16(myring + slot * kRowBytes1,
                            wcol + (size_t)ridx[wa + i + kStages1] * row_stride);
@@ -535,23 +495,20 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
         fold(G, Xg);
     }
 
-    // This warp's partial tile, in real units (x 2^(64-S), two exact
-    // factors), into its own ring region: every cp.async of this warp has
-    // landed and been read, so nothing else touches that region any more.
+    // This warp's partial tile, in real units (x 2^-S, two exact factors),
+    // into its own ring region: every cp.async of this warp has landed and
+    // been read, so nothing else touches that region any more.
     cp_async_wait_all();
     __syncwarp();
     {
         float4 *part = reinterpret_cast<float4 *>(ring + (size_t)warp * kStages1 * kRowBytes1);
-        const int E = 64 - S;
+        const int E = -S;
         const float f1 = pow2f(E / 2), f2 = pow2f(E - E / 2);
         const bool live = lane_ok && n > 0;
         float out[32];
 #pragma unroll
-        for (int m2 = 0; m2 < 16; ++m2) {
-            const float2 v = unpack2(acc[m2]);
-            out[pair_out(m2, 0)] = (v.x * f1) * f2;
-            out[pair_out(m2, 1)] = (v.y * f1) * f2;
-        }
+        for (int o = 0; o < 32; ++o)
+            out[o] = (acc[o] * f1) * f2;
 #pragma unroll
         for (int c = 0; c < 8; ++c)
             part[part_chunk(lane, c)] = live ? make_float4(out[4 * c], out[4 * c + 1],
