@@ -20,14 +20,15 @@
 //    channel slice, before x is read.
 //  * Each warp takes a contiguous slice of the CTA's rows; every lane streams
 //    its own 16-byte (B = 1) or 4-byte (B > 1) column of each row through a
-//    per-lane ring in shared memory with cp.async, up to 16 rows ahead. A lane
-//    reads back only bytes it copied itself: no barrier, only its own groups.
+//    per-lane ring in shared memory with cp.async (8 rows ahead for B = 1). A
+//    lane reads back only bytes it copied itself: no barrier, only its own
+//    groups.
 //  * B = 1: codes are summed per group without dequantizing
-//    (sum s (q - z) x = s (sum q x - z sum x)). One AND turns a code into an
-//    fp32 operand (the masked bits read as the subnormal q * 2^(p-149)); pairs
-//    of codes go through one packed f32x2 FMA with x scaled by a per-warp power
-//    of two so every product is exact and normal. Scale and zero are applied
-//    once per (group, output) in a fold.
+//    (sum s (q - z) x = s (sum q x - z sum x)). One 32-bit AND takes two codes
+//    into the two halves of an fp16 pair, where they read as exact fp16
+//    subnormals; a mixed-precision FMA (fp16 x fp16 + fp32) multiplies each by
+//    x held in fp16 under a per-warp power-of-two scale, so every product is
+//    exact. Scale and zero are applied once per (group, output) in a fold.
 //  * B > 1: each code is dequantized exactly (one LOP3, one FMA, one add) and
 //    multiplied into B accumulators with packed f32x2 FMAs.
 //  * Split-K: each warp leaves its partial tile in its own (drained) ring
