@@ -252,6 +252,77 @@ int sgq_gemv_dense(const void *qweight, const void *sz, int N, int K, int group,
     return run_gemv(p, ws_bytes, workspace, stream);
 }
 
+// Fused gate + up + GLU: one GEMV over the stacked [gate; up] weights
+// (N = 2I outputs) whose epilogue writes h = act(gate) * up.
+static int run_gemv_glu(sgq::GemvProblem &p, int I, int act, size_t ws_bytes, void *workspace,
+                        void *stream)
+{
+    if (act != SGQ_ACT_SILU && act != SGQ_ACT_RELU)
+        return SGQ_ERR_ACT;
+    if (I <= 0 || I > (1 << 29))
+        return SGQ_ERR_SHAPE;
+    p.N = 2 * I;
+    p.epilogue = (act == SGQ_ACT_SILU) ? sgq::EPI_GLU_SILU : sgq::EPI_GLU_RELU;
+    return run_gemv(p, ws_bytes, workspace, stream);
+}
+
+int sgq_gemv_glu(const void *qweight, const void *sz, int I, int K, int group, const void *x,
+                 int B, const int32_t *idx, const int32_t *count, int act, void *h,
+                 float *h_f32, void *workspace, size_t ws_bytes, int32_t *status, void *stream)
+{
+    sgq::GemvProblem p{};
+    p.qweight = static_cast<const uint8_t *>(qweight);
+    p.sz = static_cast<const uint32_t *>(sz);
+    p.x = static_cast<const uint16_t *>(x);
+    p.idx = idx;
+    p.count = count;
+    p.y = static_cast<uint16_t *>(h);
+    p.y_f32 = h_f32;
+    p.status = status;
+    p.K = K;
+    p.group = group;
+    p.B = B;
+    p.source = sgq::ROWS_LIST;
+    return run_gemv_glu(p, I, act, ws_bytes, workspace, stream);
+}
+
+int sgq_gemv_glu_thresh(const void *qweight, const void *sz, int I, int K, int group,
+                        const void *x, float t, int act, void *h, float *h_f32, void *workspace,
+                        size_t ws_bytes, int32_t *status, void *stream)
+{
+    sgq::GemvProblem p{};
+    p.qweight = static_cast<const uint8_t *>(qweight);
+    p.sz = static_cast<const uint32_t *>(sz);
+    p.x = static_cast<const uint16_t *>(x);
+    p.y = static_cast<uint16_t *>(h);
+    p.y_f32 = h_f32;
+    p.status = status;
+    p.K = K;
+    p.group = group;
+    p.B = 1;
+    p.t = t;
+    p.source = sgq::ROWS_THRESH;
+    return run_gemv_glu(p, I, act, ws_bytes, workspace, stream);
+}
+
+int sgq_gemv_glu_dense(const void *qweight, const void *sz, int I, int K, int group,
+                       const void *x, int B, int act, void *h, float *h_f32, void *workspace,
+                       size_t ws_bytes, int32_t *status, void *stream)
+{
+    sgq::GemvProblem p{};
+    p.qweight = static_cast<const uint8_t *>(qweight);
+    p.sz = static_cast<const uint32_t *>(sz);
+    p.x = static_cast<const uint16_t *>(x);
+    p.y = static_cast<uint16_t *>(h);
+    p.y_f32 = h_f32;
+    p.status = status;
+    p.K = K;
+    p.group = group;
+    p.B = B;
+    p.source = sgq::ROWS_DENSE;
+    return run_gemv_glu(p, I, act, ws_bytes, workspace, stream);
+}
+
 int sgq_glu(const void *gate, const void *up, void *h, int B, int I, int act, void *stream)
 {
     if (act != SGQ_ACT_SILU && act != SGQ_ACT_RELU)

@@ -168,17 +168,33 @@ __device__ int build_rows(const KParams &kp, int split, int32_t *ridx, float *rx
 // sums to bf16 y, writes the optional fp32 copy and re-zeroes the workspace.
 // Doing this in a kernel of its own keeps memory fences and tickets out of the
 // GEMV's CTAs, which just add their partials and exit.
+//
+// GLU epilogues (the gated FFN fused behind one GEMV over the stacked gate
+// and up weights): output i of row b is act(gate) * up with gate = sum[b][i]
+// and up = sum[b][I + i], I = N / 2, computed from the fp32 sums and rounded
+// once to bf16.
+template <int EPI>
 __global__ void __launch_bounds__(256) finalize_kernel(GemvProblem p)
 {
     grid_launch_dependents();
     grid_dependency_wait();
-    const int quads = p.N / 4;
+    const int width = (EPI == EPI_PLAIN) ? p.N : p.N / 2; // outputs per row
+    const int quads = width / 4;
     for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < p.B * quads;
          e += gridDim.x * blockDim.x) {
-        const size_t o = (size_t)(e / quads) * p.N + (size_t)(e % quads) * 4;
-        float *wp = p.ws_acc + o;
-        const float4 v = ld_cg_v4(wp);
+        const int b = e / quads, i = (e % quads) * 4;
+        float *wp = p.ws_acc + (size_t)b * p.N + i;
+        float4 v = ld_cg_v4(wp);
         st_cg_v4(wp, make_float4(0.f, 0.f, 0.f, 0.f));
+        if (EPI != EPI_PLAIN) {
+            float *wu = wp + width;
+            const float4 u = ld_cg_v4(wu);
+            st_cg_v4(wu, make_float4(0.f, 0.f, 0.f, 0.f));
+            constexpr int ACT = (EPI == EPI_GLU_SILU) ? SGQ_ACT_SILU : SGQ_ACT_RELU;
+            v = make_float4(act_mul<ACT>(v.x, u.x), act_mul<ACT>(v.y, u.y),
+                            act_mul<ACT>(v.z, u.z), act_mul<ACT>(v.w, u.w));
+        }
+        const size_t o = (size_t)b * width + i;
         uint2 yb;
         yb.x = (uint32_t)float_to_bf16_bits(v.x) | ((uint32_t)float_to_bf16_bits(v.y) << 16);
         yb.y = (uint32_t)float_to_bf16_bits(v.z) | ((uint32_t)float_to_bf16_bits(v.w) << 16);
@@ -768,7 +784,14 @@ cudaError_t launch_gemv_and_finalize(Kern kern, int grid, int block, size_t smem
         return err;
     const int quads = kp.p.B * (kp.p.N / 4);
     const int fgrid = std::max(1, std::min(ceil_div(quads, 256), 148));
-    return launch_pdl(finalize_kernel, fgrid, 256, 0, stream, kp.p);
+    switch (kp.p.epilogue) {
+    case EPI_GLU_SILU:
+        return launch_pdl(finalize_kernel<EPI_GLU_SILU>, fgrid, 256, 0, stream, kp.p);
+    case EPI_GLU_RELU:
+        return launch_pdl(finalize_kernel<EPI_GLU_RELU>, fgrid, 256, 0, stream, kp.p);
+    default:
+        return launch_pdl(finalize_kernel<EPI_PLAIN>, fgrid, 256, 0, stream, kp.p);
+    }
 }
 
 template <int SRC>

@@ -11,17 +11,6 @@ namespace sgq {
 namespace {
 
 template <int ACT>
-__device__ __forceinline__ float act_mul(float g, float u)
-{
-    float a;
-    if (ACT == SGQ_ACT_SILU)
-        a = g / (1.0f + expf(-g));
-    else
-        a = g > 0.0f ? g : 0.0f;
-    return a * u;
-}
-
-template <int ACT>
 __global__ void glu_kernel(const uint4 *__restrict__ gate, const uint4 *__restrict__ up,
                            uint4 *__restrict__ h, long long nvec)
 {

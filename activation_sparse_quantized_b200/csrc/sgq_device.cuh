@@ -125,4 +125,19 @@ __device__ __forceinline__ void set_status(int32_t *status, int32_t bits)
         atomicOr(status, bits);
 }
 
+// Gated activation act(g) * u in fp32: SiLU g / (1 + e^-g) (Llama / Qwen
+// FFNs) or ReLU max(g, 0) (the ReGLU FFNs of "SVD Contextual Sparsity
+// Predictors for Fast LLM Inference", Abstract, whose zeros the down
+// projection then skips).
+template <int ACT>
+__device__ __forceinline__ float act_mul(float g, float u)
+{
+    float a;
+    if (ACT == SGQ_ACT_SILU)
+        a = g / (1.0f + expf(-g));
+    else
+        a = g > 0.0f ? g : 0.0f;
+    return a * u;
+}
+
 } // namespace sgq

@@ -20,6 +20,13 @@ enum RowSource : int {
     ROWS_THRESH = 2, // |x[k]| > t, found by each CTA for its own channel slice
 };
 
+// What the epilogue writes from the fp32 sums of the N GEMV outputs.
+enum Epilogue : int {
+    EPI_PLAIN = 0,    // y[b][n] = bf16(sum[b][n])
+    EPI_GLU_SILU = 1, // N = 2I stacked (gate; up): y[b][i] = bf16(SiLU(sum[b][i]) * sum[b][I + i])
+    EPI_GLU_RELU = 2, // the same with ReLU
+};
+
 struct GemvProblem {
     const uint8_t *qweight;
     const uint32_t *sz;
@@ -33,6 +40,7 @@ struct GemvProblem {
     int N, K, group, B;
     float t;
     int source;
+    int epilogue; // Epilogue; y (and y_f32) are [B][N/2] for the GLU epilogues
 };
 
 // Bytes of workspace (partial sums + tile counters) for N outputs, B rows.

@@ -30,7 +30,8 @@ SGQ_NOALLOC_MAX_N = 65536
 EXPORTS = (
     "sgq_packed_sizes", "sgq_pack", "sgq_select", "sgq_gemv_workspace_bytes", "sgq_gemv",
     "sgq_gemv_thresh", "sgq_gemv_dense", "sgq_glu", "sgq_status_string", "sgq_last_cuda_error",
-    "sgq_layout_version", "sgq_gemv_thresh_noalloc",
+    "sgq_layout_version", "sgq_gemv_thresh_noalloc", "sgq_gemv_glu", "sgq_gemv_glu_thresh",
+    "sgq_gemv_glu_dense",
 )
 
 
@@ -78,6 +79,9 @@ def _declare(lib):
         "sgq_gemv_dense": ([P, P, I, I, I, P, I, P, P, P, Z, P, P], I),
         "sgq_gemv_thresh_noalloc": ([P, P, I, I, I, P, F, P, P, P, P], I),
         "sgq_glu": ([P, P, P, I, I, I, P], I),
+        "sgq_gemv_glu": ([P, P, I, I, I, P, I, P, P, I, P, P, P, Z, P, P], I),
+        "sgq_gemv_glu_thresh": ([P, P, I, I, I, P, F, I, P, P, P, Z, P, P], I),
+        "sgq_gemv_glu_dense": ([P, P, I, I, I, P, I, I, P, P, P, Z, P, P], I),
         "sgq_status_string": ([I], ctypes.c_char_p),
         "sgq_last_cuda_error": ([], I),
         "sgq_layout_version": ([], I),
@@ -162,6 +166,31 @@ def sgq_gemv_dense(qweight, sz, N, K, group, x, B, y, y_f32, workspace, status=N
     _check("sgq_gemv_dense", load().sgq_gemv_dense(
         _ptr(qweight), _ptr(sz), N, K, group, _ptr(x), B, _ptr(y), _ptr(y_f32), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream)))
+
+
+def sgq_gemv_glu(qweight, sz, I, K, group, x, B, idx, count, act, h, h_f32, workspace,
+                 status=None, stream=None):
+    """Fused gate + up + act over the stacked [W_g; W_u] weights (packed with N = 2I)."""
+    _check("sgq_gemv_glu", load().sgq_gemv_glu(
+        _ptr(qweight), _ptr(sz), I, K, group, _ptr(x), B, _ptr(idx), _ptr(count), act, _ptr(h),
+        _ptr(h_f32), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _ptr(status), _stream(stream)))
+
+
+def sgq_gemv_glu_thresh(qweight, sz, I, K, group, x, t, act, h, h_f32, workspace, status=None,
+                        stream=None):
+    _check("sgq_gemv_glu_thresh", load().sgq_gemv_glu_thresh(
+        _ptr(qweight), _ptr(sz), I, K, group, _ptr(x), float(t), act, _ptr(h), _ptr(h_f32),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status),
+        _stream(stream)))
+
+
+def sgq_gemv_glu_dense(qweight, sz, I, K, group, x, B, act, h, h_f32, workspace, status=None,
+                       stream=None):
+    _check("sgq_gemv_glu_dense", load().sgq_gemv_glu_dense(
+        _ptr(qweight), _ptr(sz), I, K, group, _ptr(x), B, act, _ptr(h), _ptr(h_f32),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status),
+        _stream(stream)))
 
 
 def sgq_glu(gate, up, h, B, I, act, stream=None):

@@ -172,6 +172,45 @@ int sgq_gemv_dense(const void *qweight, const void *sz, int N, int K, int group,
 int sgq_glu(const void *gate, const void *up, void *h, int B, int I, int act, void *stream);
 
 /*
+ * Fused gated FFN front half: the gate and up projections of one FFN as a
+ * single activation-sparse GEMV, with the activation in its epilogue:
+ *
+ *     h[b][i] = act(gate[b][i]) * up[b][i],   i < I,
+ *     gate = W_g[:, S] x[S],  up = W_u[:, S] x[S]   (one active set S),
+ *
+ * where gate and up are the fp32 sums (never rounded to bf16 in between) and h
+ * is rounded once to bf16 (round to nearest even); act as in sgq_glu. The
+ * pages fuse nothing of the kind; the point is the decode FFN, where the gate
+ * and up GEMVs read the same sparse input ("Enabling Dynamic Sparsity in
+ * Quantized LLM Inference", Abstract) and ReLU gating then produces the zeros
+ * that the down projection skips ("SVD Contextual Sparsity Predictors for Fast
+ * LLM Inference", Abstract): the down projection is sgq_gemv_thresh on h with
+ * t = 0, which finds the active channels of h in its own prologue.
+ *
+ *   qweight, sz  sgq_pack of the stacked weight [W_g; W_u], fp16 [2I][K]
+ *                (rows 0..I-1 the gate, I..2I-1 the up projection), packed
+ *                with N = 2I: each active channel is then one contiguous run
+ *                of I bytes covering both projections.
+ *   I            intermediate size; 2I must be a multiple of 32.
+ *   h            bf16 [B][I]. h_f32: optional fp32 [B][I] copy of h before the
+ *                bf16 rounding (NULL = not written).
+ *   workspace    sgq_gemv_workspace_bytes(2 * I, K, B) bytes, as for sgq_gemv.
+ * The three forms take the rows as sgq_gemv (index list), sgq_gemv_thresh
+ * (B == 1, select fused) and sgq_gemv_dense (every channel). Returns as
+ * sgq_gemv, plus SGQ_ERR_ACT for an unknown act.
+ */
+int sgq_gemv_glu(const void *qweight, const void *sz, int I, int K, int group,
+                 const void *x, int B, const int32_t *idx, const int32_t *count, int act,
+                 void *h, float *h_f32, void *workspace, size_t ws_bytes, int32_t *status,
+                 void *stream);
+int sgq_gemv_glu_thresh(const void *qweight, const void *sz, int I, int K, int group,
+                        const void *x, float t, int act, void *h, float *h_f32,
+                        void *workspace, size_t ws_bytes, int32_t *status, void *stream);
+int sgq_gemv_glu_dense(const void *qweight, const void *sz, int I, int K, int group,
+                       const void *x, int B, int act, void *h, float *h_f32,
+                       void *workspace, size_t ws_bytes, int32_t *status, void *stream);
+
+/*
  * sgq_gemv_thresh without a workspace argument, for callers that cannot
  * allocate device memory (no cudaMalloc available to them, or none allowed
  * during the call). The pages have no counterpart of this entry point; it is a

@@ -94,8 +94,9 @@ def _declare(lib):
     lib.oracle_gemv.argtypes = [P, P, P, i, i, i, P, i, P, i, P, P, P]
     lib.oracle_gemv_dense.argtypes = [P, P, P, i, i, i, P, i, P, P, P]
     lib.oracle_glu.argtypes = [P, P, ctypes.c_int64, i, P, P]
+    lib.oracle_act_mul.argtypes = [P, P, ctypes.c_int64, i, P, P]
     for f in ("oracle_quantize", "oracle_pack_layout", "oracle_select",
-              "oracle_gemv", "oracle_gemv_dense", "oracle_glu"):
+              "oracle_gemv", "oracle_gemv_dense", "oracle_glu", "oracle_act_mul"):
         getattr(lib, f).restype = ctypes.c_int
     return lib
 
@@ -234,4 +235,18 @@ def glu(gate_bits, up_bits, act, lib=None):
     hb = np.empty(gt.shape, np.uint16)
     _check(lib.oracle_glu(gt.ctypes.data, up.ctypes.data, gt.size, act, h.ctypes.data,
                           hb.ctypes.data), "oracle_glu")
+    return h, hb
+
+
+def act_mul(gate, up, act, lib=None):
+    """h = act(gate) * up on fp64 inputs (act 0 = SiLU, 1 = ReLU).
+    Returns (h f64, h_bf16 u16) shaped like gate."""
+    lib = lib or load()
+    g = _c(gate, np.float64)
+    u = _c(up, np.float64)
+    assert g.shape == u.shape
+    h = np.empty(g.shape, np.float64)
+    hb = np.empty(g.shape, np.uint16)
+    _check(lib.oracle_act_mul(g.ctypes.data, u.ctypes.data, g.size, act, h.ctypes.data,
+                              hb.ctypes.data), "oracle_act_mul")
     return h, hb

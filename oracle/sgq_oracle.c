@@ -309,6 +309,15 @@ int oracle_gemv_dense(const uint8_t *q, const uint16_t *s, const uint16_t *z,
 /* h = act(gate) * up; SiLU(v) = v / (1 + e^-v); ReLU(v) = v if v > 0 else 0. */
 /* ------------------------------------------------------------------------- */
 
+/* act(g) of the gated FFN: SiLU g / (1 + e^-g) or ReLU max(g, 0) ([P5]
+ * Abstract for ReLU gating; SiLU is the Llama / Qwen gate). */
+static double oracle_act(double gv, int act)
+{
+    if (act == 0)
+        return gv / (1.0 + exp(-gv));
+    return (gv > 0.0) ? gv : 0.0;
+}
+
 int oracle_glu(const uint16_t *gate, const uint16_t *up, int64_t n, int act,
                double *h, uint16_t *h_bf16)
 {
@@ -317,12 +326,22 @@ int oracle_glu(const uint16_t *gate, const uint16_t *up, int64_t n, int act,
     for (int64_t i = 0; i < n; ++i) {
         double gv = oracle_bf16_to_double(gate[i]);
         double uv = oracle_bf16_to_double(up[i]);
-        double a;
-        if (act == 0)
-            a = gv / (1.0 + exp(-gv));
-        else
-            a = (gv > 0.0) ? gv : 0.0;
-        double hv = a * uv;
+        double hv = oracle_act(gv, act) * uv;
+        if (h)
+            h[i] = hv;
+        if (h_bf16)
+            h_bf16[i] = oracle_double_to_bf16(hv);
+    }
+    return 0;
+}
+
+int oracle_act_mul(const double *gate, const double *up, int64_t n, int act,
+                   double *h, uint16_t *h_bf16)
+{
+    if (n < 0 || (act != 0 && act != 1))
+        return -2;
+    for (int64_t i = 0; i < n; ++i) {
+        double hv = oracle_act(gate[i], act) * up[i];
         if (h)
             h[i] = hv;
         if (h_bf16)

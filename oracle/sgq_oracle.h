@@ -67,6 +67,11 @@ int oracle_gemv_dense(const uint8_t *q, const uint16_t *s, const uint16_t *z,
 int oracle_glu(const uint16_t *gate, const uint16_t *up, int64_t n, int act,
                double *h, uint16_t *h_bf16);
 
+/* The same on fp64 gate and up (the unrounded sums of the gate and up
+ * projections of one FFN): h = act(gate) * up in fp64, and rounded to bf16. */
+int oracle_act_mul(const double *gate, const double *up, int64_t n, int act,
+                   double *h, uint16_t *h_bf16);
+
 #ifdef __cplusplus
 }
 #endif

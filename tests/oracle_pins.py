@@ -436,4 +436,30 @@ def pin_glu_silu(lib):
     assert h[-6] == 0.0
 
 
+def pin_act_mul_closed_forms(lib):
+    """fp64 gated activation: sigma(ln 3) = 3/4 gives SiLU(+-ln 3) in closed
+    form; SiLU(g) - SiLU(-g) = g for every g; ReLU products are exact; h is
+    linear in up; the bf16 output is the nearest bf16 of h."""
+    l3 = np.log(3.0)
+    h, _ = oracle.act_mul(np.array([l3, -l3, 0.0, -0.0]), np.ones(4), 0, lib)
+    assert np.allclose(h, [0.75 * l3, -0.25 * l3, 0.0, 0.0], rtol=1e-15, atol=0)
+    rng = np.random.default_rng(18)
+    g = rng.standard_normal(2000) * 4
+    hp, _ = oracle.act_mul(g, np.ones_like(g), 0, lib)
+    hm, _ = oracle.act_mul(-g, np.ones_like(g), 0, lib)
+    assert np.all(np.abs((hp - hm) - g) <= 1e-14 * (1 + np.abs(g)))
+    u = rng.standard_normal(g.size)
+    h1, _ = oracle.act_mul(g, u, 0, lib)
+    h2, _ = oracle.act_mul(g, 2 * u, 0, lib)
+    assert np.array_equal(h2, 2 * h1)
+    hr, hb = oracle.act_mul(g, u, 1, lib)
+    assert np.array_equal(hr, np.where(g > 0, g, 0.0) * u)
+    # nearest bf16: no bf16 neighbour of the result is closer to h
+    dec = np.array([oracle.bf16_to_double(int(b), lib) for b in hb[:300]])
+    for d, hv, b in zip(dec, hr[:300], hb[:300]):
+        for nb in (int(b) - 1, int(b) + 1):
+            if 0 <= nb < 0x7f80 or 0x8000 <= nb < 0xff80:
+                assert abs(oracle.bf16_to_double(nb, lib) - hv) >= abs(d - hv)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -98,6 +98,20 @@ def test_host_argument_checks(lib):
     assert lib.sgq_glu(fake, fake, fake, 1, 12, 0, None) == -2               # not % 8
     assert lib.sgq_glu(fake, fake, fake, 1, 16, 5, None) == -7               # activation
     assert lib.sgq_pack(fake, 4096, 14336, 100, fake, fake, None, None) == -3
+    # fused gate + up + GLU: stacked width 2I, act checked first
+    wsg = lib.sgq_gemv_workspace_bytes(2 * 14336, 4096, 1)
+    glu = lambda **kw: [fake, fake, kw.get("I", 14336), 4096, 128, fake, kw.get("B", 1), fake,
+                        fake, kw.get("act", 0), fake, None, fake, kw.get("wsb", wsg), None, None]
+    assert lib.sgq_gemv_glu(*glu(act=2)) == -7
+    assert lib.sgq_gemv_glu(*glu(I=14344)) == -2                # 2I % 32
+    assert lib.sgq_gemv_glu(*glu(I=0)) == -2
+    assert lib.sgq_gemv_glu(*glu(B=17)) == -5
+    assert lib.sgq_gemv_glu(*glu(wsb=lib.sgq_gemv_workspace_bytes(14336, 4096, 1))) == -6
+    F = ctypes.c_float
+    assert lib.sgq_gemv_glu_thresh(fake, fake, 14336, 4096, 128, fake, F(0.5), 7, fake, None,
+                                   fake, wsg, None, None) == -7
+    assert lib.sgq_gemv_glu_dense(fake, fake, 14336, 4096, 96, fake, 1, 0, fake, None, fake,
+                                  wsg, None, None) == -3
 
 
 def test_missing_library_fails_loudly(tmp_path):
