@@ -377,6 +377,7 @@ def run_ours(args, dist: Dist):
     sel_ms = time_calls(lambda i: rep.kernel_only(i % R, "select"), 2 * period, period)
 
     e2e = run_e2e(rep, path, min(args.steps, 2000), args.warmup, dist)
+    ffn = None if args.no_ffn else run_ffn()
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": dist.world,
@@ -398,6 +399,8 @@ def run_ours(args, dist: Dist):
         "gpu_launches": args.steps * kernels_per_step,
         "clocks": clk.summary(),
     }
+    if ffn is not None:
+        line["ffn"] = ffn
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     return line
@@ -440,6 +443,106 @@ def run_e2e(rep: Replica, path: str, steps: int, warmup: int, dist: Dist):
     return {"value": round(b / (ms * 1e-3) / 1e9, 1), "unit": UNIT,
             "us_per_gemv": round(ms * 1e3 / steps, 3), "steps": steps,
             "h2d_bytes_per_step": 2 * K, "d2h_bytes_per_step": 2 * N}
+
+
+# ---------------------------------------------------------------------------
+# FFN leg: the whole decode FFN around the GEMV (secondary numbers)
+# ---------------------------------------------------------------------------
+
+class FfnReplica:
+    """R copies of one Llama-3-8B FFN (gate/up 4096 -> 14336, down 14336 -> 4096,
+    int4 g128): the stacked [W_g; W_u] for the fused path, separate W_g and W_u
+    for the unfused one, and W_d; R x bytes > 4x L2. x ~ N(0, 1) with a 50%
+    threshold into gate/up; the down projection skips |h| <= t_h, t_h the 50th
+    percentile of |h| (found once per copy, untimed)."""
+
+    def __init__(self, sparsity: float = 0.5, seed: int = 7):
+        shp = wl.LLAMA8B_LAYER["gate"]
+        self.H, self.I, self.g = shp["K"], shp["N"], shp["group"]
+        H, I, g = self.H, self.I, self.g
+        Wg, Wu, Wd = wl.weight(I, H, seed), wl.weight(I, H, seed + 1), wl.weight(H, I, seed + 2)
+        pk = lambda W: self._pack(W)
+        gu, gate, up, down = pk(torch.cat([Wg, Wu], 0)), pk(Wg), pk(Wu), pk(Wd)
+        per = sum(a.numel() * a.element_size() for t in (gu, gate, up, down) for a in t)
+        l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+        self.R = max(2, int(math.ceil(4 * l2 / per)) + 1)
+        cp = lambda t: tuple(a.clone() for a in t)
+        self.gu = [gu] + [cp(gu) for _ in range(self.R - 1)]
+        self.gate = [gate] + [cp(gate) for _ in range(self.R - 1)]
+        self.up = [up] + [cp(up) for _ in range(self.R - 1)]
+        self.down = [down] + [cp(down) for _ in range(self.R - 1)]
+        self.bytes_resident = self.R * per
+        xh = [wl.x_gaussian(1, H, 2000 + r) for r in range(self.R)]
+        self.x = [x.cuda() for x in xh]
+        self.t = [wl.percentile_threshold(x[0], sparsity) for x in xh]
+        self.h = torch.empty(1, I, dtype=torch.bfloat16, device="cuda")
+        self.yg = torch.empty(1, I, dtype=torch.bfloat16, device="cuda")
+        self.yu = torch.empty(1, I, dtype=torch.bfloat16, device="cuda")
+        self.y = torch.empty(1, H, dtype=torch.bfloat16, device="cuda")
+        self.ws_gu = sgq.alloc_workspace(2 * I, H, 1)
+        self.ws_i = sgq.alloc_workspace(I, H, 1)
+        self.ws_h = sgq.alloc_workspace(H, I, 1)
+        idx, cnt = sgq.alloc_select(max(H, I))
+        self.th, self.abytes = [], []
+        for r in range(self.R):
+            self.front_fused(r)
+            hh = self.h[0].cpu()
+            self.th.append(wl.percentile_threshold(hh, sparsity))
+            sgq.sgq_select(self.x[r], 1, H, [self.t[r]], idx, cnt)
+            a_in = int(cnt.item())
+            gin = int(np.unique(idx[:a_in].cpu().numpy() // g).size)
+            sgq.sgq_select(self.h, 1, I, [self.th[r]], idx, cnt)
+            a_h = int(cnt.item())
+            gh = int(np.unique(idx[:a_h].cpu().numpy() // g).size)
+            # stacked gate/up: a_in runs of I bytes + 8I bytes of (s, z) per group
+            self.abytes.append(a_in * I + gin * 2 * I * 4 + 2 * H + 2 * I
+                               + a_h * H // 2 + gh * H * 4 + 2 * I + 2 * H)
+        torch.cuda.synchronize()
+
+    def _pack(self, W):
+        N, K = W.shape
+        qw, sz = sgq.alloc_packed(N, K, self.g)
+        sgq.sgq_pack(W.cuda(), N, K, self.g, qw, sz)
+        return qw, sz
+
+    def front_fused(self, r):
+        qw, sz = self.gu[r]
+        sgq.sgq_gemv_glu_thresh(qw, sz, self.I, self.H, self.g, self.x[r], self.t[r],
+                                sgq.SGQ_ACT_SILU, self.h, None, self.ws_gu)
+
+    def fused(self, r):
+        self.front_fused(r)
+        qd, sd = self.down[r]
+        sgq.sgq_gemv_thresh(qd, sd, self.H, self.I, self.g, self.h, self.th[r], self.y, None,
+                            self.ws_h)
+
+    def unfused(self, r):
+        H, I, g = self.H, self.I, self.g
+        for (qw, sz), out in ((self.gate[r], self.yg), (self.up[r], self.yu)):
+            sgq.sgq_gemv_thresh(qw, sz, I, H, g, self.x[r], self.t[r], out, None, self.ws_i)
+        sgq.sgq_glu(self.yg, self.yu, self.h, 1, I, sgq.SGQ_ACT_SILU)
+        qd, sd = self.down[r]
+        sgq.sgq_gemv_thresh(qd, sd, H, I, g, self.h, self.th[r], self.y, None, self.ws_h)
+
+
+def run_ffn(n_steps: int = 2000):
+    """us per FFN, fused (4 launches) and unfused (7 launches), on the rotation."""
+    f = FfnReplica()
+    R = f.R
+    period = R * max(1, 64 // R)
+    n = max(n_steps, 2 * period)
+    ms_f = time_calls(lambda i: f.fused(i % R), n, period)
+    ms_u = time_calls(lambda i: f.unfused(i % R), n, period)
+    us_f, us_u = ms_f * 1e3 / n, ms_u * 1e3 / n
+    ab = float(np.mean(f.abytes))
+    return {"workload": "Llama-3-8B FFN decode, batch 1: gate/up 4096->14336 at 50% input "
+                        "sparsity, SiLU, down 14336->4096 over the 50% largest |h|; int4 g128",
+            "us_per_ffn_fused": round(us_f, 3), "launches_fused": 4,
+            "us_per_ffn_unfused": round(us_u, 3), "launches_unfused": 7,
+            "active_bytes_per_ffn": int(ab),
+            "fused_GBps_active": round(ab / (us_f * 1e-6) / 1e9, 1),
+            "tokens_per_s_equiv_ffn_only_32_layers": round(1e6 / (32 * us_f), 1),
+            "rotation": f"{R} copies, {f.bytes_resident / 1e6:.0f} MB"}
 
 
 # ---------------------------------------------------------------------------
@@ -533,6 +636,8 @@ def main(argv=None):
     ap.add_argument("--sparsity", type=float, default=0.5)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-ffn", action="store_true",
+                    help="skip the secondary FFN leg (fused vs unfused decode FFN)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
