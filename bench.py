@@ -377,7 +377,7 @@ def run_ours(args, dist: Dist):
     sel_ms = time_calls(lambda i: rep.kernel_only(i % R, "select"), 2 * period, period)
 
     e2e = run_e2e(rep, path, min(args.steps, 2000), args.warmup, dist)
-    ffn = None if args.no_ffn else run_ffn()
+    layer = None if args.no_ffn else run_layer()
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": dist.world,
@@ -399,8 +399,8 @@ def run_ours(args, dist: Dist):
         "gpu_launches": args.steps * kernels_per_step,
         "clocks": clk.summary(),
     }
-    if ffn is not None:
-        line["ffn"] = ffn
+    if layer is not None:
+        line.update(layer)
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     return line
@@ -446,57 +446,73 @@ def run_e2e(rep: Replica, path: str, steps: int, warmup: int, dist: Dist):
 
 
 # ---------------------------------------------------------------------------
-# FFN leg: the whole decode FFN around the GEMV (secondary numbers)
+# Layer leg: the decode FFN and the whole decode layer around the GEMV
+# (secondary numbers; attention and norms are not part of the path)
 # ---------------------------------------------------------------------------
 
-class FfnReplica:
-    """R copies of one Llama-3-8B FFN (gate/up 4096 -> 14336, down 14336 -> 4096,
-    int4 g128): the stacked [W_g; W_u] for the fused path, separate W_g and W_u
-    for the unfused one, and W_d; R x bytes > 4x L2. x ~ N(0, 1) with a 50%
-    threshold into gate/up; the down projection skips |h| <= t_h, t_h the 50th
-    percentile of |h| (found once per copy, untimed)."""
+class LayerReplica:
+    """R copies of one Llama-3-8B decode layer's projections, int4 g128:
+    q 4096->4096, k/v 4096->1024, o 4096->4096, gate/up 4096->14336,
+    down 14336->4096. Fused forms: [W_q; W_k; W_v] stacked (one GEMV, y = q|k|v)
+    and [W_g; W_u] stacked (one GEMV with the SiLU-GLU epilogue); unfused forms:
+    every projection separately plus sgq_glu. R x bytes > 4x L2.
+
+    Inputs: x ~ N(0, 1) into q/k/v and gate/up, an independent N(0, 1) stand-in
+    for the attention output into o, each with a 50% threshold; the down
+    projection skips |h| <= t_h, t_h the 50th percentile of |h| (found once
+    per copy, untimed)."""
 
     def __init__(self, sparsity: float = 0.5, seed: int = 7):
-        shp = wl.LLAMA8B_LAYER["gate"]
-        self.H, self.I, self.g = shp["K"], shp["N"], shp["group"]
+        L = wl.LLAMA8B_LAYER
+        self.H, self.I, self.g = L["gate"]["K"], L["gate"]["N"], L["gate"]["group"]
+        self.nq, self.nkv = L["q"]["N"], L["k"]["N"]
         H, I, g = self.H, self.I, self.g
-        Wg, Wu, Wd = wl.weight(I, H, seed), wl.weight(I, H, seed + 1), wl.weight(H, I, seed + 2)
-        pk = lambda W: self._pack(W)
-        gu, gate, up, down = pk(torch.cat([Wg, Wu], 0)), pk(Wg), pk(Wu), pk(Wd)
-        per = sum(a.numel() * a.element_size() for t in (gu, gate, up, down) for a in t)
+        W = {n: wl.weight(L[n]["N"], L[n]["K"], seed + j) for j, n in enumerate(L)}
+        base = {
+            "qkv": self._pack(torch.cat([W["q"], W["k"], W["v"]], 0)),
+            "q": self._pack(W["q"]), "k": self._pack(W["k"]), "v": self._pack(W["v"]),
+            "o": self._pack(W["o"]),
+            "gu": self._pack(torch.cat([W["gate"], W["up"]], 0)),
+            "gate": self._pack(W["gate"]), "up": self._pack(W["up"]), "down": self._pack(W["down"]),
+        }
+        per = sum(a.numel() * a.element_size() for t in base.values() for a in t)
         l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
         self.R = max(2, int(math.ceil(4 * l2 / per)) + 1)
-        cp = lambda t: tuple(a.clone() for a in t)
-        self.gu = [gu] + [cp(gu) for _ in range(self.R - 1)]
-        self.gate = [gate] + [cp(gate) for _ in range(self.R - 1)]
-        self.up = [up] + [cp(up) for _ in range(self.R - 1)]
-        self.down = [down] + [cp(down) for _ in range(self.R - 1)]
+        self.w = [base] + [{k: tuple(a.clone() for a in t) for k, t in base.items()}
+                           for _ in range(self.R - 1)]
         self.bytes_resident = self.R * per
-        xh = [wl.x_gaussian(1, H, 2000 + r) for r in range(self.R)]
-        self.x = [x.cuda() for x in xh]
-        self.t = [wl.percentile_threshold(x[0], sparsity) for x in xh]
-        self.h = torch.empty(1, I, dtype=torch.bfloat16, device="cuda")
-        self.yg = torch.empty(1, I, dtype=torch.bfloat16, device="cuda")
-        self.yu = torch.empty(1, I, dtype=torch.bfloat16, device="cuda")
-        self.y = torch.empty(1, H, dtype=torch.bfloat16, device="cuda")
-        self.ws_gu = sgq.alloc_workspace(2 * I, H, 1)
-        self.ws_i = sgq.alloc_workspace(I, H, 1)
-        self.ws_h = sgq.alloc_workspace(H, I, 1)
+        xa = [wl.x_gaussian(1, H, 2000 + r) for r in range(self.R)]
+        xo = [wl.x_gaussian(1, H, 3000 + r) for r in range(self.R)]
+        self.xa, self.xo = [x.cuda() for x in xa], [x.cuda() for x in xo]
+        self.ta = [wl.percentile_threshold(x[0], sparsity) for x in xa]
+        self.to = [wl.percentile_threshold(x[0], sparsity) for x in xo]
+        dev = lambda n: torch.empty(1, n, dtype=torch.bfloat16, device="cuda")
+        self.h, self.yg, self.yu = dev(I), dev(I), dev(I)
+        self.y, self.yqkv, self.yo = dev(H), dev(self.nq + 2 * self.nkv), dev(H)
+        self.yq, self.yk, self.yv = dev(self.nq), dev(self.nkv), dev(self.nkv)
+        self.ws = sgq.alloc_workspace(2 * I, max(H, I), 1)     # largest B*N of any call
         idx, cnt = sgq.alloc_select(max(H, I))
-        self.th, self.abytes = [], []
+        self.th, self.ffn_bytes, self.layer_bytes = [], [], []
+
+        def active(x, t, K):
+            sgq.sgq_select(x, 1, K, [t], idx, cnt)
+            a = int(cnt.item())
+            return a, int(np.unique(idx[:a].cpu().numpy() // g).size)
+
         for r in range(self.R):
-            self.front_fused(r)
-            hh = self.h[0].cpu()
-            self.th.append(wl.percentile_threshold(hh, sparsity))
-            sgq.sgq_select(self.x[r], 1, H, [self.t[r]], idx, cnt)
-            a_in = int(cnt.item())
-            gin = int(np.unique(idx[:a_in].cpu().numpy() // g).size)
-            sgq.sgq_select(self.h, 1, I, [self.th[r]], idx, cnt)
-            a_h = int(cnt.item())
-            gh = int(np.unique(idx[:a_h].cpu().numpy() // g).size)
-            # stacked gate/up: a_in runs of I bytes + 8I bytes of (s, z) per group
-            self.abytes.append(a_in * I + gin * 2 * I * 4 + 2 * H + 2 * I
-                               + a_h * H // 2 + gh * H * 4 + 2 * I + 2 * H)
+            self.gate_up(r)
+            self.th.append(wl.percentile_threshold(self.h[0].cpu(), sparsity))
+            a_in, g_in = active(self.xa[r], self.ta[r], H)
+            a_o, g_o = active(self.xo[r], self.to[r], H)
+            a_h, g_h = active(self.h, self.th[r], I)
+            nqkv = self.nq + 2 * self.nkv
+            # active bytes: codes of the active channels, (s, z) of touched groups, x, y
+            ffn = (a_in * I + g_in * 2 * I * 4 + 2 * H + 2 * I
+                   + a_h * H // 2 + g_h * H * 4 + 2 * I + 2 * H)
+            attn = (a_in * nqkv // 2 + g_in * nqkv * 4 + 2 * H + 2 * nqkv
+                    + a_o * H // 2 + g_o * H * 4 + 2 * H + 2 * H)
+            self.ffn_bytes.append(ffn)
+            self.layer_bytes.append(ffn + attn)
         torch.cuda.synchronize()
 
     def _pack(self, W):
@@ -505,44 +521,71 @@ class FfnReplica:
         sgq.sgq_pack(W.cuda(), N, K, self.g, qw, sz)
         return qw, sz
 
-    def front_fused(self, r):
-        qw, sz = self.gu[r]
-        sgq.sgq_gemv_glu_thresh(qw, sz, self.I, self.H, self.g, self.x[r], self.t[r],
-                                sgq.SGQ_ACT_SILU, self.h, None, self.ws_gu)
+    def _thresh(self, w, N, K, x, t, y):
+        sgq.sgq_gemv_thresh(w[0], w[1], N, K, self.g, x, t, y, None, self.ws)
 
-    def fused(self, r):
-        self.front_fused(r)
-        qd, sd = self.down[r]
-        sgq.sgq_gemv_thresh(qd, sd, self.H, self.I, self.g, self.h, self.th[r], self.y, None,
-                            self.ws_h)
+    def gate_up(self, r):
+        qw, sz = self.w[r]["gu"]
+        sgq.sgq_gemv_glu_thresh(qw, sz, self.I, self.H, self.g, self.xa[r], self.ta[r],
+                                sgq.SGQ_ACT_SILU, self.h, None, self.ws)
 
-    def unfused(self, r):
-        H, I, g = self.H, self.I, self.g
-        for (qw, sz), out in ((self.gate[r], self.yg), (self.up[r], self.yu)):
-            sgq.sgq_gemv_thresh(qw, sz, I, H, g, self.x[r], self.t[r], out, None, self.ws_i)
+    def ffn_fused(self, r):                      # 4 launches
+        self.gate_up(r)
+        self._thresh(self.w[r]["down"], self.H, self.I, self.h, self.th[r], self.y)
+
+    def ffn_unfused(self, r):                    # 7 launches
+        w, H, I = self.w[r], self.H, self.I
+        self._thresh(w["gate"], I, H, self.xa[r], self.ta[r], self.yg)
+        self._thresh(w["up"], I, H, self.xa[r], self.ta[r], self.yu)
         sgq.sgq_glu(self.yg, self.yu, self.h, 1, I, sgq.SGQ_ACT_SILU)
-        qd, sd = self.down[r]
-        sgq.sgq_gemv_thresh(qd, sd, H, I, g, self.h, self.th[r], self.y, None, self.ws_h)
+        self._thresh(w["down"], H, I, self.h, self.th[r], self.y)
+
+    def layer_fused(self, r):                    # 8 launches
+        w, H = self.w[r], self.H
+        self._thresh(w["qkv"], self.nq + 2 * self.nkv, H, self.xa[r], self.ta[r], self.yqkv)
+        self._thresh(w["o"], H, H, self.xo[r], self.to[r], self.yo)
+        self.ffn_fused(r)
+
+    def layer_unfused(self, r):                  # 15 launches
+        w, H = self.w[r], self.H
+        for n, N, y in (("q", self.nq, self.yq), ("k", self.nkv, self.yk),
+                        ("v", self.nkv, self.yv)):
+            self._thresh(w[n], N, H, self.xa[r], self.ta[r], y)
+        self._thresh(w["o"], H, H, self.xo[r], self.to[r], self.yo)
+        self.ffn_unfused(r)
 
 
-def run_ffn(n_steps: int = 2000):
-    """us per FFN, fused (4 launches) and unfused (7 launches), on the rotation."""
-    f = FfnReplica()
+def run_layer(n_steps: int = 1000):
+    """us per decode FFN and per decode layer (projections only), fused and
+    unfused, on the rotation."""
+    f = LayerReplica()
     R = f.R
-    period = R * max(1, 64 // R)
+    period = R * max(1, 32 // R)
     n = max(n_steps, 2 * period)
-    ms_f = time_calls(lambda i: f.fused(i % R), n, period)
-    ms_u = time_calls(lambda i: f.unfused(i % R), n, period)
-    us_f, us_u = ms_f * 1e3 / n, ms_u * 1e3 / n
-    ab = float(np.mean(f.abytes))
-    return {"workload": "Llama-3-8B FFN decode, batch 1: gate/up 4096->14336 at 50% input "
-                        "sparsity, SiLU, down 14336->4096 over the 50% largest |h|; int4 g128",
-            "us_per_ffn_fused": round(us_f, 3), "launches_fused": 4,
-            "us_per_ffn_unfused": round(us_u, 3), "launches_unfused": 7,
-            "active_bytes_per_ffn": int(ab),
-            "fused_GBps_active": round(ab / (us_f * 1e-6) / 1e9, 1),
-            "tokens_per_s_equiv_ffn_only_32_layers": round(1e6 / (32 * us_f), 1),
-            "rotation": f"{R} copies, {f.bytes_resident / 1e6:.0f} MB"}
+    us = {}
+    for name in ("ffn_fused", "ffn_unfused", "layer_fused", "layer_unfused"):
+        fn = getattr(f, name)
+        us[name] = time_calls(lambda i: fn(i % R), n, period) * 1e3 / n
+    fb, lb = float(np.mean(f.ffn_bytes)), float(np.mean(f.layer_bytes))
+    return {
+        "ffn": {"workload": "Llama-3-8B FFN decode, batch 1: gate/up 4096->14336 at 50% input "
+                            "sparsity, SiLU, down 14336->4096 over the 50% largest |h|; int4 g128",
+                "us_per_ffn_fused": round(us["ffn_fused"], 3), "launches_fused": 4,
+                "us_per_ffn_unfused": round(us["ffn_unfused"], 3), "launches_unfused": 7,
+                "active_bytes_per_ffn": int(fb),
+                "fused_GBps_active": round(fb / (us["ffn_fused"] * 1e-6) / 1e9, 1),
+                "tokens_per_s_equiv_ffn_only_32_layers": round(1e6 / (32 * us["ffn_fused"]), 1)},
+        "layer": {"workload": "Llama-3-8B decode layer projections, batch 1: q/k/v (stacked), "
+                              "o, gate/up (stacked, SiLU-GLU epilogue), down; 50% sparsity per "
+                              "projection input; attention and norms excluded",
+                  "us_per_layer_fused": round(us["layer_fused"], 3), "launches_fused": 8,
+                  "us_per_layer_unfused": round(us["layer_unfused"], 3), "launches_unfused": 15,
+                  "active_bytes_per_layer": int(lb),
+                  "fused_GBps_active": round(lb / (us["layer_fused"] * 1e-6) / 1e9, 1),
+                  "tokens_per_s_equiv_32_layers_projections_only":
+                      round(1e6 / (32 * us["layer_fused"]), 1)},
+        "rotation": f"{R} copies, {f.bytes_resident / 1e6:.0f} MB",
+    }
 
 
 # ---------------------------------------------------------------------------
@@ -637,7 +680,7 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-ffn", action="store_true",
-                    help="skip the secondary FFN leg (fused vs unfused decode FFN)")
+                    help="skip the secondary FFN / decode-layer leg (fused vs unfused)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

@@ -202,3 +202,30 @@ def test_glu_fused_all_masked_gives_zero():
         for act in (SILU, RELU):
             h, h32 = gg.run(path, x.to(DEV), [float("inf")], act)
             assert (h32 == 0).all() and bits(h).max() == 0
+
+
+def test_qkv_stacked_single_gemv():
+    """Llama-3-8B q/k/v (4096 -> 4096 / 1024 / 1024) stacked as one weight:
+    one threshold-GEMV gives y = q | k | v, each part within the GEMV bound of
+    the oracle's own projection, every output checked."""
+    L = wl.LLAMA8B_LAYER
+    K, g = L["q"]["K"], L["q"]["group"]
+    Ws = [wl.weight(L[n]["N"], K, 370 + j) for j, n in enumerate(("q", "k", "v"))]
+    W = torch.cat(Ws, 0)
+    x = wl.x_gaussian(1, K, 373)
+    t = [wl.percentile_threshold(x[0], 0.5)]
+    qw, sz, _ = gpu_pack(W, g)
+    N = W.shape[0]
+    y = torch.full((1, N), float("nan"), dtype=torch.bfloat16, device=DEV)
+    y32 = torch.full((1, N), float("nan"), dtype=torch.float32, device=DEV)
+    ws = sgq.alloc_workspace(N, K, 1)
+    sgq.sgq_gemv_thresh(qw, sz, N, K, g, x.to(DEV), t[0], y, y32, ws)
+    xb = bits(x)
+    idx = oracle.select(xb, t)
+    o = 0
+    for Wp, name in zip(Ws, ("q", "k", "v")):
+        n = Wp.shape[0]
+        q, s, z = oracle_codes(Wp, g)
+        y64, sa, _ = oracle.gemv(q, s, z, g, xb, idx)
+        check_y(y[:, o:o + n], y32[:, o:o + n], y64, sa, f"stacked {name}")
+        o += n
