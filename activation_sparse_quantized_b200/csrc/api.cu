@@ -76,6 +76,10 @@ int run_gemv(sgq::GemvProblem &p, size_t ws_bytes, void *workspace, void *stream
         return SGQ_ERR_NULL;
     if (p.source == sgq::ROWS_LIST && (!p.idx || !p.count))
         return SGQ_ERR_NULL;
+    if (p.source == sgq::ROWS_MASK && !p.mask)
+        return SGQ_ERR_NULL;
+    if (p.source == sgq::ROWS_MASK && !aligned16(p.mask))
+        return SGQ_ERR_ALIGN;
     if (!aligned16(p.qweight) || !aligned16(p.sz) || !aligned16(p.x) || !aligned16(p.y) ||
         !aligned16(workspace) || (p.y_f32 && !aligned16(p.y_f32)))
         return SGQ_ERR_ALIGN;
@@ -184,6 +188,28 @@ int sgq_select(const void *x, int B, int K, const float *t_host, int32_t *idx, i
     return e == cudaSuccess ? SGQ_OK : fail_cuda(e);
 }
 
+int sgq_select_mask(const void *x, int B, int K, const float *t_host, uint32_t *mask,
+                    int32_t *count, void *stream)
+{
+    if (B < 1 || B > SGQ_MAX_BATCH)
+        return SGQ_ERR_BATCH;
+    if (K <= 0 || K % 8 != 0)
+        return SGQ_ERR_SHAPE;
+    if (!x || !t_host || !mask)
+        return SGQ_ERR_NULL;
+    if (!aligned16(x) || !aligned16(mask))
+        return SGQ_ERR_ALIGN;
+    int sms = current_device_sms();
+    if (sms < 0)
+        return sms;
+    sgq::Thresholds th{};
+    for (int b = 0; b < B; ++b)
+        th.t[b] = t_host[b];
+    cudaError_t e = sgq::launch_select_mask(static_cast<const uint16_t *>(x), B, K, th, mask,
+                                            count, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SGQ_OK : fail_cuda(e);
+}
+
 size_t sgq_gemv_workspace_bytes(int N, int K, int B)
 {
     (void)K;
@@ -230,6 +256,26 @@ int sgq_gemv_thresh(const void *qweight, const void *sz, int N, int K, int group
     p.B = 1;
     p.t = t;
     p.source = sgq::ROWS_THRESH;
+    return run_gemv(p, ws_bytes, workspace, stream);
+}
+
+int sgq_gemv_mask(const void *qweight, const void *sz, int N, int K, int group, const void *x,
+                  int B, const uint32_t *mask, void *y, float *y_f32, void *workspace,
+                  size_t ws_bytes, int32_t *status, void *stream)
+{
+    sgq::GemvProblem p{};
+    p.qweight = static_cast<const uint8_t *>(qweight);
+    p.sz = static_cast<const uint32_t *>(sz);
+    p.x = static_cast<const uint16_t *>(x);
+    p.mask = mask;
+    p.y = static_cast<uint16_t *>(y);
+    p.y_f32 = y_f32;
+    p.status = status;
+    p.N = N;
+    p.K = K;
+    p.group = group;
+    p.B = B;
+    p.source = sgq::ROWS_MASK;
     return run_gemv(p, ws_bytes, workspace, stream);
 }
 

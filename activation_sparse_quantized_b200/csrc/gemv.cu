@@ -115,6 +115,40 @@ __device__ int build_rows(const KParams &kp, int split, int32_t *ridx, float *rx
             ridx[j] = r0 + j;
         __syncthreads();
         return r1 - r0;
+    } else if (SRC == ROWS_MASK) {
+        // Decode this CTA's channel slice of the bitmask: runs of 32 channels,
+        // one per lane, a ballot per run, the count of each run in scan[]; a
+        // second pass recomputes the ballots (the mask words stay in L1) and
+        // writes each active channel at its ascending position.
+        int c0, c1;
+        channel_slice(kp, split, c0, c1);
+        const int lane = tid & 31, warp = tid >> 5;
+        const int runs = (c1 - c0 + 31) / 32;
+        auto run_bits = [&](int q) -> uint32_t {
+            const int c = c0 + q * 32 + lane;
+            const bool act = (c < c1) && ((__ldg(p.mask + (c >> 5)) >> (c & 31)) & 1u);
+            return __ballot_sync(0xffffffffu, act);
+        };
+        for (int q = warp; q < runs; q += NT / 32) {
+            const uint32_t m = run_bits(q);
+            if (lane == 0)
+                scan[q] = __popc(m);
+        }
+        __syncthreads();
+        int total = 0;
+        for (int q = 0; q < runs; ++q)
+            total += scan[q];
+        for (int q = warp; q < runs; q += NT / 32) {
+            const uint32_t m = run_bits(q);
+            if ((m >> lane) & 1u) {
+                int pos = __popc(m & ((1u << lane) - 1u));
+                for (int r = 0; r < q; ++r)
+                    pos += scan[r];
+                ridx[pos] = c0 + q * 32 + lane;
+            }
+        }
+        __syncthreads();
+        return total;
     } else {
         // Threshold this CTA's channel slice: each warp takes runs of 32
         // channels, one per lane; a ballot gives each run's active channels,
@@ -343,7 +377,7 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
     };
     if (SRC != ROWS_LIST) {
         int c0, c1;
-        if (SRC == ROWS_THRESH) {
+        if (SRC == ROWS_THRESH || SRC == ROWS_MASK) {
             channel_slice(kp, split, c0, c1);
         } else {
             c0 = (int)((long long)p.K * split / kp.k_splits);
@@ -571,7 +605,7 @@ __host__ __device__ inline SmemB smemB_layout(int span_cap, int rows_cap, int BT
     s.ridx = s.red + (size_t)BT * kTileNB * 4;
     s.rx = s.ridx + (size_t)rows_cap * 4;
     s.scan = s.rx + (size_t)rows_cap * BT * 4;
-    s.total = s.scan + 64;
+    s.total = s.scan + (size_t)((rows_cap + 31) / 32 + 4) * 4;
     return s;
 }
 
@@ -870,11 +904,14 @@ cudaError_t launch_gemv(const GemvProblem &p, int num_sms, cudaStream_t stream)
         switch (p.source) {
         case ROWS_LIST: return launch_b1<ROWS_LIST>(kp, num_sms, stream);
         case ROWS_DENSE: return launch_b1<ROWS_DENSE>(kp, num_sms, stream);
+        case ROWS_MASK: return launch_b1<ROWS_MASK>(kp, num_sms, stream);
         default: return launch_b1<ROWS_THRESH>(kp, num_sms, stream);
         }
     }
     if (p.source == ROWS_DENSE)
         return launch_bn<ROWS_DENSE>(kp, num_sms, stream);
+    if (p.source == ROWS_MASK)
+        return launch_bn<ROWS_MASK>(kp, num_sms, stream);
     return launch_bn<ROWS_LIST>(kp, num_sms, stream);
 }
 

@@ -18,6 +18,7 @@ enum RowSource : int {
     ROWS_LIST = 0,   // device list idx[0..*count)
     ROWS_DENSE = 1,  // every channel
     ROWS_THRESH = 2, // |x[k]| > t, found by each CTA for its own channel slice
+    ROWS_MASK = 3,   // bit k of a device bitmask, decoded by each CTA for its own slice
 };
 
 // What the epilogue writes from the fp32 sums of the N GEMV outputs.
@@ -33,6 +34,7 @@ struct GemvProblem {
     const uint16_t *x;
     const int32_t *idx;
     const int32_t *count;
+    const uint32_t *mask; // ROWS_MASK: bit k % 32 of word k / 32 = channel k active
     uint16_t *y;
     float *y_f32;
     float *ws_acc;
@@ -50,6 +52,8 @@ cudaError_t launch_pack(const uint16_t *W, int N, int K, int g, uint8_t *qweight
                         int32_t *status, cudaStream_t stream);
 cudaError_t launch_select(const uint16_t *x, int B, int K, const Thresholds &th, int32_t *idx,
                           int32_t *count, cudaStream_t stream);
+cudaError_t launch_select_mask(const uint16_t *x, int B, int K, const Thresholds &th,
+                               uint32_t *mask, int32_t *count, cudaStream_t stream);
 cudaError_t launch_gemv(const GemvProblem &p, int num_sms, cudaStream_t stream);
 // Records e as the last CUDA error of this thread; returns SGQ_ERR_CUDA.
 int record_cuda_error(cudaError_t e);

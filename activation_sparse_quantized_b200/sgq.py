@@ -31,7 +31,7 @@ EXPORTS = (
     "sgq_packed_sizes", "sgq_pack", "sgq_select", "sgq_gemv_workspace_bytes", "sgq_gemv",
     "sgq_gemv_thresh", "sgq_gemv_dense", "sgq_glu", "sgq_status_string", "sgq_last_cuda_error",
     "sgq_layout_version", "sgq_gemv_thresh_noalloc", "sgq_gemv_glu", "sgq_gemv_glu_thresh",
-    "sgq_gemv_glu_dense",
+    "sgq_gemv_glu_dense", "sgq_select_mask", "sgq_gemv_mask",
 )
 
 
@@ -82,6 +82,8 @@ def _declare(lib):
         "sgq_gemv_glu": ([P, P, I, I, I, P, I, P, P, I, P, P, P, Z, P, P], I),
         "sgq_gemv_glu_thresh": ([P, P, I, I, I, P, F, I, P, P, P, Z, P, P], I),
         "sgq_gemv_glu_dense": ([P, P, I, I, I, P, I, I, P, P, P, Z, P, P], I),
+        "sgq_select_mask": ([P, I, I, P, P, P, P], I),
+        "sgq_gemv_mask": ([P, P, I, I, I, P, I, P, P, P, P, Z, P, P], I),
         "sgq_status_string": ([I], ctypes.c_char_p),
         "sgq_last_cuda_error": ([], I),
         "sgq_layout_version": ([], I),
@@ -131,6 +133,20 @@ def sgq_select(x, B, K, t_host, idx, count, stream=None):
     t = (ctypes.c_float * B)(*[float(v) for v in t_host])
     _check("sgq_select", load().sgq_select(_ptr(x), B, K, t, _ptr(idx), _ptr(count),
                                            _stream(stream)))
+
+
+def sgq_select_mask(x, B, K, t_host, mask, count=None, stream=None):
+    t = (ctypes.c_float * B)(*[float(v) for v in t_host])
+    _check("sgq_select_mask", load().sgq_select_mask(_ptr(x), B, K, t, _ptr(mask), _ptr(count),
+                                                     _stream(stream)))
+
+
+def sgq_gemv_mask(qweight, sz, N, K, group, x, B, mask, y, y_f32, workspace, status=None,
+                  stream=None):
+    _check("sgq_gemv_mask", load().sgq_gemv_mask(
+        _ptr(qweight), _ptr(sz), N, K, group, _ptr(x), B, _ptr(mask), _ptr(y), _ptr(y_f32),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status),
+        _stream(stream)))
 
 
 def sgq_gemv_workspace_bytes(N: int, K: int, B: int) -> int:
@@ -210,6 +226,11 @@ def alloc_packed(N, K, group, device="cuda"):
 def alloc_workspace(N, K, B, device="cuda"):
     nbytes = sgq_gemv_workspace_bytes(N, K, B)
     return torch.zeros(nbytes // 4, dtype=torch.int32, device=device)
+
+
+def alloc_mask(K, device="cuda"):
+    """uint32 words for a K-channel bitmask (int32 tensor; bits are what matter)."""
+    return torch.zeros((K + 31) // 32, dtype=torch.int32, device=device)
 
 
 def alloc_select(K, device="cuda"):

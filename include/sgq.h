@@ -109,6 +109,23 @@ int sgq_select(const void *x, int B, int K, const float *t_host,
                int32_t *idx, int32_t *count, void *stream);
 
 /*
+ * The same active set as a bitmask, one bit per channel: the compact form an
+ * activation predictor or a previous kernel can emit instead of an index list
+ * (the bitmask indexing of "SparseDecoding: Decoding-Aware Pruning for
+ * Accurate and Efficient LLM Inference", Abstract; the shared-memory bitmap
+ * decoding of "Unified Static-Dynamic Pruning for Efficient LLM Inference",
+ * Abstract, listed on that page).
+ *
+ *   mask    uint32 [(K + 31) / 32]: bit k % 32 of word k / 32 is 1 when
+ *           |x[b][k]| > t[b] for some b (strict; NaN never active). Bits of
+ *           channels k >= K in the last word are written 0.
+ *   count   optional int32 device scalar (NULL = not written): |S|.
+ * Requires 1 <= B <= 16, K % 8 == 0. K/8 bytes instead of 4|S| bytes.
+ */
+int sgq_select_mask(const void *x, int B, int K, const float *t_host,
+                    uint32_t *mask, int32_t *count, void *stream);
+
+/*
  * Workspace for sgq_gemv / sgq_gemv_thresh / sgq_gemv_dense: B*N floats of
  * split-K partial sums. It must be zero-filled once when it is allocated;
  * every call leaves it zero-filled again. Calls that may run concurrently
@@ -153,6 +170,19 @@ int sgq_gemv(const void *qweight, const void *sz, int N, int K, int group,
 int sgq_gemv_thresh(const void *qweight, const void *sz, int N, int K, int group,
                     const void *x, float t, void *y, float *y_f32,
                     void *workspace, size_t ws_bytes, int32_t *status, void *stream);
+
+/*
+ * The activation-sparse GEMV with the active set given as a bitmask (as
+ * written by sgq_select_mask, or by any producer of the same format): the
+ * same result as sgq_gemv over the ascending list of the set bits. Each CTA
+ * decodes the bits of its own channel slice in shared memory, so no global
+ * list or count is needed. Bits of channels >= K are ignored. 1 <= B <= 16;
+ * every batch row uses the one mask (normally the union). Other arguments as
+ * sgq_gemv.
+ */
+int sgq_gemv_mask(const void *qweight, const void *sz, int N, int K, int group,
+                  const void *x, int B, const uint32_t *mask, void *y, float *y_f32,
+                  void *workspace, size_t ws_bytes, int32_t *status, void *stream);
 
 /*
  * The dense int4 GEMV over the same packed weights (every channel active): the

@@ -95,8 +95,9 @@ def _declare(lib):
     lib.oracle_gemv_dense.argtypes = [P, P, P, i, i, i, P, i, P, P, P]
     lib.oracle_glu.argtypes = [P, P, ctypes.c_int64, i, P, P]
     lib.oracle_act_mul.argtypes = [P, P, ctypes.c_int64, i, P, P]
+    lib.oracle_select_mask.argtypes = [P, i, i, P, P, P]
     for f in ("oracle_quantize", "oracle_pack_layout", "oracle_select",
-              "oracle_gemv", "oracle_gemv_dense", "oracle_glu", "oracle_act_mul"):
+              "oracle_gemv", "oracle_gemv_dense", "oracle_glu", "oracle_act_mul", "oracle_select_mask"):
         getattr(lib, f).restype = ctypes.c_int
     return lib
 
@@ -250,3 +251,16 @@ def act_mul(gate, up, act, lib=None):
     _check(lib.oracle_act_mul(g.ctypes.data, u.ctypes.data, g.size, act, h.ctypes.data,
                               hb.ctypes.data), "oracle_act_mul")
     return h, hb
+
+
+def select_mask(x_bits, t, lib=None):
+    """Bitmask of the active set of x [B][K] (bf16 bits): uint32 [(K + 31) / 32]."""
+    lib = lib or load()
+    x = _c(np.atleast_2d(x_bits), np.uint16)
+    B, K = x.shape
+    tt = _c(np.broadcast_to(np.asarray(t, np.float32), (B,)), np.float32)
+    mask = np.empty((K + 31) // 32, np.uint32)
+    cnt = ctypes.c_int32()
+    _check(lib.oracle_select_mask(x.ctypes.data, B, K, tt.ctypes.data, mask.ctypes.data,
+                                  ctypes.byref(cnt)), "oracle_select_mask")
+    return mask, cnt.value

@@ -16,6 +16,7 @@
 #include "sgq_oracle.h"
 
 #include <math.h>
+#include <stdlib.h>
 #include <stddef.h>
 #include <stdint.h>
 
@@ -228,6 +229,30 @@ int oracle_select(const uint16_t *x, int B, int K, const float *t,
     }
     *count = c;
     return 0;
+}
+
+/* The same active set as a bitmask: bit k % 32 of word k / 32 set exactly for
+ * k in S (the bitmask indexing of "SparseDecoding: Decoding-Aware Pruning for
+ * Accurate and Efficient LLM Inference", Abstract). */
+int oracle_select_mask(const uint16_t *x, int B, int K, const float *t,
+                       uint32_t *mask, int32_t *count)
+{
+    if (B <= 0 || K <= 0)
+        return -2;
+    int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * (size_t)K);
+    if (!idx)
+        return -3;
+    int32_t c = 0;
+    int rc = oracle_select(x, B, K, t, idx, &c);
+    if (rc == 0) {
+        for (int w = 0; w < (K + 31) / 32; ++w)
+            mask[w] = 0u;
+        for (int32_t i = 0; i < c; ++i)
+            mask[idx[i] / 32] |= 1u << (idx[i] % 32);
+        *count = c;
+    }
+    free(idx);
+    return rc;
 }
 
 /* ------------------------------------------------------------------------- */

@@ -49,6 +49,11 @@ int oracle_pack_layout(const uint8_t *q, const uint16_t *s, const uint16_t *z,
 int oracle_select(const uint16_t *x, int B, int K, const float *t,
                   int32_t *idx, int32_t *count);
 
+/* The same set as a bitmask: mask [(K + 31) / 32] words, bit k % 32 of word
+ * k / 32 set exactly when k is in S; *count <- |S|. */
+int oracle_select_mask(const uint16_t *x, int B, int K, const float *t,
+                       uint32_t *mask, int32_t *count);
+
 /* y[b][n] = sum over the listed k of W_deq[n][k] * x[b][k], in fp64, ascending
  * k. Also returns sumabs[b][n] = sum of |W_deq[n][k] * x[b][k]| over the same
  * k, and y rounded to bf16. Any of y, sumabs, y_bf16 may be NULL. */

@@ -462,4 +462,28 @@ def pin_act_mul_closed_forms(lib):
                 assert abs(oracle.bf16_to_double(nb, lib) - hv) >= abs(d - hv)
 
 
+def pin_select_mask_bits(lib):
+    """Bitmask of the active set: a hand fixture fixes the bit order (channel k
+    is bit k % 32 of word k / 32), and brute force on random batches fixes the
+    union and the strict comparison."""
+    K = 72
+    x = np.zeros((1, K), np.float32)
+    for k in (0, 31, 32, 33, 63, 71):
+        x[0, k] = 1.0
+    x[0, 5] = 0.5                                   # equal to t: not active
+    m, c = oracle.select_mask(bf16_bits_from_f32(x), [0.5], lib)
+    assert m.tolist() == [0x80000001, 0x80000003, 0x80] and c == 6
+    rng = np.random.default_rng(19)
+    for B, K in ((1, 256), (3, 1000), (16, 136)):
+        xv = rng.standard_normal((B, K)).astype(np.float32)
+        xb = bf16_bits_from_f32(xv)
+        t = np.abs(rng.standard_normal(B)).astype(np.float32)
+        act = (np.abs(torch_bf16(xb).reshape(B, K)) > t[:, None]).any(axis=0)
+        m, c = oracle.select_mask(xb, t, lib)
+        words = np.zeros((K + 31) // 32, np.uint64)
+        for k in np.nonzero(act)[0]:
+            words[k // 32] |= np.uint64(1) << np.uint64(k % 32)
+        assert np.array_equal(m.astype(np.uint64), words) and c == int(act.sum())
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

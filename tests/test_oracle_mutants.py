@@ -38,6 +38,10 @@ MUTANTS = {
     "union_last_row_only": ("for (int b = 0; b < B; ++b) {\n            double a",
                             "for (int b = B - 1; b < B; ++b) {\n            double a"),
     "sumabs_signed": ("acc_abs += fabs(p);", "acc_abs += p;"),
+    "mask_bit_order": ("mask[idx[i] / 32] |= 1u << (idx[i] % 32);",
+                       "mask[idx[i] / 32] |= 1u << (31 - idx[i] % 32);"),
+    "mask_word_index": ("mask[idx[i] / 32] |= 1u << (idx[i] % 32);",
+                        "mask[idx[i] / 8 % ((K + 31) / 32)] |= 1u << (idx[i] % 32);"),
     "act_mul_drops_up": ("double hv = oracle_act(gate[i], act) * up[i];",
                          "double hv = oracle_act(gate[i], act);"),
     "act_mul_swapped": ("double hv = oracle_act(gate[i], act) * up[i];",
