@@ -86,8 +86,9 @@ __device__ __forceinline__ void channel_slice(const KParams &kp, int split, int 
 // return nr. Entries outside [0, K) become -1 (their x is 0; they read row 0).
 // Must be called by all threads; ends with a barrier.
 // ---------------------------------------------------------------------------
-template <int SRC, int NT>
-__device__ int build_rows(const KParams &kp, int split, int32_t *ridx, float *rx, int *scan)
+template <int SRC, int NT, bool FILL_X = false>
+__device__ int build_rows(const KParams &kp, int split, int32_t *ridx, float *rx, int *scan,
+                          float *xs = nullptr)
 {
     const GemvProblem &p = kp.p;
     const int tid = threadIdx.x;
@@ -119,7 +120,10 @@ __device__ int build_rows(const KParams &kp, int split, int32_t *ridx, float *rx
         // Decode this CTA's channel slice of the bitmask: runs of 32 channels,
         // one per lane, a ballot per run, the count of each run in scan[]; a
         // second pass recomputes the ballots (the mask words stay in L1) and
-        // writes each active channel at its ascending position.
+        // writes each active channel at its ascending position. With FILL_X
+        // (batch 1) the first pass also reads the slice of x, coalesced and
+        // alongside the mask words, into xs[], and the second copies the x of
+        // each active channel into rx[].
         int c0, c1;
         channel_slice(kp, split, c0, c1);
         const int lane = tid & 31, warp = tid >> 5;
@@ -130,6 +134,11 @@ __device__ int build_rows(const KParams &kp, int split, int32_t *ridx, float *rx
             return __ballot_sync(0xffffffffu, act);
         };
         for (int q = warp; q < runs; q += NT / 32) {
+            if (FILL_X) {
+                const int c = c0 + q * 32 + lane;
+                if (c < c1)
+                    xs[c - c0] = bf16_bits_to_float(__ldg(p.x + c));
+            }
             const uint32_t m = run_bits(q);
             if (lane == 0)
                 scan[q] = __popc(m);
@@ -145,6 +154,8 @@ __device__ int build_rows(const KParams &kp, int split, int32_t *ridx, float *rx
                 for (int r = 0; r < q; ++r)
                     pos += scan[r];
                 ridx[pos] = c0 + q * 32 + lane;
+                if (FILL_X)
+                    rx[pos] = xs[q * 32 + lane];
             }
         }
         __syncthreads();
@@ -258,14 +269,15 @@ __host__ __device__ constexpr int code_shift(int o)
 }
 
 struct Smem1 {
-    size_t ring, szs, rxh, ridx, rx, scan, total;
+    size_t ring, szs, rxh, ridx, rx, scan, xs, total;
 };
 
 // ring: each warp's kStages1 rows of 512 B (4 KB), which also holds the warp's
 // partial tile once the warp is done. szs: the (s, z) fp16 pairs of the staged
 // groups, 1024 words per group, lane l's 8 chunks of 4 words swizzled as
 // part_chunk(l, c). ridx: the CTA's rows (channels). rx: x of each row. rxh:
-// x' = x 2^S of each row as fp16.
+// x' = x 2^S of each row as fp16. xs: x of the CTA's channel slice (bitmask
+// rows only).
 __host__ __device__ inline Smem1 smem1_layout(int span_cap, int rows_cap)
 {
     Smem1 s;
@@ -275,7 +287,8 @@ __host__ __device__ inline Smem1 smem1_layout(int span_cap, int rows_cap)
     s.rx = s.ridx + (size_t)rows_cap * 4;
     s.scan = s.rx + (size_t)rows_cap * 4;
     s.rxh = s.scan + (size_t)((rows_cap + 31) / 32 + 4) * 4;
-    s.total = s.rxh + ((size_t)rows_cap * 2 + 15) / 16 * 16;
+    s.xs = s.rxh + ((size_t)rows_cap * 2 + 15) / 16 * 16;
+    s.total = s.xs + (size_t)rows_cap * 4;
     return s;
 }
 
@@ -393,7 +406,9 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
     grid_dependency_wait(); // x, idx, count may come from the previous kernel
 
     // Rows; invalid list entries become row 0 with x = 0 (below).
-    const int nr = build_rows<SRC, kThreads1>(kp, split, ridx, rx, scan); // ends with a barrier
+    const int nr = build_rows<SRC, kThreads1, true>(kp, split, ridx, rx, scan,
+                                                    reinterpret_cast<float *>(smem + L.xs));
+    // (build_rows ends with a barrier)
 
     if (SRC == ROWS_LIST) {
         if (nr > 0) {
@@ -421,7 +436,7 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
     // x of this warp's rows (list / dense paths, after the weights are in
     // flight), and the rows made >= 0 (an invalid list entry reads row 0 with
     // x = 0).
-    if (SRC != ROWS_THRESH) {
+    if (SRC == ROWS_LIST || SRC == ROWS_DENSE) {
         for (int j = lane; j < n; j += 32) {
             const int k = ridx[wa + j];
             rx[wa + j] = (k >= 0) ? bf16_bits_to_float(__ldg(p.x + k)) : 0.f;

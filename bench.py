@@ -233,6 +233,13 @@ class Replica:
         self.y = torch.empty(1, N, dtype=torch.bfloat16, device="cuda")
         self.ws = sgq.alloc_workspace(N, K, 1)
         self.sidx, self.scnt = sgq.alloc_select(K)
+        # per-copy bitmasks (for timing the mask GEMV alone) and a scratch mask
+        self.mask = []
+        for r in range(self.R):
+            m = sgq.alloc_mask(K)
+            sgq.sgq_select_mask(self.x[r], 1, K, [self.t[r]], m)
+            self.mask.append(m)
+        self.smask = sgq.alloc_mask(K)
 
     def step(self, r: int, path: str):
         """One pass of the hot path on copy r (kernels launched: 2 or 1)."""
@@ -240,6 +247,10 @@ class Replica:
             sgq.sgq_select(self.x[r], 1, K, [self.t[r]], self.sidx, self.scnt)
             sgq.sgq_gemv(self.qw[r], self.sz[r], N, K, GROUP, self.x[r], 1, self.sidx,
                          self.scnt, self.y, None, self.ws)
+        elif path == "mask":
+            sgq.sgq_select_mask(self.x[r], 1, K, [self.t[r]], self.smask)
+            sgq.sgq_gemv_mask(self.qw[r], self.sz[r], N, K, GROUP, self.x[r], 1, self.smask,
+                              self.y, None, self.ws)
         else:
             sgq.sgq_gemv_thresh(self.qw[r], self.sz[r], N, K, GROUP, self.x[r], self.t[r],
                                 self.y, None, self.ws)
@@ -256,6 +267,11 @@ class Replica:
                                 self.y, None, self.ws)
         elif which == "select":
             sgq.sgq_select(self.x[r], 1, K, [self.t[r]], self.sidx, self.scnt)
+        elif which == "mask":
+            sgq.sgq_gemv_mask(self.qw[r], self.sz[r], N, K, GROUP, self.x[r], 1, self.mask[r],
+                              self.y, None, self.ws)
+        elif which == "select_mask":
+            sgq.sgq_select_mask(self.x[r], 1, K, [self.t[r]], self.smask)
 
 
 class GraphRunner:
@@ -327,7 +343,9 @@ def run_ours(args, dist: Dist):
     path = args.path
     if path == "auto":
         path = "thresh"
-    kernels_per_step = 2 if path == "list" else 1
+    # kernels per step: every GEMV call is the GEMV kernel plus its split-K
+    # epilogue kernel; the list and mask paths add their select kernel
+    kernels_per_step = {"thresh": 2, "list": 3, "mask": 3}[path]
     period = R * max(1, 64 // R)
 
     # warm-up (untimed) then exactly K timed steps
@@ -356,13 +374,15 @@ def run_ours(args, dist: Dist):
     us_per_gemv = ms * 1e3 / args.steps
 
     # the dominant kernel alone, same rotation, for the roofline
-    dom = "thresh" if path == "thresh" else "gemv"
+    dom = {"thresh": "thresh", "list": "gemv", "mask": "mask"}[path]
     nk = max(args.steps, 2 * R)
     kms = time_calls(lambda i: rep.kernel_only(i % R, dom), nk, period)
     k_us = kms * 1e3 / nk
     k_bytes = sum(rep.abytes[i % R] for i in range(nk)) / nk
     if dom == "thresh":   # reads all of x, no index list
         k_bytes = k_bytes - 6 * np.mean(rep.active) + 2 * K
+    elif dom == "mask":   # K/8 bytes of mask instead of the 4a-byte index list
+        k_bytes = k_bytes - 4 * np.mean(rep.active) + K // 8
     peak, peak_kind = measured_peak()
     achieved = k_bytes / (k_us * 1e-6) / 1e9
     src = source_hash("gemv.cu", "sgq_device.cuh")
@@ -370,11 +390,17 @@ def run_ours(args, dist: Dist):
                 "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
                 "traffic": profiled_traffic(dom, src), "kernel": f"sgq_{dom}",
                 "kernel_us": round(k_us, 3), "algorithmic_bytes": int(k_bytes),
-                "frac_of_8TBps": round(achieved / 8000.0, 4)}
+                "frac_of_8TBps": round(achieved / 8000.0, 4),
+                "timed": "the GEMV call on its stream (GEMV kernel + split-K epilogue kernel)"}
 
     # comparison points on the same rotation: dense int4 GEMV, select alone
-    dense_ms = time_calls(lambda i: rep.kernel_only(i % R, "dense"), 2 * period, period)
-    sel_ms = time_calls(lambda i: rep.kernel_only(i % R, "select"), 2 * period, period)
+    nc = max(min(args.steps, 4000), 2 * period)
+    dense_ms = time_calls(lambda i: rep.kernel_only(i % R, "dense"), nc, period)
+    sel_ms = time_calls(lambda i: rep.kernel_only(i % R, "select"), nc, period)
+    cmp_us = {}
+    for name in ("gemv", "thresh", "mask", "select_mask"):
+        cms = time_calls(lambda i: rep.kernel_only(i % R, name), nc, period)
+        cmp_us[name] = round(cms * 1e3 / nc, 3)
 
     e2e = run_e2e(rep, path, min(args.steps, 2000), args.warmup, dist)
     layer = None if args.no_ffn else run_layer()
@@ -386,15 +412,20 @@ def run_ours(args, dist: Dist):
         "data": "synthetic (seeded; weights N(0,0.02), x = SiLU(g)*u)",
         "config": {"workload": WORKLOAD, "K": K, "N": N, "group": GROUP, "batch": 1,
                    "sparsity": args.sparsity, "active_channels": int(np.mean(rep.active)),
-                   "path": "select+gemv" if path == "list" else "gemv_thresh (select fused)",
+                   "path": {"list": "select+gemv", "mask": "select_mask+gemv_mask",
+                            "thresh": "gemv_thresh (select fused)"}[path],
                    "l2": f"inputs larger than L2: {R} rotating weight copies, "
                          f"{rep.bytes_resident / 1e6:.0f} MB vs L2 {rep.l2 / 1e6:.0f} MB",
                    "parallelism": f"replicas x{dist.world}" if dist.world > 1 else "single GPU"},
         "us_per_gemv": round(us_per_gemv, 3),
         "active_bytes_per_gemv": int(np.mean(rep.abytes)),
         "roofline": roofline,
-        "dense_int4_gemv_us": round(dense_ms * 1e3 / (2 * period), 3),
-        "select_us": round(sel_ms * 1e3 / (2 * period), 3),
+        "dense_int4_gemv_us": round(dense_ms * 1e3 / nc, 3),
+        "select_us": round(sel_ms * 1e3 / nc, 3),
+        "call_us": {"gemv_list": cmp_us["gemv"], "gemv_thresh": cmp_us["thresh"],
+                    "gemv_mask": cmp_us["mask"], "select_mask": cmp_us["select_mask"],
+                    "note": "one C-ABI call each on the same rotation; a GEMV call is the "
+                            "GEMV kernel plus its split-K epilogue kernel"},
         "e2e": e2e,
         "gpu_launches": args.steps * kernels_per_step,
         "clocks": clk.summary(),
@@ -421,6 +452,10 @@ def run_e2e(rep: Replica, path: str, steps: int, warmup: int, dist: Dist):
             sgq.sgq_select(xd, 1, K, [rep.t[r]], rep.sidx, rep.scnt)
             sgq.sgq_gemv(rep.qw[r], rep.sz[r], N, K, GROUP, xd, 1, rep.sidx, rep.scnt, rep.y,
                          None, rep.ws)
+        elif path == "mask":
+            sgq.sgq_select_mask(xd, 1, K, [rep.t[r]], rep.smask)
+            sgq.sgq_gemv_mask(rep.qw[r], rep.sz[r], N, K, GROUP, xd, 1, rep.smask, rep.y, None,
+                              rep.ws)
         else:
             sgq.sgq_gemv_thresh(rep.qw[r], rep.sz[r], N, K, GROUP, xd, rep.t[r], rep.y, None,
                                 rep.ws)
@@ -675,7 +710,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--path", choices=["auto", "list", "thresh"], default="auto")
+    ap.add_argument("--path", choices=["auto", "list", "thresh", "mask"], default="auto")
     ap.add_argument("--sparsity", type=float, default=0.5)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
