@@ -12,25 +12,26 @@
 // and at these sizes the whole GEMV is about one latency-bandwidth product of
 // HBM, so the kernel's job is to have nearly all of its bytes in flight early
 // and to keep the arithmetic under the memory time:
-//  * Outputs are cut into tiles (1024 outputs = 512 bytes of a packed row for
-//    B = 1; 256 outputs for B > 1); the rows (active channels) of each tile into
-//    k_splits shares so that n_tiles * k_splits CTAs cover the SMs.
+//  * Outputs are cut into tiles of 1024 (512 bytes of a packed row); the rows
+//    (active channels) of each tile into k_splits shares so that
+//    n_tiles * k_splits CTAs cover the SMs.
 //  * Scale/zero of the CTA's groups are prefetched first; in the threshold
 //    path (select fused into the prologue) their span is known from the CTA's
 //    channel slice, before x is read.
 //  * Each warp takes a contiguous slice of the CTA's rows; every lane streams
-//    its own 16-byte (B = 1) or 4-byte (B > 1) column of each row through a
-//    per-lane ring in shared memory with cp.async (8 rows ahead for B = 1). A
-//    lane reads back only bytes it copied itself: no barrier, only its own
-//    groups.
-//  * B = 1: codes are summed per group without dequantizing
+//    its own 16-byte column of each row through a per-lane ring in shared
+//    memory with cp.async, 8 rows ahead. A lane reads back only bytes it
+//    copied itself: no barrier, only its own groups.
+//  * Codes are summed per group without dequantizing
 //    (sum s (q - z) x = s (sum q x - z sum x)). One 32-bit AND takes two codes
 //    into the two halves of an fp16 pair, where they read as exact fp16
 //    subnormals; a mixed-precision FMA (fp16 x fp16 + fp32) multiplies each by
 //    x held in fp16 under a per-warp power-of-two scale, so every product is
 //    exact. Scale and zero are applied once per (group, output) in a fold.
-//  * B > 1: each code is dequantized exactly (one LOP3, one FMA, one add) and
-//    multiplied into B accumulators with packed f32x2 FMAs.
+//  * B > 1: each warp carries two batch rows, which share the extracted codes;
+//    the warps form ceil(B / 2) (rounded to a power of two) batch groups that
+//    read the same rows, the later reads hitting L2, so HBM still sees each
+//    active row once.
 //  * Split-K: each warp leaves its partial tile in its own (drained) ring
 //    region; after one barrier the CTA sums the warps' tiles (no shared
 //    atomics: many-way float atomics on the same addresses serialize) and adds
@@ -51,8 +52,6 @@ namespace {
 
 constexpr int kTileN1 = 1024;            // B = 1: outputs per tile, 32 per lane
 constexpr int kRowBytes1 = kTileN1 / 2;  // bytes of one packed row per tile
-constexpr int kTileNB = 256;             // B > 1: outputs per tile, 8 per lane
-constexpr int kRowBytesB = kTileNB / 2;
 
 struct KParams {
     GemvProblem p;
@@ -61,6 +60,7 @@ struct KParams {
     int rows_cap;  // capacity of the per-CTA row arrays
     int span_cap;  // groups of scale/zero staged in shared memory per CTA
     int lg;        // log2(group)
+    int nb;        // batch groups of warps (1 for B = 1)
 };
 
 __device__ __forceinline__ int warp_max_exponent(float m)
@@ -250,12 +250,23 @@ __global__ void __launch_bounds__(256) finalize_kernel(GemvProblem p)
 }
 
 // ---------------------------------------------------------------------------
-// B = 1
+// The GEMV kernel, 1 <= B <= 16
 // ---------------------------------------------------------------------------
 
 constexpr int kWarps1 = 8;
 constexpr int kThreads1 = kWarps1 * 32;
 constexpr int kStages1 = 8; // rows in flight per warp (power of two); deeper rings measured slower
+
+// Batch rows per warp: 1 for B = 1, 2 for B > 1 (the codes a lane extracts
+// from a row serve both). With B > 1 the warps form kp.nb batch groups of
+// kWarps1 / nb warps; each group covers BW batch rows and reads the same rows
+// as the other groups (the later reads hit L2).
+__host__ __device__ constexpr int warp_region_bytes(int bw)
+{
+    // a warp's ring, which also holds its partial tiles (BW x 1024 floats)
+    return (kStages1 * kRowBytes1 > bw * kTileN1 * 4) ? kStages1 * kRowBytes1
+                                                      : bw * kTileN1 * 4;
+}
 
 // Output o (0..31) of a lane is code o % 8 of packed word o / 8. One 32-bit AND
 // takes two codes of a word at once, one into each fp16 half: the masked half
@@ -272,22 +283,22 @@ struct Smem1 {
     size_t ring, szs, rxh, ridx, rx, scan, xs, total;
 };
 
-// ring: each warp's kStages1 rows of 512 B (4 KB), which also holds the warp's
-// partial tile once the warp is done. szs: the (s, z) fp16 pairs of the staged
-// groups, 1024 words per group, lane l's 8 chunks of 4 words swizzled as
-// part_chunk(l, c). ridx: the CTA's rows (channels). rx: x of each row. rxh:
-// x' = x 2^S of each row as fp16. xs: x of the CTA's channel slice (bitmask
-// rows only).
-__host__ __device__ inline Smem1 smem1_layout(int span_cap, int rows_cap)
+// ring: each warp's region (its kStages1 rows of 512 B, then its partial
+// tiles). szs: the (s, z) fp16 pairs of the staged groups, 1024 words per
+// group, lane l's 8 chunks of 4 words swizzled as part_chunk(l, c). ridx: the
+// CTA's rows (channels). rx: x of each row, per batch row b at b * rows_cap.
+// rxh: x' = x 2^S of each row as fp16, same indexing. xs: x of the CTA's
+// channel slice (bitmask rows, batch 1). bp = batch rows padded to nb * BW.
+__host__ __device__ inline Smem1 smem1_layout(int span_cap, int rows_cap, int bp, int bw)
 {
     Smem1 s;
     s.ring = 0;
-    s.szs = s.ring + (size_t)kWarps1 * kStages1 * kRowBytes1;
+    s.szs = s.ring + (size_t)kWarps1 * warp_region_bytes(bw);
     s.ridx = s.szs + (size_t)span_cap * kTileN1 * 4;
     s.rx = s.ridx + (size_t)rows_cap * 4;
-    s.scan = s.rx + (size_t)rows_cap * 4;
+    s.scan = s.rx + (size_t)rows_cap * bp * 4;
     s.rxh = s.scan + (size_t)((rows_cap + 31) / 32 + 4) * 4;
-    s.xs = s.rxh + ((size_t)rows_cap * 2 + 15) / 16 * 16;
+    s.xs = s.rxh + ((size_t)rows_cap * bp * 2 + 15) / 16 * 16;
     s.total = s.xs + (size_t)rows_cap * 4;
     return s;
 }
@@ -323,13 +334,61 @@ __device__ __forceinline__ void mac_word(uint32_t w, uint16_t xh, float *a)
         : "r"(w), "h"(xh));
 }
 
-// One row (16 bytes = 4 words of this lane) into the 32 group accumulators.
-__device__ __forceinline__ void mac_row(const uint4 &v, uint16_t xh, float *accg)
+// The same for two batch rows: one extraction, sixteen FMAs.
+__device__ __forceinline__ void mac_word2(uint32_t w, uint16_t x0, uint16_t x1, float *a,
+                                          float *b)
 {
-    mac_word(v.x, xh, accg);
-    mac_word(v.y, xh, accg + 8);
-    mac_word(v.z, xh, accg + 16);
-    mac_word(v.w, xh, accg + 24);
+    asm("{\n\t"
+        ".reg .b32 h, p;\n\t"
+        ".reg .f16 lo, hi;\n\t"
+        "mul.hi.u32 h, %16, 16777216;\n\t"
+        "and.b32 p, %16, 0x000F000F;\n\t"
+        "mov.b32 {lo, hi}, p;\n\t"
+        "fma.rn.f32.f16 %0, lo, %17, %0;\n\t"
+        "fma.rn.f32.f16 %4, hi, %17, %4;\n\t"
+        "fma.rn.f32.f16 %8, lo, %18, %8;\n\t"
+        "fma.rn.f32.f16 %12, hi, %18, %12;\n\t"
+        "and.b32 p, %16, 0x00F000F0;\n\t"
+        "mov.b32 {lo, hi}, p;\n\t"
+        "fma.rn.f32.f16 %1, lo, %17, %1;\n\t"
+        "fma.rn.f32.f16 %5, hi, %17, %5;\n\t"
+        "fma.rn.f32.f16 %9, lo, %18, %9;\n\t"
+        "fma.rn.f32.f16 %13, hi, %18, %13;\n\t"
+        "and.b32 p, h, 0x000F000F;\n\t"
+        "mov.b32 {lo, hi}, p;\n\t"
+        "fma.rn.f32.f16 %2, lo, %17, %2;\n\t"
+        "fma.rn.f32.f16 %6, hi, %17, %6;\n\t"
+        "fma.rn.f32.f16 %10, lo, %18, %10;\n\t"
+        "fma.rn.f32.f16 %14, hi, %18, %14;\n\t"
+        "and.b32 p, h, 0x00F000F0;\n\t"
+        "mov.b32 {lo, hi}, p;\n\t"
+        "fma.rn.f32.f16 %3, lo, %17, %3;\n\t"
+        "fma.rn.f32.f16 %7, hi, %17, %7;\n\t"
+        "fma.rn.f32.f16 %11, lo, %18, %11;\n\t"
+        "fma.rn.f32.f16 %15, hi, %18, %15;\n\t"
+        "}"
+        : "+f"(a[0]), "+f"(a[1]), "+f"(a[2]), "+f"(a[3]), "+f"(a[4]), "+f"(a[5]), "+f"(a[6]),
+          "+f"(a[7]), "+f"(b[0]), "+f"(b[1]), "+f"(b[2]), "+f"(b[3]), "+f"(b[4]), "+f"(b[5]),
+          "+f"(b[6]), "+f"(b[7])
+        : "r"(w), "h"(x0), "h"(x1));
+}
+
+// One row (16 bytes = 4 words of this lane) into the group accumulators of
+// the warp's BW batch rows.
+template <int BW>
+__device__ __forceinline__ void mac_row(const uint4 &v, const uint16_t *xh, float (*accg)[32])
+{
+    if (BW == 1) {
+        mac_word(v.x, xh[0], accg[0]);
+        mac_word(v.y, xh[0], accg[0] + 8);
+        mac_word(v.z, xh[0], accg[0] + 16);
+        mac_word(v.w, xh[0], accg[0] + 24);
+    } else {
+        mac_word2(v.x, xh[0], xh[1], accg[0], accg[BW - 1]);
+        mac_word2(v.y, xh[0], xh[1], accg[0] + 8, accg[BW - 1] + 8);
+        mac_word2(v.z, xh[0], xh[1], accg[0] + 16, accg[BW - 1] + 16);
+        mac_word2(v.w, xh[0], xh[1], accg[0] + 24, accg[BW - 1] + 24);
+    }
 }
 
 __device__ __forceinline__ float half_lo(uint32_t w)
@@ -351,18 +410,20 @@ __device__ __forceinline__ int part_chunk(int l, int c)
     return 8 * l + (c ^ (l & 7));
 }
 
-template <int SRC>
-__global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
+template <int SRC, int BW>
+__global__ void __launch_bounds__(kThreads1, 1) gemv_kernel(const KParams kp)
 {
     extern __shared__ __align__(16) uint8_t smem[];
     const GemvProblem &p = kp.p;
-    const Smem1 L = smem1_layout(kp.span_cap, kp.rows_cap);
+    const int bp = kp.nb * BW; // batch rows padded to whole groups
+    const Smem1 L = smem1_layout(kp.span_cap, kp.rows_cap, bp, BW);
     uint8_t *ring = smem + L.ring;
     const uint4 *szs = reinterpret_cast<const uint4 *>(smem + L.szs);
     int32_t *ridx = reinterpret_cast<int32_t *>(smem + L.ridx);
     float *rx = reinterpret_cast<float *>(smem + L.rx);
     uint16_t *rxh = reinterpret_cast<uint16_t *>(smem + L.rxh);
     int *scan = reinterpret_cast<int *>(smem + L.scan);
+    const int rcap = kp.rows_cap;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int tile = blockIdx.x % kp.n_tiles;
@@ -376,8 +437,8 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
 
     // Scale/zero of the CTA's groups, staged asynchronously (the oldest
     // cp.async group of every thread). With a fixed channel slice (threshold /
-    // dense) the groups are known now, so the copies start before waiting on
-    // the previous kernel; with an index list they follow the list.
+    // mask / dense) the groups are known now, so the copies start before
+    // waiting on the previous kernel; with an index list they follow the list.
     int G0 = 0, span = 0;
     auto stage_sz = [&]() {
         for (int c = tid; c < span * (kTileN1 / 4); c += kThreads1) {
@@ -403,61 +464,74 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
         stage_sz();
     }
 
-    grid_dependency_wait(); // x, idx, count may come from the previous kernel
+    grid_dependency_wait(); // x, idx, count, mask may come from the previous kernel
 
-    // Rows; invalid list entries become row 0 with x = 0 (below).
-    const int nr = build_rows<SRC, kThreads1, true>(kp, split, ridx, rx, scan,
-                                                    reinterpret_cast<float *>(smem + L.xs));
-    // (build_rows ends with a barrier)
+    // Rows (build_rows ends with a barrier). Invalid list entries stay -1: they
+    // are read as row 0 with x = 0, so they add nothing.
+    const int nr = build_rows<SRC, kThreads1, (BW == 1)>(kp, split, ridx, rx, scan,
+                                                         reinterpret_cast<float *>(smem + L.xs));
+    auto row = [&](int j) { return (SRC == ROWS_LIST) ? max(ridx[j], 0) : ridx[j]; };
 
     if (SRC == ROWS_LIST) {
         if (nr > 0) {
-            const int kf = max(ridx[0], 0), kl = max(ridx[nr - 1], 0);
+            const int kf = row(0), kl = row(nr - 1);
             G0 = kf >> lg;
             span = min(max((kl >> lg) - G0 + 1, 1), kp.span_cap);
         }
         stage_sz(); // stays the oldest cp.async group
     }
 
-    // This warp's contiguous slice of the CTA's rows.
-    const int wa = (int)((long long)nr * warp / kWarps1);
-    const int n = (int)((long long)nr * (warp + 1) / kWarps1) - wa;
+    // This warp's batch rows and its contiguous slice of the CTA's rows.
+    const int wpg = (BW == 1) ? kWarps1 : kWarps1 / kp.nb;
+    const int b0 = (BW == 1) ? 0 : (warp / wpg) * BW;
+    const int wq = (BW == 1) ? warp : warp % wpg;
+    const int nbw = (BW == 1) ? 1 : max(0, min(BW, p.B - b0)); // real batch rows of this warp
+    const int wa = (int)((long long)nr * wq / wpg);
+    const int n = (nbw > 0) ? (int)((long long)nr * (wq + 1) / wpg) - wa : 0;
 
     // Ring prologue. Lanes past N read column 0 (valid memory, result unused).
     const uint8_t *wcol = p.qweight + (lane_ok ? ((size_t)n0 / 2 + lane * 16) : 0);
-    uint8_t *myring = ring + (size_t)warp * kStages1 * kRowBytes1 + lane * 16;
+    uint8_t *region = ring + (size_t)warp * warp_region_bytes(BW);
+    uint8_t *myring = region + lane * 16;
 #pragma unroll
     for (int s = 0; s < kStages1; ++s) {
         if (s < n)
-            cp_async16(myring + s * kRowBytes1, wcol + (size_t)max(ridx[wa + s], 0) * row_stride);
+            cp_async16(myring + s * kRowBytes1, wcol + (size_t)row(wa + s) * row_stride);
         cp_async_commit();
     }
 
-    // x of this warp's rows (list / dense paths, after the weights are in
-    // flight), and the rows made >= 0 (an invalid list entry reads row 0 with
-    // x = 0).
-    if (SRC == ROWS_LIST || SRC == ROWS_DENSE) {
-        for (int j = lane; j < n; j += 32) {
+    // x of this warp's rows and batch rows (after the weights are in flight),
+    // unless build_rows already read it (threshold; bitmask at batch 1).
+    // Padded batch rows and invalid list entries get x = 0.
+    if (!(SRC == ROWS_THRESH || (SRC == ROWS_MASK && BW == 1))) {
+        for (int e = lane; e < n * BW; e += 32) {
+            const int j = e / BW, bb = e - j * BW;
             const int k = ridx[wa + j];
-            rx[wa + j] = (k >= 0) ? bf16_bits_to_float(__ldg(p.x + k)) : 0.f;
-            ridx[wa + j] = max(k, 0);
+            rx[(b0 + bb) * rcap + wa + j] =
+                (k >= 0 && bb < nbw) ? bf16_bits_to_float(__ldg(p.x + (size_t)(b0 + bb) * p.K + k))
+                                     : 0.f;
         }
         __syncwarp();
     }
 
-    // x' = x 2^S in fp16 with 2^14 <= max |x'| < 2^15 over the warp's rows:
-    // exact for every |x| >= 2^-28 max |x| (fp16 normals); smaller x round on
-    // the fp16 subnormal grid, an error below 2^-39 max |x'|. Each product
-    // q 2^-24 x' (or q 2^-20 x') is then exact in fp32.
-    float m = 0.f;
-    for (int j = lane; j < n; j += 32)
-        m = fmaxf(m, fabsf(rx[wa + j]));
-    const int e = warp_max_exponent(m);
-    const int S = (e == INT32_MIN) ? 0 : 14 - e;
-    {
-        const float fa = pow2f(S - S / 2), fb = pow2f(S / 2);
+    // Per batch row: x' = x 2^S in fp16 with 2^14 <= max |x'| < 2^15 over the
+    // warp's rows: exact for every |x| >= 2^-28 max |x| (fp16 normals);
+    // smaller x round on the fp16 subnormal grid, an error below
+    // 2^-39 max |x'|. Each product q 2^-24 x' (or q 2^-20 x') is then exact in
+    // fp32.
+    int S[BW];
+#pragma unroll
+    for (int bb = 0; bb < BW; ++bb) {
+        const float *xr = rx + (b0 + bb) * rcap;
+        uint16_t *hr = rxh + (b0 + bb) * rcap;
+        float m = 0.f;
         for (int j = lane; j < n; j += 32)
-            rxh[wa + j] = __half_as_ushort(__float2half_rn((rx[wa + j] * fa) * fb));
+            m = fmaxf(m, fabsf(xr[wa + j]));
+        const int e = warp_max_exponent(m);
+        S[bb] = (e == INT32_MIN) ? 0 : 14 - e;
+        const float fa = pow2f(S[bb] - S[bb] / 2), fb = pow2f(S[bb] / 2);
+        for (int j = lane; j < n; j += 32)
+            hr[wa + j] = __half_as_ushort(__float2half_rn((xr[wa + j] * fa) * fb));
     }
     __syncwarp();
     // The staged scale/zero (every thread's oldest cp.async group) have landed
@@ -465,17 +539,19 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
     cp_async_wait<kStages1>();
     __syncthreads();
 
-    // accg[o] = this group's sum of q x' 2^-code_shift(o); acc[o] = folded
-    // result in units of 2^-S.
-    float accg[32], acc[32];
+    // accg[bb][o] = this group's sum of q x' 2^-code_shift(o); acc[bb][o] =
+    // folded result in units of 2^-S.
+    float accg[BW][32], acc[BW][32];
 #pragma unroll
-    for (int o = 0; o < 32; ++o) {
-        accg[o] = 0.f;
-        acc[o] = 0.f;
-    }
+    for (int bb = 0; bb < BW; ++bb)
+#pragma unroll
+        for (int o = 0; o < 32; ++o) {
+            accg[bb][o] = 0.f;
+            acc[bb][o] = 0.f;
+        }
 
     //   acc += s * (2^code_shift accg - z * sum x')
-    auto fold = [&](int G, float Xg) {
+    auto fold = [&](int G, const float *Xg) {
         const bool staged = (G >= G0) && (G < G0 + span);
         uint32_t w[32]; // (s, z) of this lane's 32 outputs
         if (staged) {
@@ -501,10 +577,20 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
         }
 #pragma unroll
         for (int o = 0; o < 32; ++o) {
-            const float t = accg[o] * pow2f(code_shift(o));
-            acc[o] = fmaf(half_lo(w[o]), fmaf(-half_hi(w[o]), Xg, t), acc[o]);
-            accg[o] = 0.f;
+            const float s = half_lo(w[o]), z = half_hi(w[o]);
+#pragma unroll
+            for (int bb = 0; bb < BW; ++bb) {
+                const float t = accg[bb][o] * pow2f(code_shift(o));
+                acc[bb][o] = fmaf(s, fmaf(-z, Xg[bb], t), acc[bb][o]);
+                accg[bb][o] = 0.f;
+            }
         }
+    };
+
+    auto xrow = [&](int j, uint16_t *xh) {
+#pragma unroll
+        for (int bb = 0; bb < BW; ++bb)
+            xh[bb] = rxh[(b0 + bb) * rcap + wa + j];
     };
 
     // Runs of rows of one group: the run end comes from one ballot per 32
@@ -512,38 +598,49 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
     // is the ring read, the codes and the refill only.
     int i = 0;
     while (i < n) {
-        const int G = ridx[wa + i] >> lg;
+        const int G = row(wa + i) >> lg;
         int i1 = i;
-        float Xg = 0.f;
+        float Xg[BW];
+#pragma unroll
+        for (int bb = 0; bb < BW; ++bb)
+            Xg[bb] = 0.f;
         for (;;) {
             const int j = i1 + lane;
-            const bool in = (j < n) && ((ridx[wa + j] >> lg) == G);
+            const bool in = (j < n) && ((row(wa + j) >> lg) == G);
             const uint32_t bal = __ballot_sync(0xffffffffu, in);
             const int len = (bal == 0xffffffffu) ? 32 : (__ffs(~bal) - 1);
-            if (lane < len)
-                Xg += __half2float(__ushort_as_half(rxh[wa + j]));
+            if (lane < len) {
+#pragma unroll
+                for (int bb = 0; bb < BW; ++bb)
+                    Xg[bb] += __half2float(__ushort_as_half(rxh[(b0 + bb) * rcap + wa + j]));
+            }
             i1 += len;
             if (len < 32)
                 break;
         }
 #pragma unroll
-        for (int d = 16; d > 0; d >>= 1)
-            Xg += __shfl_xor_sync(0xffffffffu, Xg, d);
+        for (int bb = 0; bb < BW; ++bb)
+#pragma unroll
+            for (int d = 16; d > 0; d >>= 1)
+                Xg[bb] += __shfl_xor_sync(0xffffffffu, Xg[bb], d);
 
         for (; i + 1 < i1; i += 2) {
             cp_async_wait<kStages1 - 2>(); // rows i and i + 1 have landed
             const int slot = i & (kStages1 - 1), slot1 = (i + 1) & (kStages1 - 1);
             const uint4 v0 = *reinterpret_cast<const uint4 *>(myring + slot * kRowBytes1);
             const uint4 v1 = *reinterpret_cast<const uint4 *>(myring + slot1 * kRowBytes1);
-            mac_row(v0, rxh[wa + i], accg);
-            mac_row(v1, rxh[wa + i + 1], accg);
+            uint16_t xh0[BW], xh1[BW];
+            xrow(i, xh0);
+            xrow(i + 1, xh1);
+            mac_row<BW>(v0, xh0, accg);
+            mac_row<BW>(v1, xh1, accg);
             if (i + kStages1 < n)
                 cp_async16(myring + slot * kRowBytes1,
-                           wcol + (size_t)ridx[wa + i + kStages1] * row_stride);
+                           wcol + (size_t)row(wa + i + kStages1) * row_stride);
             cp_async_commit();
             if (i + 1 + kStages1 < n)
                 cp_async16(myring + slot1 * kRowBytes1,
-                           wcol + (size_t)ridx[wa + i + 1 + kStages1] * row_stride);
+                           wcol + (size_t)row(wa + i + 1 + kStages1) * row_stride);
             cp_async_commit();
         }
         if (i < i1) {
@@ -551,44 +648,47 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
             cp_async_wait<kStages1 - 1>();
             const int slot = i & (kStages1 - 1);
             const uint4 v = *reinterpret_cast<const uint4 *>(myring + slot * kRowBytes1);
-            mac_row(v, rxh[wa + i], accg);
+            uint16_t xh[BW];
+            xrow(i, xh);
+            mac_row<BW>(v, xh, accg);
             if (i + kStages1 < n)
                 cp_async16(myring + slot * kRowBytes1,
-                           wcol + (size_t)ridx[wa + i + kStages1] * row_stride);
+                           wcol + (size_t)row(wa + i + kStages1) * row_stride);
             cp_async_commit();
             ++i;
         }
         fold(G, Xg);
     }
 
-    // This warp's partial tile, in real units (x 2^-S, two exact factors),
-    // into its own ring region: every cp.async of this warp has landed and
-    // been read, so nothing else touches that region any more.
+    // This warp's partial tiles, in real units (x 2^-S, two exact factors),
+    // into its own region: every cp.async of this warp has landed and been
+    // read, so nothing else touches that region any more.
     cp_async_wait_all();
     __syncwarp();
-    {
-        float4 *part = reinterpret_cast<float4 *>(ring + (size_t)warp * kStages1 * kRowBytes1);
-        const int E = -S;
-        const float f1 = pow2f(E / 2), f2 = pow2f(E - E / 2);
-        const bool live = lane_ok && n > 0;
-        float out[32];
 #pragma unroll
-        for (int o = 0; o < 32; ++o)
-            out[o] = (acc[o] * f1) * f2;
+    for (int bb = 0; bb < BW; ++bb) {
+        float4 *part = reinterpret_cast<float4 *>(region) + bb * (kTileN1 / 4);
+        const int E = -S[bb];
+        const float f1 = pow2f(E / 2), f2 = pow2f(E - E / 2);
+        const bool live = lane_ok && n > 0 && bb < nbw;
 #pragma unroll
         for (int c = 0; c < 8; ++c)
-            part[part_chunk(lane, c)] = live ? make_float4(out[4 * c], out[4 * c + 1],
-                                                           out[4 * c + 2], out[4 * c + 3])
-                                             : make_float4(0.f, 0.f, 0.f, 0.f);
+            part[part_chunk(lane, c)] =
+                live ? make_float4((acc[bb][4 * c] * f1) * f2, (acc[bb][4 * c + 1] * f1) * f2,
+                                   (acc[bb][4 * c + 2] * f1) * f2, (acc[bb][4 * c + 3] * f1) * f2)
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();
-    if (tid < kTileN1 / 4) {
+    // Each thread owns one chunk of 4 outputs of the tile; for every batch row
+    // it sums the partial tiles of the warps of that row's group and adds the
+    // sum into the workspace.
+    if (BW == 1) {
         const int l = tid >> 3, c = tid & 7;
         float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int w = 0; w < kWarps1; ++w) {
             const float4 u = reinterpret_cast<const float4 *>(
-                ring + (size_t)w * kStages1 * kRowBytes1)[part_chunk(l, c)];
+                ring + (size_t)w * warp_region_bytes(BW))[part_chunk(l, c)];
             v.x += u.x;
             v.y += u.y;
             v.z += u.z;
@@ -596,199 +696,22 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_b1_kernel(const KParams kp)
         }
         if (n0 + 4 * tid < p.N)
             red_add_v4(p.ws_acc + n0 + 4 * tid, v);
-    }
-}
-
-// ---------------------------------------------------------------------------
-// 1 < B <= 16
-// ---------------------------------------------------------------------------
-
-constexpr int kWarpsB = 8;
-constexpr int kThreadsB = kWarpsB * 32;
-constexpr int kStagesB = 32; // 8 warps * 32 * 128 B = 32 KB ring
-
-struct SmemB {
-    size_t ring, szs, red, ridx, rx, scan, total;
-};
-
-__host__ __device__ inline SmemB smemB_layout(int span_cap, int rows_cap, int BT)
-{
-    SmemB s;
-    s.ring = 0;
-    s.szs = s.ring + (size_t)kWarpsB * kStagesB * kRowBytesB;
-    s.red = s.szs + (size_t)span_cap * kTileNB * 4;
-    s.ridx = s.red + (size_t)BT * kTileNB * 4;
-    s.rx = s.ridx + (size_t)rows_cap * 4;
-    s.scan = s.rx + (size_t)rows_cap * BT * 4;
-    s.total = s.scan + (size_t)((rows_cap + 31) / 32 + 4) * 4;
-    return s;
-}
-
-__host__ __device__ constexpr int code_pos(int j)
-{
-    // Bit offset of code j (0..7) of a packed word inside the register it is
-    // extracted from: codes 0..4 from the word itself, 5..7 from word >> 12.
-    return (j < 5) ? 4 * j : 4 * j - 12;
-}
-
-__host__ __device__ constexpr uint32_t code_mask(int j)
-{
-    return 0xFu << code_pos(j);
-}
-
-template <int BT, int SRC>
-__global__ void __launch_bounds__(kThreadsB, 1) gemv_bn_kernel(const KParams kp)
-{
-    extern __shared__ __align__(16) uint8_t smem[];
-    const GemvProblem &p = kp.p;
-    const SmemB L = smemB_layout(kp.span_cap, kp.rows_cap, BT);
-    uint8_t *ring = smem + L.ring;
-    const uint32_t *szs = reinterpret_cast<const uint32_t *>(smem + L.szs);
-    float *red = reinterpret_cast<float *>(smem + L.red);
-    int32_t *ridx = reinterpret_cast<int32_t *>(smem + L.ridx);
-    float *rx = reinterpret_cast<float *>(smem + L.rx);
-    int *scan = reinterpret_cast<int *>(smem + L.scan);
-
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int tile = blockIdx.x % kp.n_tiles;
-    const int split = blockIdx.x / kp.n_tiles;
-    const int n0 = tile * kTileNB;
-    const int lg = kp.lg;
-    const int B = p.B;
-    const size_t row_stride = (size_t)(p.N / 2);
-    const bool lane_ok = (n0 + lane * 8) < p.N;
-
-    grid_launch_dependents();
-    grid_dependency_wait();
-    for (int i = tid; i < BT * kTileNB; i += kThreadsB)
-        red[i] = 0.f;
-
-    const int nr = build_rows<SRC, kThreadsB>(kp, split, ridx, rx, scan);
-
-    const int wa = (int)((long long)nr * warp / kWarpsB);
-    const int n = (int)((long long)nr * (warp + 1) / kWarpsB) - wa;
-
-    int G0 = 0, span = 0;
-    if (nr > 0) {
-        const int kf = max(ridx[0], 0), kl = max(ridx[nr - 1], 0);
-        G0 = kf >> lg;
-        span = min(max((kl >> lg) - G0 + 1, 1), kp.span_cap);
-    }
-    // 256 outputs * 4 bytes = 64 chunks of 16 bytes per group.
-    for (int c = tid; c < span * (kTileNB / 4); c += kThreadsB) {
-        const int r = c / (kTileNB / 4), o = (c % (kTileNB / 4)) * 4;
-        if (n0 + o < p.N)
-            cp_async16(smem + L.szs + ((size_t)r * kTileNB + o) * 4,
-                       p.sz + (size_t)(G0 + r) * p.N + n0 + o);
-    }
-    cp_async_commit();
-
-    const uint8_t *wcol = p.qweight + (lane_ok ? ((size_t)n0 / 2 + lane * 4) : 0);
-    uint8_t *myring = ring + (size_t)warp * kStagesB * kRowBytesB + lane * 4;
-#pragma unroll
-    for (int s = 0; s < kStagesB; ++s) {
-        if (s < n)
-            cp_async4(myring + s * kRowBytesB, wcol + (size_t)max(ridx[wa + s], 0) * row_stride);
-        cp_async_commit();
-    }
-
-    // x of every batch row for this warp's rows: rx[j * BT + b].
-    for (int e2 = lane; e2 < n * BT; e2 += 32) {
-        const int j = e2 / BT, b = e2 % BT;
-        const int k = ridx[wa + j];
-        rx[(size_t)(wa + j) * BT + b] =
-            (k >= 0 && b < B) ? bf16_bits_to_float(__ldg(p.x + (size_t)b * p.K + k)) : 0.f;
-    }
-    __syncwarp();
-
-    float2 acc[BT][4];
-#pragma unroll
-    for (int b = 0; b < BT; ++b)
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-            acc[b][j] = make_float2(0.f, 0.f);
-    // Per-group constants of the 8 outputs: sp = s 2^-p, cb = -2^(23-p) s, zs = z s,
-    // so that fma(2^23 + q 2^p, sp, cb) - zs = (q - z) s exactly.
-    float sp[8], cb[8], zs[8];
-    int curG = -1;
-
-    auto load_group = [&](int G) {
-        const bool staged = (G >= G0) && (G < G0 + span);
-        const uint32_t *src = staged ? (szs + (size_t)(G - G0) * kTileNB + lane * 8)
-                                     : (p.sz + (size_t)G * p.N + n0 + (lane_ok ? lane * 8 : 0));
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            uint4 v4 = staged ? *reinterpret_cast<const uint4 *>(src + 4 * c)
-                              : __ldg(reinterpret_cast<const uint4 *>(src + 4 * c));
-            const uint32_t w4[4] = {v4.x, v4.y, v4.z, v4.w};
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int j = 4 * c + u;
-                const float s = half_lo(w4[u]);
-                const float z = half_hi(w4[u]);
-                sp[j] = s * pow2f(-code_pos(j));
-                cb[j] = -(s * pow2f(23 - code_pos(j)));
-                zs[j] = z * s;
+    } else {
+        const int l = tid >> 3, c = tid & 7;
+        for (int b = 0; b < p.B; ++b) {
+            const int w0 = (b / BW) * wpg, bb = b % BW;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int w = w0; w < w0 + wpg; ++w) {
+                const float4 u = reinterpret_cast<const float4 *>(
+                    ring + (size_t)w * warp_region_bytes(BW))[bb * (kTileN1 / 4) + part_chunk(l, c)];
+                v.x += u.x;
+                v.y += u.y;
+                v.z += u.z;
+                v.w += u.w;
             }
+            if (n0 + 4 * tid < p.N)
+                red_add_v4(p.ws_acc + (size_t)b * p.N + n0 + 4 * tid, v);
         }
-    };
-
-    cp_async_wait<kStagesB>();
-    __syncthreads();
-
-    for (int i = 0; i < n; ++i) {
-        cp_async_wait<kStagesB - 1>();
-        const int slot = i % kStagesB;
-        const uint32_t word = *reinterpret_cast<const uint32_t *>(myring + slot * kRowBytesB);
-        const int k = max(ridx[wa + i], 0);
-        const int G = k >> lg;
-        if (G != curG) {
-            load_group(G);
-            curG = G;
-        }
-        const uint32_t hi = word >> 12;
-        float w[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const uint32_t src = (j < 5) ? word : hi;
-            const float v = __uint_as_float((src & code_mask(j)) | 0x4B000000u);
-            w[j] = fmaf(v, sp[j], cb[j]) - zs[j];
-        }
-        const float *xr = rx + (size_t)(wa + i) * BT;
-#pragma unroll
-        for (int b = 0; b < BT; ++b) {
-            const float xv = xr[b];
-            const float2 xb = make_float2(xv, xv);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                acc[b][j] = ffma2(make_float2(w[2 * j], w[2 * j + 1]), xb, acc[b][j]);
-        }
-        const int nxt = i + kStagesB;
-        if (nxt < n)
-            cp_async4(myring + slot * kRowBytesB, wcol + (size_t)max(ridx[wa + nxt], 0) * row_stride);
-        cp_async_commit();
-    }
-
-    if (lane_ok && n > 0) {
-#pragma unroll
-        for (int b = 0; b < BT; ++b)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                // rotate by lane inside the 8 outputs of a lane to spread banks
-                atomicAdd(red + b * kTileNB + lane * 8 + ((2 * j + lane) & 7), acc[b][j].x);
-                atomicAdd(red + b * kTileNB + lane * 8 + ((2 * j + 1 + lane) & 7), acc[b][j].y);
-            }
-    }
-    cp_async_wait_all();
-    __syncthreads();
-    for (int e2 = tid; e2 < B * (kTileNB / 4); e2 += kThreadsB) {
-        const int b = e2 / (kTileNB / 4), o = (e2 % (kTileNB / 4)) * 4;
-        const int l = o >> 3;
-        const float *rb = red + b * kTileNB + (l << 3);
-        const float4 v = make_float4(rb[(o + l) & 7], rb[(o + 1 + l) & 7], rb[(o + 2 + l) & 7],
-                                     rb[(o + 3 + l) & 7]);
-        if (n0 + o < p.N)
-            red_add_v4(p.ws_acc + (size_t)b * p.N + n0 + o, v);
     }
 }
 
@@ -843,10 +766,22 @@ cudaError_t launch_gemv_and_finalize(Kern kern, int grid, int block, size_t smem
     }
 }
 
-template <int SRC>
-cudaError_t launch_b1(KParams kp, int num_sms, cudaStream_t stream)
+// Batch groups of warps for B > 1: ceil(B / 2) rounded up to 1, 2, 4 or 8.
+int batch_groups(int B)
+{
+    const int need = (B + 1) / 2;
+    int nb = 1;
+    while (nb < need)
+        nb *= 2;
+    return nb;
+}
+
+template <int SRC, int BW>
+cudaError_t launch_gemv_t(KParams kp, int num_sms, cudaStream_t stream)
 {
     const GemvProblem &p = kp.p;
+    kp.nb = (BW == 1) ? 1 : batch_groups(p.B);
+    const int bp = kp.nb * BW;
     kp.n_tiles = ceil_div(p.N, kTileN1);
     kp.k_splits = std::max(1, num_sms / kp.n_tiles);
     const int G = p.K >> kp.lg;
@@ -854,7 +789,7 @@ cudaError_t launch_b1(KParams kp, int num_sms, cudaStream_t stream)
     for (;;) {
         kp.rows_cap = ceil_div(p.K, kp.k_splits) + 8;
         kp.span_cap = std::min(G, ceil_div(p.K, (long long)kp.k_splits << kp.lg) + 2);
-        L = smem1_layout(kp.span_cap, kp.rows_cap);
+        L = smem1_layout(kp.span_cap, kp.rows_cap, bp, BW);
         // the threshold path handles at most 4 runs of 32 channels per warp
         const bool runs_ok = (SRC != ROWS_THRESH) || (kp.rows_cap <= 4 * kThreads1);
         if ((L.total <= kMaxSmem && runs_ok) || kp.k_splits >= p.K / 8)
@@ -863,43 +798,16 @@ cudaError_t launch_b1(KParams kp, int num_sms, cudaStream_t stream)
     }
     if (L.total > kMaxSmem || (SRC == ROWS_THRESH && kp.rows_cap > 4 * kThreads1))
         return cudaErrorInvalidConfiguration;
-    return launch_gemv_and_finalize(gemv_b1_kernel<SRC>, kp.n_tiles * kp.k_splits, kThreads1,
+    return launch_gemv_and_finalize(gemv_kernel<SRC, BW>, kp.n_tiles * kp.k_splits, kThreads1,
                                     L.total, stream, kp);
 }
 
-template <int BT, int SRC>
-cudaError_t launch_bn_t(KParams kp, int num_sms, cudaStream_t stream)
-{
-    const GemvProblem &p = kp.p;
-    kp.n_tiles = ceil_div(p.N, kTileNB);
-    kp.k_splits = std::max(1, num_sms / kp.n_tiles);
-    const int G = p.K >> kp.lg;
-    SmemB L;
-    for (;;) {
-        kp.rows_cap = ceil_div(p.K, kp.k_splits) + 8;
-        kp.span_cap = std::min(G, ceil_div(p.K, (long long)kp.k_splits << kp.lg) + 2);
-        L = smemB_layout(kp.span_cap, kp.rows_cap, BT);
-        if (L.total <= kMaxSmem || kp.k_splits >= p.K / 8)
-            break;
-        kp.k_splits *= 2;
-    }
-    if (L.total > kMaxSmem)
-        return cudaErrorInvalidConfiguration;
-    return launch_gemv_and_finalize(gemv_bn_kernel<BT, SRC>, kp.n_tiles * kp.k_splits,
-                                    kThreadsB, L.total, stream, kp);
-}
-
 template <int SRC>
-cudaError_t launch_bn(KParams kp, int num_sms, cudaStream_t stream)
+cudaError_t launch_src(KParams kp, int num_sms, cudaStream_t stream)
 {
-    const int B = kp.p.B;
-    if (B <= 2)
-        return launch_bn_t<2, SRC>(kp, num_sms, stream);
-    if (B <= 4)
-        return launch_bn_t<4, SRC>(kp, num_sms, stream);
-    if (B <= 8)
-        return launch_bn_t<8, SRC>(kp, num_sms, stream);
-    return launch_bn_t<16, SRC>(kp, num_sms, stream);
+    if (kp.p.B == 1)
+        return launch_gemv_t<SRC, 1>(kp, num_sms, stream);
+    return launch_gemv_t<SRC, 2>(kp, num_sms, stream);
 }
 
 } // namespace
@@ -915,19 +823,14 @@ cudaError_t launch_gemv(const GemvProblem &p, int num_sms, cudaStream_t stream)
     KParams kp{};
     kp.p = p;
     kp.lg = __builtin_ctz((unsigned)p.group);
-    if (p.B == 1) {
-        switch (p.source) {
-        case ROWS_LIST: return launch_b1<ROWS_LIST>(kp, num_sms, stream);
-        case ROWS_DENSE: return launch_b1<ROWS_DENSE>(kp, num_sms, stream);
-        case ROWS_MASK: return launch_b1<ROWS_MASK>(kp, num_sms, stream);
-        default: return launch_b1<ROWS_THRESH>(kp, num_sms, stream);
-        }
+    switch (p.source) {
+    case ROWS_LIST: return launch_src<ROWS_LIST>(kp, num_sms, stream);
+    case ROWS_DENSE: return launch_src<ROWS_DENSE>(kp, num_sms, stream);
+    case ROWS_MASK: return launch_src<ROWS_MASK>(kp, num_sms, stream);
+    default:
+        // the API admits the threshold path at B = 1 only
+        return launch_gemv_t<ROWS_THRESH, 1>(kp, num_sms, stream);
     }
-    if (p.source == ROWS_DENSE)
-        return launch_bn<ROWS_DENSE>(kp, num_sms, stream);
-    if (p.source == ROWS_MASK)
-        return launch_bn<ROWS_MASK>(kp, num_sms, stream);
-    return launch_bn<ROWS_LIST>(kp, num_sms, stream);
 }
 
 } // namespace sgq
