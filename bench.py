@@ -404,6 +404,7 @@ def run_ours(args, dist: Dist):
 
     e2e = run_e2e(rep, path, min(args.steps, 2000), args.warmup, dist)
     layer = None if args.no_ffn else run_layer()
+    batch = None if args.no_ffn else run_batch()
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": dist.world,
@@ -432,6 +433,8 @@ def run_ours(args, dist: Dist):
     }
     if layer is not None:
         line.update(layer)
+    if batch is not None:
+        line["batch_ffn"] = batch
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     return line
@@ -621,6 +624,90 @@ def run_layer(n_steps: int = 1000):
                       round(1e6 / (32 * us["layer_fused"]), 1)},
         "rotation": f"{R} copies, {f.bytes_resident / 1e6:.0f} MB",
     }
+
+
+class BatchFfnReplica:
+    """R copies of one Qwen3-32B FFN (hidden 5120, intermediate 25600, int4
+    g128): stacked [W_g; W_u] and W_d; R x bytes > 4x L2. At batch B, x has B
+    rows of SiLU(g) * u, each with its own 50% threshold; gate/up and down read
+    the union of the rows' active sets (index lists from sgq_select), the down
+    projection over each row's 50% largest |h|."""
+
+    def __init__(self, seed: int = 11):
+        cfg = wl.QWEN32B_FFN
+        self.H, self.I, self.g = cfg["hidden"], cfg["inter"], cfg["group"]
+        H, I, g = self.H, self.I, self.g
+        pk = lambda W: self._pack(W)
+        gu = pk(torch.cat([wl.weight(I, H, seed), wl.weight(I, H, seed + 1)], 0))
+        down = pk(wl.weight(H, I, seed + 2))
+        per = sum(a.numel() * a.element_size() for t in (gu, down) for a in t)
+        l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+        self.R = max(2, int(math.ceil(4 * l2 / per)) + 1)
+        self.gu = [gu] + [tuple(a.clone() for a in gu) for _ in range(self.R - 1)]
+        self.down = [down] + [tuple(a.clone() for a in down) for _ in range(self.R - 1)]
+        self.bytes_resident = self.R * per
+        self.ws = sgq.alloc_workspace(2 * I, H, sgq.SGQ_MAX_BATCH)
+        self.idx_x, self.cnt_x = sgq.alloc_select(H)
+        self.idx_h, self.cnt_h = sgq.alloc_select(I)
+
+    def _pack(self, W):
+        N, K = W.shape
+        qw, sz = sgq.alloc_packed(N, K, self.g)
+        sgq.sgq_pack(W.cuda(), N, K, self.g, qw, sz)
+        return qw, sz
+
+    def setup(self, B: int):
+        H, I = self.H, self.I
+        xh = [wl.x_silu_gated(B, H, 4000 + 17 * B + r) for r in range(self.R)]
+        self.B = B
+        self.x = [x.cuda() for x in xh]
+        self.t = [[wl.percentile_threshold(x[b], 0.5) for b in range(B)] for x in xh]
+        self.h = torch.empty(B, I, dtype=torch.bfloat16, device="cuda")
+        self.y = torch.empty(B, H, dtype=torch.bfloat16, device="cuda")
+        self.th, self.union_x, self.union_h = [], [], []
+        for r in range(self.R):
+            self.front(r)
+            hc = self.h.cpu()
+            self.th.append([wl.percentile_threshold(hc[b], 0.5) for b in range(B)])
+            self.union_x.append(int(self.cnt_x.item()) / H)
+            sgq.sgq_select(self.h, B, I, self.th[r], self.idx_h, self.cnt_h)
+            self.union_h.append(int(self.cnt_h.item()) / I)
+        torch.cuda.synchronize()
+
+    def front(self, r):
+        B, H, I, g = self.B, self.H, self.I, self.g
+        sgq.sgq_select(self.x[r], B, H, self.t[r], self.idx_x, self.cnt_x)
+        qw, sz = self.gu[r]
+        sgq.sgq_gemv_glu(qw, sz, I, H, g, self.x[r], B, self.idx_x, self.cnt_x,
+                         sgq.SGQ_ACT_SILU, self.h, None, self.ws)
+
+    def ffn(self, r):                            # 6 launches
+        B, H, I, g = self.B, self.H, self.I, self.g
+        self.front(r)
+        sgq.sgq_select(self.h, B, I, self.th[r], self.idx_h, self.cnt_h)
+        qd, sd = self.down[r]
+        sgq.sgq_gemv(qd, sd, H, I, g, self.h, B, self.idx_h, self.cnt_h, self.y, None, self.ws)
+
+
+def run_batch(batches=(1, 2, 4, 8, 16), n_steps: int = 64):
+    """us per FFN at each batch size on the rotation (Qwen3-32B shapes)."""
+    f = BatchFfnReplica()
+    R = f.R
+    out = []
+    for B in batches:
+        f.setup(B)
+        n = max(n_steps, 2 * R)
+        us = time_calls(lambda i: f.ffn(i % R), n, R) * 1e3 / n
+        ux, uh = float(np.mean(f.union_x)), float(np.mean(f.union_h))
+        wbytes = ux * f.H * f.I + uh * f.I * f.H / 2    # codes of the union rows (gate+up, down)
+        out.append({"batch": B, "us_per_ffn": round(us, 2), "union_active_in": round(ux, 3),
+                    "union_active_h": round(uh, 3),
+                    "weight_code_GBps": round(wbytes / (us * 1e-6) / 1e9, 1),
+                    "tokens_per_s_equiv_ffn_only_64_layers": round(B * 1e6 / (64 * us), 1)})
+    return {"workload": "Qwen3-32B FFN decode (hidden 5120, intermediate 25600, int4 g128, "
+                        "SiLU): per-row 50% thresholds, union active sets, fused gate/up GLU; "
+                        "6 launches per FFN (two selects, two GEMV calls)",
+            "rows": out, "rotation": f"{R} copies, {f.bytes_resident / 1e6:.0f} MB"}
 
 
 # ---------------------------------------------------------------------------
