@@ -166,6 +166,49 @@ int sgq_pack(const void *W, int N, int K, int group, void *qweight, void *sz, in
     return e == cudaSuccess ? SGQ_OK : fail_cuda(e);
 }
 
+static int check_weights_nm(int N, int K, int group)
+{
+    int rc = check_weights(N, K, group);
+    if (rc)
+        return rc;
+    return (N % 64 == 0) ? SGQ_OK : SGQ_ERR_SHAPE;
+}
+
+int sgq_packed_sizes_nm(int N, int K, int group, size_t *qweight_bytes, size_t *keep_bytes,
+                        size_t *sz_bytes)
+{
+    int rc = check_weights_nm(N, K, group);
+    if (rc)
+        return rc;
+    if (!qweight_bytes || !keep_bytes || !sz_bytes)
+        return SGQ_ERR_NULL;
+    *qweight_bytes = (size_t)K * (N / 4);
+    *keep_bytes = (size_t)(K / group) * (N / 8);
+    *sz_bytes = (size_t)(K / group) * (N / 2) * 4;
+    return SGQ_OK;
+}
+
+int sgq_pack_nm(const void *W, int N, int K, int group, void *qweight, void *keep, void *sz,
+                int32_t *status, void *stream)
+{
+    int rc = check_weights_nm(N, K, group);
+    if (rc)
+        return rc;
+    if (!W || !qweight || !keep || !sz)
+        return SGQ_ERR_NULL;
+    if (!aligned16(W) || !aligned16(qweight) || !aligned16(keep) || !aligned16(sz))
+        return SGQ_ERR_ALIGN;
+    int sms = current_device_sms();
+    if (sms < 0)
+        return sms;
+    cudaError_t e = sgq::launch_pack_nm(static_cast<const uint16_t *>(W), N, K, group,
+                                        static_cast<uint8_t *>(qweight),
+                                        static_cast<uint8_t *>(keep),
+                                        static_cast<uint32_t *>(sz), status,
+                                        static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SGQ_OK : fail_cuda(e);
+}
+
 int sgq_select(const void *x, int B, int K, const float *t_host, int32_t *idx, int32_t *count,
                void *stream)
 {
@@ -277,6 +320,61 @@ int sgq_gemv_mask(const void *qweight, const void *sz, int N, int K, int group, 
     p.B = B;
     p.source = sgq::ROWS_MASK;
     return run_gemv(p, ws_bytes, workspace, stream);
+}
+
+static int run_gemv_nm(sgq::GemvProblem &p, const void *keep, size_t ws_bytes, void *workspace,
+                       void *stream)
+{
+    int rc = check_weights_nm(p.N, p.K, p.group);
+    if (rc)
+        return rc;
+    if (!keep)
+        return SGQ_ERR_NULL;
+    if (!aligned16(keep))
+        return SGQ_ERR_ALIGN;
+    p.keep = static_cast<const uint8_t *>(keep);
+    return run_gemv(p, ws_bytes, workspace, stream);
+}
+
+int sgq_gemv_nm(const void *qweight, const void *keep, const void *sz, int N, int K, int group,
+                const void *x, const int32_t *idx, const int32_t *count, void *y, float *y_f32,
+                void *workspace, size_t ws_bytes, int32_t *status, void *stream)
+{
+    sgq::GemvProblem p{};
+    p.qweight = static_cast<const uint8_t *>(qweight);
+    p.sz = static_cast<const uint32_t *>(sz);
+    p.x = static_cast<const uint16_t *>(x);
+    p.idx = idx;
+    p.count = count;
+    p.y = static_cast<uint16_t *>(y);
+    p.y_f32 = y_f32;
+    p.status = status;
+    p.N = N;
+    p.K = K;
+    p.group = group;
+    p.B = 1;
+    p.source = sgq::ROWS_LIST;
+    return run_gemv_nm(p, keep, ws_bytes, workspace, stream);
+}
+
+int sgq_gemv_nm_thresh(const void *qweight, const void *keep, const void *sz, int N, int K,
+                       int group, const void *x, float t, void *y, float *y_f32, void *workspace,
+                       size_t ws_bytes, int32_t *status, void *stream)
+{
+    sgq::GemvProblem p{};
+    p.qweight = static_cast<const uint8_t *>(qweight);
+    p.sz = static_cast<const uint32_t *>(sz);
+    p.x = static_cast<const uint16_t *>(x);
+    p.y = static_cast<uint16_t *>(y);
+    p.y_f32 = y_f32;
+    p.status = status;
+    p.N = N;
+    p.K = K;
+    p.group = group;
+    p.B = 1;
+    p.t = t;
+    p.source = sgq::ROWS_THRESH;
+    return run_gemv_nm(p, keep, ws_bytes, workspace, stream);
 }
 
 int sgq_gemv_dense(const void *qweight, const void *sz, int N, int K, int group, const void *x,

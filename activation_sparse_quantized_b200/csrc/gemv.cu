@@ -261,11 +261,13 @@ constexpr int kStages1 = 8; // rows in flight per warp (power of two); deeper ri
 // from a row serve both). With B > 1 the warps form kp.nb batch groups of
 // kWarps1 / nb warps; each group covers BW batch rows and reads the same rows
 // as the other groups (the later reads hit L2).
-__host__ __device__ constexpr int warp_region_bytes(int bw)
+__host__ __device__ constexpr int warp_region_bytes(int bw, bool nm = false)
 {
-    // a warp's ring, which also holds its partial tiles (BW x 1024 floats)
-    return (kStages1 * kRowBytes1 > bw * kTileN1 * 4) ? kStages1 * kRowBytes1
-                                                      : bw * kTileN1 * 4;
+    // a warp's ring, which also holds its partial tiles (BW x the tile's
+    // outputs as floats: 1024, or 2048 for the 2:4 layout)
+    return (kStages1 * kRowBytes1 > bw * kTileN1 * (nm ? 2 : 1) * 4)
+               ? kStages1 * kRowBytes1
+               : bw * kTileN1 * (nm ? 2 : 1) * 4;
 }
 
 // Output o (0..31) of a lane is code o % 8 of packed word o / 8. One 32-bit AND
@@ -289,11 +291,12 @@ struct Smem1 {
 // CTA's rows (channels). rx: x of each row, per batch row b at b * rows_cap.
 // rxh: x' = x 2^S of each row as fp16, same indexing. xs: x of the CTA's
 // channel slice (bitmask rows, batch 1). bp = batch rows padded to nb * BW.
-__host__ __device__ inline Smem1 smem1_layout(int span_cap, int rows_cap, int bp, int bw)
+__host__ __device__ inline Smem1 smem1_layout(int span_cap, int rows_cap, int bp, int bw,
+                                              bool nm = false)
 {
     Smem1 s;
     s.ring = 0;
-    s.szs = s.ring + (size_t)kWarps1 * warp_region_bytes(bw);
+    s.szs = s.ring + (size_t)kWarps1 * warp_region_bytes(bw, nm);
     s.ridx = s.szs + (size_t)span_cap * kTileN1 * 4;
     s.rx = s.ridx + (size_t)rows_cap * 4;
     s.scan = s.rx + (size_t)rows_cap * bp * 4;
@@ -410,13 +413,25 @@ __device__ __forceinline__ int part_chunk(int l, int c)
     return 8 * l + (c ^ (l & 7));
 }
 
-template <int SRC, int BW>
+// The same for the 2:4 layout's 64 outputs per lane (16 chunks of 4).
+__device__ __forceinline__ int part_chunk16(int l, int c)
+{
+    return 16 * l + (c ^ (l & 15));
+}
+
+// NM: the 2:4 layout (batch 1): the codes of a row are the kept outputs'
+// slots, 1024 slots = 2048 outputs per tile, 64 outputs per lane; the fold
+// adds each slot's sum to its output through the group's keep nibbles.
+template <int SRC, int BW, bool NM = false>
 __global__ void __launch_bounds__(kThreads1, 1) gemv_kernel(const KParams kp)
 {
+    static_assert(!NM || BW == 1, "the 2:4 layout is batch 1 only");
+    constexpr int OPL = NM ? 64 : 32;  // outputs per lane
+    constexpr int TO = 32 * OPL;       // outputs per tile
     extern __shared__ __align__(16) uint8_t smem[];
     const GemvProblem &p = kp.p;
     const int bp = kp.nb * BW; // batch rows padded to whole groups
-    const Smem1 L = smem1_layout(kp.span_cap, kp.rows_cap, bp, BW);
+    const Smem1 L = smem1_layout(kp.span_cap, kp.rows_cap, bp, BW, NM);
     uint8_t *ring = smem + L.ring;
     const uint4 *szs = reinterpret_cast<const uint4 *>(smem + L.szs);
     int32_t *ridx = reinterpret_cast<int32_t *>(smem + L.ridx);
@@ -428,10 +443,12 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_kernel(const KParams kp)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int tile = blockIdx.x % kp.n_tiles;
     const int split = blockIdx.x / kp.n_tiles;
-    const int n0 = tile * kTileN1;
+    const int n0 = tile * TO;           // first output of the tile
+    const int s0 = tile * kTileN1;      // first code slot of the tile
+    const int SN = NM ? p.N / 2 : p.N;  // code slots (and (s, z) pairs) per row and group
     const int lg = kp.lg;
-    const size_t row_stride = (size_t)(p.N / 2);
-    const bool lane_ok = (n0 + lane * 32) < p.N;
+    const size_t row_stride = (size_t)(SN / 2);
+    const bool lane_ok = (n0 + lane * OPL) < p.N;
 
     grid_launch_dependents();
 
@@ -442,10 +459,10 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_kernel(const KParams kp)
     int G0 = 0, span = 0;
     auto stage_sz = [&]() {
         for (int c = tid; c < span * (kTileN1 / 4); c += kThreads1) {
-            const int g = c >> 8, q = c & 255; // q: chunk of 4 outputs in the tile
-            if (n0 + 4 * q < p.N)
+            const int g = c >> 8, q = c & 255; // q: chunk of 4 slots in the tile
+            if (s0 + 4 * q < SN)
                 cp_async16(smem + L.szs + ((size_t)g * 256 + part_chunk(q >> 3, q & 7)) * 16,
-                           p.sz + (size_t)(G0 + g) * p.N + n0 + 4 * q);
+                           p.sz + (size_t)(G0 + g) * SN + s0 + 4 * q);
         }
         cp_async_commit();
     };
@@ -490,8 +507,8 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_kernel(const KParams kp)
     const int n = (nbw > 0) ? (int)((long long)nr * (wq + 1) / wpg) - wa : 0;
 
     // Ring prologue. Lanes past N read column 0 (valid memory, result unused).
-    const uint8_t *wcol = p.qweight + (lane_ok ? ((size_t)n0 / 2 + lane * 16) : 0);
-    uint8_t *region = ring + (size_t)warp * warp_region_bytes(BW);
+    const uint8_t *wcol = p.qweight + (lane_ok ? ((size_t)s0 / 2 + lane * 16) : 0);
+    uint8_t *region = ring + (size_t)warp * warp_region_bytes(BW, NM);
     uint8_t *myring = region + lane * 16;
 #pragma unroll
     for (int s = 0; s < kStages1; ++s) {
@@ -539,16 +556,18 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_kernel(const KParams kp)
     cp_async_wait<kStages1>();
     __syncthreads();
 
-    // accg[bb][o] = this group's sum of q x' 2^-code_shift(o); acc[bb][o] =
-    // folded result in units of 2^-S.
-    float accg[BW][32], acc[BW][32];
+    // accg[bb][o] = this group's sum of q x' 2^-code_shift(o) for code slot o;
+    // acc[bb][o] = folded result of output o in units of 2^-S.
+    float accg[BW][32], acc[BW][OPL];
 #pragma unroll
-    for (int bb = 0; bb < BW; ++bb)
+    for (int bb = 0; bb < BW; ++bb) {
 #pragma unroll
-        for (int o = 0; o < 32; ++o) {
+        for (int o = 0; o < 32; ++o)
             accg[bb][o] = 0.f;
+#pragma unroll
+        for (int o = 0; o < OPL; ++o)
             acc[bb][o] = 0.f;
-        }
+    }
 
     //   acc += s * (2^code_shift accg - z * sum x')
     auto fold = [&](int G, const float *Xg) {
@@ -565,7 +584,7 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_kernel(const KParams kp)
             }
         } else {
             const uint4 *g4 = reinterpret_cast<const uint4 *>(
-                p.sz + (size_t)G * p.N + n0 + (lane_ok ? lane * 32 : 0));
+                p.sz + (size_t)G * SN + s0 + (lane_ok ? lane * 32 : 0));
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 const uint4 v = __ldg(g4 + c);
@@ -575,14 +594,40 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_kernel(const KParams kp)
                 w[4 * c + 3] = v.w;
             }
         }
+        if (!NM) {
 #pragma unroll
-        for (int o = 0; o < 32; ++o) {
-            const float s = half_lo(w[o]), z = half_hi(w[o]);
+            for (int o = 0; o < 32; ++o) {
+                const float s = half_lo(w[o]), z = half_hi(w[o]);
 #pragma unroll
-            for (int bb = 0; bb < BW; ++bb) {
-                const float t = accg[bb][o] * pow2f(code_shift(o));
-                acc[bb][o] = fmaf(s, fmaf(-z, Xg[bb], t), acc[bb][o]);
-                accg[bb][o] = 0.f;
+                for (int bb = 0; bb < BW; ++bb) {
+                    const float t = accg[bb][o] * pow2f(code_shift(o));
+                    acc[bb][o] = fmaf(s, fmaf(-z, Xg[bb], t), acc[bb][o]);
+                    accg[bb][o] = 0.f;
+                }
+            }
+        } else {
+            // Keep nibbles of this lane's 16 blocks (8 bytes); block j's slots
+            // 2j, 2j + 1 go to its first and second kept output.
+            const uint2 km = lane_ok ? __ldg(reinterpret_cast<const uint2 *>(
+                                           p.keep + (size_t)G * (p.N / 8) + n0 / 8 + lane * 8))
+                                     : make_uint2(0u, 0u);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                float f[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int o = 2 * j + h;
+                    const float t = accg[0][o] * pow2f(code_shift(o));
+                    f[h] = half_lo(w[o]) * fmaf(-half_hi(w[o]), Xg[0], t);
+                    accg[0][o] = 0.f;
+                }
+                const uint32_t m = ((j < 8 ? km.x : km.y) >> (4 * (j & 7))) & 0xFu;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const bool kept = (m >> i) & 1u;
+                    const bool second = (m & ((1u << i) - 1u)) != 0u; // a kept output below i
+                    acc[0][4 * j + i] += kept ? (second ? f[1] : f[0]) : 0.f;
+                }
             }
         }
     };
@@ -667,22 +712,40 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_kernel(const KParams kp)
     __syncwarp();
 #pragma unroll
     for (int bb = 0; bb < BW; ++bb) {
-        float4 *part = reinterpret_cast<float4 *>(region) + bb * (kTileN1 / 4);
+        float4 *part = reinterpret_cast<float4 *>(region) + bb * (TO / 4);
         const int E = -S[bb];
         const float f1 = pow2f(E / 2), f2 = pow2f(E - E / 2);
         const bool live = lane_ok && n > 0 && bb < nbw;
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-            part[part_chunk(lane, c)] =
+        for (int c = 0; c < OPL / 4; ++c)
+            part[NM ? part_chunk16(lane, c) : part_chunk(lane, c)] =
                 live ? make_float4((acc[bb][4 * c] * f1) * f2, (acc[bb][4 * c + 1] * f1) * f2,
                                    (acc[bb][4 * c + 2] * f1) * f2, (acc[bb][4 * c + 3] * f1) * f2)
                      : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();
-    // Each thread owns one chunk of 4 outputs of the tile; for every batch row
-    // it sums the partial tiles of the warps of that row's group and adds the
-    // sum into the workspace.
-    if (BW == 1) {
+    // Each thread owns chunks of 4 outputs of the tile (one, or two for the
+    // 2:4 tile); for every batch row it sums the partial tiles of the warps of
+    // that row's group and adds the sum into the workspace.
+    if (NM) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int q = tid + r * kThreads1; // chunk of the 2048-output tile
+            const int l = q >> 4, c = q & 15;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int w = 0; w < kWarps1; ++w) {
+                const float4 u = reinterpret_cast<const float4 *>(
+                    ring + (size_t)w * warp_region_bytes(BW, NM))[part_chunk16(l, c)];
+                v.x += u.x;
+                v.y += u.y;
+                v.z += u.z;
+                v.w += u.w;
+            }
+            if (n0 + 4 * q < p.N)
+                red_add_v4(p.ws_acc + n0 + 4 * q, v);
+        }
+    } else     if (BW == 1) {
         const int l = tid >> 3, c = tid & 7;
         float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
@@ -776,20 +839,20 @@ int batch_groups(int B)
     return nb;
 }
 
-template <int SRC, int BW>
+template <int SRC, int BW, bool NM = false>
 cudaError_t launch_gemv_t(KParams kp, int num_sms, cudaStream_t stream)
 {
     const GemvProblem &p = kp.p;
     kp.nb = (BW == 1) ? 1 : batch_groups(p.B);
     const int bp = kp.nb * BW;
-    kp.n_tiles = ceil_div(p.N, kTileN1);
+    kp.n_tiles = ceil_div(p.N, NM ? 2 * kTileN1 : kTileN1);
     kp.k_splits = std::max(1, num_sms / kp.n_tiles);
     const int G = p.K >> kp.lg;
     Smem1 L;
     for (;;) {
         kp.rows_cap = ceil_div(p.K, kp.k_splits) + 8;
         kp.span_cap = std::min(G, ceil_div(p.K, (long long)kp.k_splits << kp.lg) + 2);
-        L = smem1_layout(kp.span_cap, kp.rows_cap, bp, BW);
+        L = smem1_layout(kp.span_cap, kp.rows_cap, bp, BW, NM);
         // the threshold path handles at most 4 runs of 32 channels per warp
         const bool runs_ok = (SRC != ROWS_THRESH) || (kp.rows_cap <= 4 * kThreads1);
         if ((L.total <= kMaxSmem && runs_ok) || kp.k_splits >= p.K / 8)
@@ -798,13 +861,15 @@ cudaError_t launch_gemv_t(KParams kp, int num_sms, cudaStream_t stream)
     }
     if (L.total > kMaxSmem || (SRC == ROWS_THRESH && kp.rows_cap > 4 * kThreads1))
         return cudaErrorInvalidConfiguration;
-    return launch_gemv_and_finalize(gemv_kernel<SRC, BW>, kp.n_tiles * kp.k_splits, kThreads1,
-                                    L.total, stream, kp);
+    return launch_gemv_and_finalize(gemv_kernel<SRC, BW, NM>, kp.n_tiles * kp.k_splits,
+                                    kThreads1, L.total, stream, kp);
 }
 
 template <int SRC>
 cudaError_t launch_src(KParams kp, int num_sms, cudaStream_t stream)
 {
+    if (kp.p.keep) // the 2:4 layout (batch 1 only, checked by the API)
+        return launch_gemv_t<SRC, 1, true>(kp, num_sms, stream);
     if (kp.p.B == 1)
         return launch_gemv_t<SRC, 1>(kp, num_sms, stream);
     return launch_gemv_t<SRC, 2>(kp, num_sms, stream);
@@ -829,6 +894,8 @@ cudaError_t launch_gemv(const GemvProblem &p, int num_sms, cudaStream_t stream)
     case ROWS_MASK: return launch_src<ROWS_MASK>(kp, num_sms, stream);
     default:
         // the API admits the threshold path at B = 1 only
+        if (p.keep)
+            return launch_gemv_t<ROWS_THRESH, 1, true>(kp, num_sms, stream);
         return launch_gemv_t<ROWS_THRESH, 1>(kp, num_sms, stream);
     }
 }

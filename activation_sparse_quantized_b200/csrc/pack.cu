@@ -105,6 +105,93 @@ __global__ void pack_kernel(const uint16_t *__restrict__ W, int N, int K, int g,
     }
 }
 
+// 2:4 weight sparsity along the outputs of each channel row (the N:M
+// sparsity of "SparseDecoding: Decoding-Aware Pruning for Accurate and
+// Efficient LLM Inference", Abstract, placed so that it composes with
+// skipping whole input channels). Per quantization group G and block of 4
+// outputs, the 2 outputs with the largest sum of squared weights over the
+// group are kept (ties to the lower output); the group's channels share that
+// choice. Sums of squares of fp16 values are exact in fp64, so the choice is
+// fixed bit for bit. Kept outputs are quantized as in the dense layout.
+//
+// Layout (N % 64 == 0): qweight u8 [K][N/4], byte j of row k = code of slot
+// 2j | slot 2j+1 << 4, where slots 2j and 2j+1 are the kept outputs of block j
+// in ascending order; keep u8 [K/g][N/8], byte j = keep nibble of block 2j |
+// that of block 2j+1 << 4 (bit i = output 4 block + i kept); sz [K/g][N/2]
+// (fp16 s, fp16 z) per slot. A block holding NaN/Inf keeps outputs 0 and 1
+// with s = 1, z = 0, q = 0 and sets SGQ_STATUS_NONFINITE_W.
+//
+// One thread per (group, pair of blocks): it owns one keep byte and two bytes
+// of each of the group's packed rows.
+__global__ void pack_nm_kernel(const uint16_t *__restrict__ W, int N, int K, int g,
+                               uint8_t *__restrict__ qweight, uint8_t *__restrict__ keep,
+                               uint32_t *__restrict__ sz, int32_t *status)
+{
+    const int pairs = N / 8;
+    const int G = K / g;
+    const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= (long long)pairs * G)
+        return;
+    const int jj = (int)(t % pairs);
+    const int grp = (int)(t / pairs);
+    uint32_t kbyte = 0;
+    for (int h = 0; h < 2; ++h) {
+        const int j = 2 * jj + h; // block: outputs 4j .. 4j + 3
+        double e[4];
+        bool bad = false;
+        for (int i = 0; i < 4; ++i) {
+            const uint16_t *w = W + (size_t)(4 * j + i) * K + (size_t)grp * g;
+            double acc = 0.0;
+            for (int r = 0; r < g; ++r) {
+                const double d = half_bits_to_double(w[r]);
+                if (!isfinite(d))
+                    bad = true;
+                acc = __dadd_rn(acc, __dmul_rn(d, d)); // no contraction: fixed rounding
+            }
+            e[i] = acc;
+        }
+        int a = 0, b = 1;
+        if (!bad) {
+            a = 0;
+            for (int i = 1; i < 4; ++i)
+                if (e[i] > e[a])
+                    a = i;
+            b = (a == 0) ? 1 : 0;
+            for (int i = 0; i < 4; ++i)
+                if (i != a && e[i] > e[b])
+                    b = i;
+            if (a > b) {
+                const int tmp = a;
+                a = b;
+                b = tmp;
+            }
+        } else {
+            set_status(status, SGQ_STATUS_NONFINITE_W);
+        }
+        kbyte |= ((1u << a) | (1u << b)) << (4 * h);
+        GroupQuant p0, p1;
+        if (bad) {
+            p0.bad = p1.bad = true;
+            p0.s = p1.s = 1.0;
+            p0.z = p1.z = 0.0;
+            p0.packed = p1.packed = 0x3c00u; // s = 1, z = +0
+        } else {
+            p0 = quantize_group(W + (size_t)(4 * j + a) * K + (size_t)grp * g, g);
+            p1 = quantize_group(W + (size_t)(4 * j + b) * K + (size_t)grp * g, g);
+        }
+        sz[(size_t)grp * (N / 2) + 2 * j] = p0.packed;
+        sz[(size_t)grp * (N / 2) + 2 * j + 1] = p1.packed;
+        const uint16_t *w0 = W + (size_t)(4 * j + a) * K + (size_t)grp * g;
+        const uint16_t *w1 = W + (size_t)(4 * j + b) * K + (size_t)grp * g;
+        for (int r = 0; r < g; ++r) {
+            const uint32_t c0 = code_of(w0[r], p0);
+            const uint32_t c1 = code_of(w1[r], p1);
+            qweight[(size_t)(grp * g + r) * (N / 4) + j] = (uint8_t)(c0 | (c1 << 4));
+        }
+    }
+    keep[(size_t)grp * (N / 8) + jj] = (uint8_t)kbyte;
+}
+
 } // namespace
 
 cudaError_t launch_pack(const uint16_t *W, int N, int K, int g, uint8_t *qweight, uint32_t *sz,
@@ -114,6 +201,16 @@ cudaError_t launch_pack(const uint16_t *W, int N, int K, int g, uint8_t *qweight
     const int block = 128;
     const long long grid = (threads + block - 1) / block;
     pack_kernel<<<(unsigned)grid, block, 0, stream>>>(W, N, K, g, qweight, sz, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack_nm(const uint16_t *W, int N, int K, int g, uint8_t *qweight,
+                           uint8_t *keep, uint32_t *sz, int32_t *status, cudaStream_t stream)
+{
+    const long long threads = (long long)(N / 8) * (K / g);
+    const int block = 128;
+    const long long grid = (threads + block - 1) / block;
+    pack_nm_kernel<<<(unsigned)grid, block, 0, stream>>>(W, N, K, g, qweight, keep, sz, status);
     return cudaGetLastError();
 }
 

@@ -35,6 +35,7 @@ struct GemvProblem {
     const int32_t *idx;
     const int32_t *count;
     const uint32_t *mask; // ROWS_MASK: bit k % 32 of word k / 32 = channel k active
+    const uint8_t *keep;  // 2:4 layout: keep nibbles [K/g][N/4] (NULL = dense layout)
     uint16_t *y;
     float *y_f32;
     float *ws_acc;
@@ -50,6 +51,8 @@ size_t gemv_workspace_bytes(int N, int B);
 
 cudaError_t launch_pack(const uint16_t *W, int N, int K, int g, uint8_t *qweight, uint32_t *sz,
                         int32_t *status, cudaStream_t stream);
+cudaError_t launch_pack_nm(const uint16_t *W, int N, int K, int g, uint8_t *qweight,
+                           uint8_t *keep, uint32_t *sz, int32_t *status, cudaStream_t stream);
 cudaError_t launch_select(const uint16_t *x, int B, int K, const Thresholds &th, int32_t *idx,
                           int32_t *count, cudaStream_t stream);
 cudaError_t launch_select_mask(const uint16_t *x, int B, int K, const Thresholds &th,

@@ -31,7 +31,8 @@ EXPORTS = (
     "sgq_packed_sizes", "sgq_pack", "sgq_select", "sgq_gemv_workspace_bytes", "sgq_gemv",
     "sgq_gemv_thresh", "sgq_gemv_dense", "sgq_glu", "sgq_status_string", "sgq_last_cuda_error",
     "sgq_layout_version", "sgq_gemv_thresh_noalloc", "sgq_gemv_glu", "sgq_gemv_glu_thresh",
-    "sgq_gemv_glu_dense", "sgq_select_mask", "sgq_gemv_mask",
+    "sgq_gemv_glu_dense", "sgq_select_mask", "sgq_gemv_mask", "sgq_packed_sizes_nm",
+    "sgq_pack_nm", "sgq_gemv_nm", "sgq_gemv_nm_thresh",
 )
 
 
@@ -84,6 +85,11 @@ def _declare(lib):
         "sgq_gemv_glu_dense": ([P, P, I, I, I, P, I, I, P, P, P, Z, P, P], I),
         "sgq_select_mask": ([P, I, I, P, P, P, P], I),
         "sgq_gemv_mask": ([P, P, I, I, I, P, I, P, P, P, P, Z, P, P], I),
+        "sgq_packed_sizes_nm": ([I, I, I, ctypes.POINTER(Z), ctypes.POINTER(Z),
+                                 ctypes.POINTER(Z)], I),
+        "sgq_pack_nm": ([P, I, I, I, P, P, P, P, P], I),
+        "sgq_gemv_nm": ([P, P, P, I, I, I, P, P, P, P, P, P, Z, P, P], I),
+        "sgq_gemv_nm_thresh": ([P, P, P, I, I, I, P, F, P, P, P, Z, P, P], I),
         "sgq_status_string": ([I], ctypes.c_char_p),
         "sgq_last_cuda_error": ([], I),
         "sgq_layout_version": ([], I),
@@ -147,6 +153,34 @@ def sgq_gemv_mask(qweight, sz, N, K, group, x, B, mask, y, y_f32, workspace, sta
         _ptr(qweight), _ptr(sz), N, K, group, _ptr(x), B, _ptr(mask), _ptr(y), _ptr(y_f32),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status),
         _stream(stream)))
+
+
+def sgq_packed_sizes_nm(N: int, K: int, group: int):
+    a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check("sgq_packed_sizes_nm", load().sgq_packed_sizes_nm(
+        N, K, group, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)))
+    return a.value, b.value, c.value
+
+
+def sgq_pack_nm(W, N, K, group, qweight, keep, sz, status=None, stream=None):
+    _check("sgq_pack_nm", load().sgq_pack_nm(_ptr(W), N, K, group, _ptr(qweight), _ptr(keep),
+                                             _ptr(sz), _ptr(status), _stream(stream)))
+
+
+def sgq_gemv_nm(qweight, keep, sz, N, K, group, x, idx, count, y, y_f32, workspace, status=None,
+                stream=None):
+    _check("sgq_gemv_nm", load().sgq_gemv_nm(
+        _ptr(qweight), _ptr(keep), _ptr(sz), N, K, group, _ptr(x), _ptr(idx), _ptr(count),
+        _ptr(y), _ptr(y_f32), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _ptr(status), _stream(stream)))
+
+
+def sgq_gemv_nm_thresh(qweight, keep, sz, N, K, group, x, t, y, y_f32, workspace, status=None,
+                       stream=None):
+    _check("sgq_gemv_nm_thresh", load().sgq_gemv_nm_thresh(
+        _ptr(qweight), _ptr(keep), _ptr(sz), N, K, group, _ptr(x), float(t), _ptr(y),
+        _ptr(y_f32), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _ptr(status), _stream(stream)))
 
 
 def sgq_gemv_workspace_bytes(N: int, K: int, B: int) -> int:
@@ -226,6 +260,14 @@ def alloc_packed(N, K, group, device="cuda"):
 def alloc_workspace(N, K, B, device="cuda"):
     nbytes = sgq_gemv_workspace_bytes(N, K, B)
     return torch.zeros(nbytes // 4, dtype=torch.int32, device=device)
+
+
+def alloc_packed_nm(N, K, group, device="cuda"):
+    """(qweight u8, keep u8, sz int32) buffers of the 2:4 layout."""
+    qb, kb, sb = sgq_packed_sizes_nm(N, K, group)
+    return (torch.empty(qb, dtype=torch.uint8, device=device),
+            torch.empty(kb, dtype=torch.uint8, device=device),
+            torch.empty(sb // 4, dtype=torch.int32, device=device))
 
 
 def alloc_mask(K, device="cuda"):

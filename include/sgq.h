@@ -193,6 +193,41 @@ int sgq_gemv_dense(const void *qweight, const void *sz, int N, int K, int group,
                    void *workspace, size_t ws_bytes, int32_t *status, void *stream);
 
 /*
+ * Static 2:4 weight sparsity composed with the dynamic activation sparsity
+ * (the N:M sparse GEMV with bitmask indexing of "SparseDecoding: Decoding-
+ * Aware Pruning for Accurate and Efficient LLM Inference", Abstract, placed
+ * so that skipped input channels stay whole skipped runs).
+ *
+ * The 2:4 pattern runs along the outputs of each channel row: in every block
+ * of 4 consecutive outputs, 2 are kept, and the g channels of a quantization
+ * group share that choice. sgq_pack_nm prunes and packs W: per (group, block)
+ * it keeps the 2 outputs with the largest sum over the group of w^2 (exact in
+ * fp64; ties keep the lower output), then quantizes the kept outputs exactly
+ * as sgq_pack does. Layout (N % 64 == 0):
+ *   qweight u8 [K][N/4]: byte j of row k = code of slot 2j | slot 2j+1 << 4,
+ *                        slots 2j, 2j+1 = the kept outputs of block j, ascending.
+ *   keep    u8 [K/group][N/8]: byte j = keep nibble of block 2j | that of
+ *                        block 2j+1 << 4 (bit i set = output 4 block + i kept).
+ *   sz      [K/group][N/2] (fp16 scale, fp16 zero) per slot.
+ * An active channel costs N/4 bytes instead of N/2. A block holding NaN/Inf
+ * keeps outputs 0 and 1 as zeros and sets SGQ_STATUS_NONFINITE_W.
+ *
+ * sgq_gemv_nm / sgq_gemv_nm_thresh: y = W_pruned[:, S] x[S] (pruned weights
+ * are zero), batch 1, rows from an index list (as sgq_gemv) or the fused
+ * threshold (as sgq_gemv_thresh). Workspace as sgq_gemv with B = 1.
+ */
+int sgq_packed_sizes_nm(int N, int K, int group, size_t *qweight_bytes, size_t *keep_bytes,
+                        size_t *sz_bytes);
+int sgq_pack_nm(const void *W, int N, int K, int group, void *qweight, void *keep, void *sz,
+                int32_t *status, void *stream);
+int sgq_gemv_nm(const void *qweight, const void *keep, const void *sz, int N, int K, int group,
+                const void *x, const int32_t *idx, const int32_t *count, void *y, float *y_f32,
+                void *workspace, size_t ws_bytes, int32_t *status, void *stream);
+int sgq_gemv_nm_thresh(const void *qweight, const void *keep, const void *sz, int N, int K,
+                       int group, const void *x, float t, void *y, float *y_f32,
+                       void *workspace, size_t ws_bytes, int32_t *status, void *stream);
+
+/*
  * Gated FFN activation h = act(gate) * up, elementwise over [B][I] bf16
  * (fp32 arithmetic, bf16 round-to-nearest-even output). act = SGQ_ACT_SILU
  * (v / (1 + e^-v)) or SGQ_ACT_RELU (v if v > 0 else 0, the ReGLU of the SVD

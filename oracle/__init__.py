@@ -96,8 +96,11 @@ def _declare(lib):
     lib.oracle_glu.argtypes = [P, P, ctypes.c_int64, i, P, P]
     lib.oracle_act_mul.argtypes = [P, P, ctypes.c_int64, i, P, P]
     lib.oracle_select_mask.argtypes = [P, i, i, P, P, P]
+    lib.oracle_nm_keep.argtypes = [P, i, i, i, P, P]
+    lib.oracle_pack_layout_nm.argtypes = [P, P, P, P, P, i, i, i, P, P, P]
     for f in ("oracle_quantize", "oracle_pack_layout", "oracle_select",
-              "oracle_gemv", "oracle_gemv_dense", "oracle_glu", "oracle_act_mul", "oracle_select_mask"):
+              "oracle_gemv", "oracle_gemv_dense", "oracle_glu", "oracle_act_mul", "oracle_select_mask", "oracle_nm_keep",
+              "oracle_pack_layout_nm"):
         getattr(lib, f).restype = ctypes.c_int
     return lib
 
@@ -264,3 +267,46 @@ def select_mask(x_bits, t, lib=None):
     _check(lib.oracle_select_mask(x.ctypes.data, B, K, tt.ctypes.data, mask.ctypes.data,
                                   ctypes.byref(cnt)), "oracle_select_mask")
     return mask, cnt.value
+
+
+def nm_keep(W_bits, g, lib=None):
+    """2:4 choice of W [N, K] (fp16 bits): (keep [K/g, N/4] nibbles, bad [K/g, N/4])."""
+    lib = lib or load()
+    W = _c(W_bits, np.uint16)
+    N, K = W.shape
+    keep = np.empty((K // g, N // 4), np.uint8)
+    bad = np.empty((K // g, N // 4), np.uint8)
+    _check(lib.oracle_nm_keep(W.ctypes.data, N, K, g, keep.ctypes.data, bad.ctypes.data),
+           "oracle_nm_keep")
+    return keep, bad
+
+
+def pack_layout_nm(q, s, z, keep, bad, g, lib=None):
+    """The 2:4 packed layout: (qweight [K, N/4] u8, keep_packed [K/g, N/8] u8,
+    sz [K/g, N/2, 2] u16)."""
+    lib = lib or load()
+    q = _c(q, np.uint8)
+    N, K = q.shape
+    s, z = _c(s, np.uint16), _c(z, np.uint16)
+    keep, bad = _c(keep, np.uint8), _c(bad, np.uint8)
+    qw = np.empty((K, N // 4), np.uint8)
+    kp = np.empty((K // g, N // 8), np.uint8)
+    sz = np.empty((K // g, N // 2, 2), np.uint16)
+    _check(lib.oracle_pack_layout_nm(q.ctypes.data, s.ctypes.data, z.ctypes.data,
+                                     keep.ctypes.data, bad.ctypes.data, N, K, g, qw.ctypes.data,
+                                     kp.ctypes.data, sz.ctypes.data), "oracle_pack_layout_nm")
+    return qw, kp, sz
+
+
+def gemv_nm(q, s, z, keep, bad, g, x_bits, idx, lib=None):
+    """The GEMV over the 2:4-pruned weights: the pruned outputs of each
+    (group, block), and every output of a bad block, weigh zero (their scale
+    and zero are set to 0 before the plain GEMV). Returns as gemv."""
+    N = q.shape[0]
+    G = s.shape[1]
+    kept = np.zeros((N, G), bool)
+    for i in range(4):
+        kept[i::4, :] = (((keep >> i) & 1) == 1).T & (bad == 0).T
+    s2 = np.where(kept, s, np.uint16(0)).astype(np.uint16)
+    z2 = np.where(kept, z, np.uint16(0)).astype(np.uint16)
+    return gemv(q, s2, z2, g, x_bits, idx, lib)

@@ -204,6 +204,92 @@ int oracle_pack_layout(const uint8_t *q, const uint16_t *s, const uint16_t *z,
 }
 
 /* ------------------------------------------------------------------------- */
+/* Static 2:4 weight sparsity composed with activation sparsity ([P3]        */
+/* "SparseDecoding: Decoding-Aware Pruning for Accurate and Efficient LLM     */
+/* Inference", Abstract: an N:M sparse matrix-vector product with bitmask    */
+/* indexing). Reading: the 2:4 blocks run along the outputs of each channel  */
+/* row and the g channels of a quantization group share the choice; in each */
+/* (group, block of 4 outputs) the 2 outputs with the largest sum of w^2     */
+/* over the group are kept, equal sums keeping the lower output. A block     */
+/* holding NaN/Inf keeps outputs 0 and 1 with zero codes (s = 1, z = 0).     */
+/* ------------------------------------------------------------------------- */
+
+int oracle_nm_keep(const uint16_t *W, int N, int K, int g, uint8_t *keep, uint8_t *bad)
+{
+    if (N <= 0 || K <= 0 || g <= 0 || K % g != 0 || N % 4 != 0)
+        return -2;
+    int G = K / g;
+    for (int grp = 0; grp < G; ++grp)
+        for (int j = 0; j < N / 4; ++j) {
+            double e[4];
+            int nonfinite = 0;
+            for (int i = 0; i < 4; ++i) {
+                double acc = 0.0;
+                for (int r = 0; r < g; ++r) {
+                    double w = oracle_half_to_double(W[(size_t)(4 * j + i) * K + (size_t)grp * g + r]);
+                    if (!isfinite(w))
+                        nonfinite = 1;
+                    acc += w * w;
+                }
+                e[i] = acc;
+            }
+            uint8_t nib = 0x3;
+            if (!nonfinite) {
+                int first = -1, second = -1;
+                for (int i = 0; i < 4; ++i) {
+                    if (first < 0 || e[i] > e[first]) {
+                        second = first;
+                        first = i;
+                    } else if (second < 0 || e[i] > e[second]) {
+                        second = i;
+                    }
+                }
+                nib = (uint8_t)((1u << first) | (1u << second));
+            }
+            keep[(size_t)grp * (N / 4) + j] = nib;
+            bad[(size_t)grp * (N / 4) + j] = (uint8_t)nonfinite;
+        }
+    return 0;
+}
+
+int oracle_pack_layout_nm(const uint8_t *q, const uint16_t *s, const uint16_t *z,
+                          const uint8_t *keep, const uint8_t *bad, int N, int K, int g,
+                          uint8_t *qweight, uint8_t *keep_packed, uint16_t *sz)
+{
+    if (N <= 0 || K <= 0 || g <= 0 || K % g != 0 || N % 8 != 0)
+        return -2;
+    int G = K / g;
+    for (int grp = 0; grp < G; ++grp) {
+        for (int j = 0; j < N / 4; ++j) {
+            uint8_t nib = keep[(size_t)grp * (N / 4) + j];
+            int isbad = bad[(size_t)grp * (N / 4) + j];
+            int out[2], h = 0;
+            for (int i = 0; i < 4 && h < 2; ++i)
+                if (nib & (1u << i))
+                    out[h++] = 4 * j + i;
+            if (h != 2)
+                return -2;
+            for (h = 0; h < 2; ++h) {
+                size_t slot = (size_t)grp * (N / 2) + 2 * j + h;
+                sz[slot * 2 + 0] = isbad ? (uint16_t)0x3c00 : s[(size_t)out[h] * G + grp];
+                sz[slot * 2 + 1] = isbad ? (uint16_t)0 : z[(size_t)out[h] * G + grp];
+            }
+            for (int r = 0; r < g; ++r) {
+                int k = grp * g + r;
+                uint8_t c0 = isbad ? 0 : q[(size_t)out[0] * K + k];
+                uint8_t c1 = isbad ? 0 : q[(size_t)out[1] * K + k];
+                qweight[(size_t)k * (N / 4) + j] = (uint8_t)(c0 | (c1 << 4));
+            }
+        }
+        for (int jj = 0; jj < N / 8; ++jj)
+            keep_packed[(size_t)grp * (N / 8) + jj] =
+                (uint8_t)(keep[(size_t)grp * (N / 4) + 2 * jj] |
+                          (keep[(size_t)grp * (N / 4) + 2 * jj + 1] << 4));
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
 /* Active set ([P1] Abstract: dynamic sparsity, runtime gathering of the     */
 /* sparse indices; [P5] Abstract: ReGLU neurons that are zero are skipped).  */
 /* Readings: channel k is active when |x[k]| > t (strict), so t = 0 keeps    */

@@ -44,6 +44,21 @@ int oracle_quantize(const uint16_t *W, int N, int K, int g,
 int oracle_pack_layout(const uint8_t *q, const uint16_t *s, const uint16_t *z,
                        int N, int K, int g, uint8_t *qweight, uint16_t *sz);
 
+/* 2:4 weight sparsity along the outputs, shared by the g channels of a group:
+ * keep [K/g][N/4] nibbles (bit i = output 4j + i kept; the 2 largest sums of
+ * w^2 over the group, ties to the lower output), bad [K/g][N/4] = 1 where the
+ * block holds NaN/Inf (then keep = 0x3). */
+int oracle_nm_keep(const uint16_t *W, int N, int K, int g, uint8_t *keep, uint8_t *bad);
+
+/* The 2:4 packed layout from the codes of oracle_quantize and the keep choice:
+ * qweight [K][N/4] (byte j = slot 2j | slot 2j+1 << 4, slots = kept outputs of
+ * block j ascending), keep_packed [K/g][N/8] (block 2jj | block 2jj+1 << 4),
+ * sz [K/g][N/2][2] fp16 (scale, zero) per slot; bad blocks get zero codes
+ * with s = 1, z = 0. */
+int oracle_pack_layout_nm(const uint8_t *q, const uint16_t *s, const uint16_t *z,
+                          const uint8_t *keep, const uint8_t *bad, int N, int K, int g,
+                          uint8_t *qweight, uint8_t *keep_packed, uint16_t *sz);
+
 /* Active set of a bf16 activation batch x [B][K] against thresholds t[B]:
  * idx <- ascending unique k with |x[b][k]| > t[b] for some b; *count <- size. */
 int oracle_select(const uint16_t *x, int B, int K, const float *t,

@@ -486,4 +486,81 @@ def pin_select_mask_bits(lib):
         assert np.array_equal(m.astype(np.uint64), words) and c == int(act.sum())
 
 
+def _nm_fixture_weights():
+    K, N = 32, 8
+    W = np.zeros((N, K), np.float64)
+    W[0, 0::2] = 15 / 16
+    W[2, :] = 1 / 32
+    W[3, 1::2] = 15 / 8
+    W[4:8, :] = 15 / 16
+    return W.astype(np.float16).view(np.uint16)
+
+
+def pin_nm_layout_hand(lib):
+    """The 2:4 choice and packed layout of a hand-worked case (largest sums of
+    w^2, ties to the lower output, nibble and slot order, (s, z) per slot)."""
+    d = _golden("nm_layout_hand.json")
+    Wb = _nm_fixture_weights()
+    g = d["group"]
+    keep, bad = oracle.nm_keep(Wb, g, lib)
+    assert keep.tolist() == d["keep_nibbles"] and not bad.any()
+    q, s, z = oracle.quantize(Wb, g, lib)
+    qw, kp, sz = oracle.pack_layout_nm(q, s, z, keep, bad, g, lib)
+    h = lambda v: int(v, 16)
+    assert kp.tolist() == [[h(v) for v in r] for r in d["keep_packed"]]
+    even = [h(v) for v in d["qweight_even_row"]]
+    odd = [h(v) for v in d["qweight_odd_row"]]
+    for k in range(d["K"]):
+        assert qw[k].tolist() == (even if k % 2 == 0 else odd), k
+    assert sz.tolist() == [[[h(v) for v in pair] for pair in blk] for blk in d["sz"]]
+
+
+def pin_nm_keep_brute_force(lib):
+    """Brute force of the 2:4 choice on random weights with planted ties:
+    sums of squares in numpy, a stable sort by (-energy, output)."""
+    rng = np.random.default_rng(20)
+    for N, K, g in ((16, 64, 32), (64, 256, 64), (32, 128, 128)):
+        Wf = (rng.standard_normal((N, K)) * 0.02).astype(np.float16)
+        Wf[5] = Wf[4]                       # equal energies inside a block
+        Wf[8:12] = Wf[8]                    # a block of four equal rows
+        Wf[13] = -Wf[12]                    # equal energy, opposite sign
+        keep, bad = oracle.nm_keep(Wf.view(np.uint16), g, lib)
+        assert not bad.any()
+        Wd = Wf.astype(np.float64)
+        for grp in range(K // g):
+            e = (Wd[:, grp * g:(grp + 1) * g] ** 2).sum(axis=1)
+            for j in range(N // 4):
+                order = sorted(range(4), key=lambda i: (-e[4 * j + i], i))
+                nib = (1 << order[0]) | (1 << order[1])
+                assert keep[grp, j] == nib, (N, K, g, grp, j)
+    Wf = (rng.standard_normal((8, 64)) * 0.02).astype(np.float16)
+    Wf[6, 40] = np.float16(np.nan)
+    keep, bad = oracle.nm_keep(Wf.view(np.uint16), 32, lib)
+    assert bad.tolist() == [[0, 0], [0, 1]] and keep[1, 1] == 0x3
+
+
+def pin_nm_gemv_is_gemv_of_pruned_weights(lib):
+    """The 2:4 GEMV equals the plain GEMV of W with the pruned weights set to
+    zero and quantized as usual (a zeroed group gets s = 1, z = 0, q = 0):
+    every fp64 partial sum is the same, so y and sum |w x| agree bit for bit."""
+    rng = np.random.default_rng(21)
+    N, K, g = 32, 256, 64
+    Wf = (rng.standard_normal((N, K)) * 0.02).astype(np.float16)
+    Wb = Wf.view(np.uint16)
+    keep, bad = oracle.nm_keep(Wb, g, lib)
+    q, s, z = oracle.quantize(Wb, g, lib)
+    x = bf16_bits_from_f32(rng.standard_normal((2, K)).astype(np.float32))
+    idx = oracle.select(x, [0.5, 0.7], lib)
+    y, sa, yb = oracle.gemv_nm(q, s, z, keep, bad, g, x, idx, lib)
+    Wp = Wf.copy()
+    for grp in range(K // g):
+        for n in range(N):
+            if not (keep[grp, n // 4] >> (n % 4)) & 1:
+                Wp[n, grp * g:(grp + 1) * g] = 0
+    q2, s2, z2 = oracle.quantize(Wp.view(np.uint16), g, lib)
+    y2, sa2, yb2 = oracle.gemv(q2, s2, z2, g, x, idx, lib)
+    assert np.array_equal(y, y2) and np.array_equal(sa, sa2) and np.array_equal(yb, yb2)
+    assert np.mean(y == 0) < 0.1          # the pruned GEMV is not trivially zero
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -112,6 +112,13 @@ def test_host_argument_checks(lib):
                                    fake, wsg, None, None) == -7
     assert lib.sgq_gemv_glu_dense(fake, fake, 14336, 4096, 96, fake, 1, 0, fake, None, fake,
                                   wsg, None, None) == -3
+    # 2:4 layout: N % 64, null keep, sizes
+    assert lib.sgq_pack_nm(fake, 4064, 14336, 128, fake, fake, fake, None, None) == -2
+    assert lib.sgq_gemv_nm(fake, None, fake, 4096, 14336, 128, fake, fake, fake, fake, None,
+                           fake, ws, None, None) == -1
+    assert lib.sgq_gemv_nm_thresh(fake, fake, fake, 4000, 14336, 128, fake, F(0.5), fake, None,
+                                  fake, ws, None, None) == -2
+    assert sgq.sgq_packed_sizes_nm(4096, 14336, 128) == (14336 * 1024, 112 * 512, 112 * 2048 * 4)
 
 
 def test_missing_library_fails_loudly(tmp_path):

@@ -42,6 +42,14 @@ MUTANTS = {
                        "mask[idx[i] / 32] |= 1u << (31 - idx[i] % 32);"),
     "mask_word_index": ("mask[idx[i] / 32] |= 1u << (idx[i] % 32);",
                         "mask[idx[i] / 8 % ((K + 31) / 32)] |= 1u << (idx[i] % 32);"),
+    "nm_ties_to_higher": ("if (first < 0 || e[i] > e[first]) {",
+                          "if (first < 0 || e[i] >= e[first]) {"),
+    "nm_energy_abs": ("                    acc += w * w;\n",
+                      "                    acc += fabs(w);\n"),
+    "nm_keep_nibble_order": ("(uint8_t)(keep[(size_t)grp * (N / 4) + 2 * jj] |",
+                             "(uint8_t)(keep[(size_t)grp * (N / 4) + 2 * jj + 1] |"),
+    "nm_slot_order": ("qweight[(size_t)k * (N / 4) + j] = (uint8_t)(c0 | (c1 << 4));",
+                      "qweight[(size_t)k * (N / 4) + j] = (uint8_t)(c1 | (c0 << 4));"),
     "act_mul_drops_up": ("double hv = oracle_act(gate[i], act) * up[i];",
                          "double hv = oracle_act(gate[i], act);"),
     "act_mul_swapped": ("double hv = oracle_act(gate[i], act) * up[i];",
