@@ -302,6 +302,54 @@ int sgq_gemv_thresh(const void *qweight, const void *sz, int N, int K, int group
     return run_gemv(p, ws_bytes, workspace, stream);
 }
 
+// Accumulating forms: y_acc [B][N] fp32 (caller-owned) += the GEMV; the GEMV
+// kernel's split-K reductions land in y_acc itself, so there is no workspace
+// and no epilogue kernel.
+static int run_gemv_acc(sgq::GemvProblem &p, float *y_acc, void *stream)
+{
+    if (!y_acc)
+        return SGQ_ERR_NULL;
+    p.accumulate = true;
+    p.y = reinterpret_cast<uint16_t *>(y_acc); // non-null for the checks; never written
+    return run_gemv(p, sgq::gemv_workspace_bytes(p.N, p.B), y_acc, stream);
+}
+
+int sgq_gemv_acc(const void *qweight, const void *sz, int N, int K, int group, const void *x,
+                 int B, const int32_t *idx, const int32_t *count, float *y_acc, int32_t *status,
+                 void *stream)
+{
+    sgq::GemvProblem p{};
+    p.qweight = static_cast<const uint8_t *>(qweight);
+    p.sz = static_cast<const uint32_t *>(sz);
+    p.x = static_cast<const uint16_t *>(x);
+    p.idx = idx;
+    p.count = count;
+    p.status = status;
+    p.N = N;
+    p.K = K;
+    p.group = group;
+    p.B = B;
+    p.source = sgq::ROWS_LIST;
+    return run_gemv_acc(p, y_acc, stream);
+}
+
+int sgq_gemv_thresh_acc(const void *qweight, const void *sz, int N, int K, int group,
+                        const void *x, float t, float *y_acc, int32_t *status, void *stream)
+{
+    sgq::GemvProblem p{};
+    p.qweight = static_cast<const uint8_t *>(qweight);
+    p.sz = static_cast<const uint32_t *>(sz);
+    p.x = static_cast<const uint16_t *>(x);
+    p.status = status;
+    p.N = N;
+    p.K = K;
+    p.group = group;
+    p.B = 1;
+    p.t = t;
+    p.source = sgq::ROWS_THRESH;
+    return run_gemv_acc(p, y_acc, stream);
+}
+
 int sgq_gemv_mask(const void *qweight, const void *sz, int N, int K, int group, const void *x,
                   int B, const uint32_t *mask, void *y, float *y_f32, void *workspace,
                   size_t ws_bytes, int32_t *status, void *stream)

@@ -815,7 +815,7 @@ cudaError_t launch_gemv_and_finalize(Kern kern, int grid, int block, size_t smem
                                      cudaStream_t stream, const KParams &kp)
 {
     cudaError_t err = launch_pdl(kern, grid, block, smem, stream, kp);
-    if (err != cudaSuccess)
+    if (err != cudaSuccess || kp.p.accumulate)
         return err;
     const int quads = kp.p.B * (kp.p.N / 4);
     const int fgrid = std::max(1, std::min(ceil_div(quads, 256), 148));

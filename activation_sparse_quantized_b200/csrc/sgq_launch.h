@@ -44,6 +44,7 @@ struct GemvProblem {
     float t;
     int source;
     int epilogue; // Epilogue; y (and y_f32) are [B][N/2] for the GLU epilogues
+    bool accumulate; // add into ws_acc (the caller's fp32 [B][N]) and launch no epilogue kernel
 };
 
 // Bytes of workspace (partial sums + tile counters) for N outputs, B rows.

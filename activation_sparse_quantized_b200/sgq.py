@@ -32,7 +32,7 @@ EXPORTS = (
     "sgq_gemv_thresh", "sgq_gemv_dense", "sgq_glu", "sgq_status_string", "sgq_last_cuda_error",
     "sgq_layout_version", "sgq_gemv_thresh_noalloc", "sgq_gemv_glu", "sgq_gemv_glu_thresh",
     "sgq_gemv_glu_dense", "sgq_select_mask", "sgq_gemv_mask", "sgq_packed_sizes_nm",
-    "sgq_pack_nm", "sgq_gemv_nm", "sgq_gemv_nm_thresh",
+    "sgq_pack_nm", "sgq_gemv_nm", "sgq_gemv_nm_thresh", "sgq_gemv_acc", "sgq_gemv_thresh_acc",
 )
 
 
@@ -90,6 +90,8 @@ def _declare(lib):
         "sgq_pack_nm": ([P, I, I, I, P, P, P, P, P], I),
         "sgq_gemv_nm": ([P, P, P, I, I, I, P, P, P, P, P, P, Z, P, P], I),
         "sgq_gemv_nm_thresh": ([P, P, P, I, I, I, P, F, P, P, P, Z, P, P], I),
+        "sgq_gemv_acc": ([P, P, I, I, I, P, I, P, P, P, P, P], I),
+        "sgq_gemv_thresh_acc": ([P, P, I, I, I, P, F, P, P, P], I),
         "sgq_status_string": ([I], ctypes.c_char_p),
         "sgq_last_cuda_error": ([], I),
         "sgq_layout_version": ([], I),
@@ -181,6 +183,19 @@ def sgq_gemv_nm_thresh(qweight, keep, sz, N, K, group, x, t, y, y_f32, workspace
         _ptr(qweight), _ptr(keep), _ptr(sz), N, K, group, _ptr(x), float(t), _ptr(y),
         _ptr(y_f32), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _ptr(status), _stream(stream)))
+
+
+def sgq_gemv_acc(qweight, sz, N, K, group, x, B, idx, count, y_acc, status=None, stream=None):
+    """y_acc (fp32 [B][N]) += the sparse GEMV; one kernel, no workspace."""
+    _check("sgq_gemv_acc", load().sgq_gemv_acc(
+        _ptr(qweight), _ptr(sz), N, K, group, _ptr(x), B, _ptr(idx), _ptr(count), _ptr(y_acc),
+        _ptr(status), _stream(stream)))
+
+
+def sgq_gemv_thresh_acc(qweight, sz, N, K, group, x, t, y_acc, status=None, stream=None):
+    _check("sgq_gemv_thresh_acc", load().sgq_gemv_thresh_acc(
+        _ptr(qweight), _ptr(sz), N, K, group, _ptr(x), float(t), _ptr(y_acc), _ptr(status),
+        _stream(stream)))
 
 
 def sgq_gemv_workspace_bytes(N: int, K: int, B: int) -> int:

@@ -240,6 +240,7 @@ class Replica:
             sgq.sgq_select_mask(self.x[r], 1, K, [self.t[r]], m)
             self.mask.append(m)
         self.smask = sgq.alloc_mask(K)
+        self.yacc = torch.zeros(1, N, dtype=torch.float32, device="cuda")
 
     def step(self, r: int, path: str):
         """One pass of the hot path on copy r (kernels launched: 2 or 1)."""
@@ -272,6 +273,12 @@ class Replica:
                               self.y, None, self.ws)
         elif which == "select_mask":
             sgq.sgq_select_mask(self.x[r], 1, K, [self.t[r]], self.smask)
+        elif which == "thresh_acc":   # the GEMV kernel alone (adds into fp32, no epilogue)
+            sgq.sgq_gemv_thresh_acc(self.qw[r], self.sz[r], N, K, GROUP, self.x[r], self.t[r],
+                                    self.yacc)
+        elif which == "gemv_acc":
+            sgq.sgq_gemv_acc(self.qw[r], self.sz[r], N, K, GROUP, self.x[r], 1, self.idx[r],
+                             self.cnt[r], self.yacc)
 
 
 class GraphRunner:
@@ -373,14 +380,19 @@ def run_ours(args, dist: Dist):
     value = total_bytes / (ms * 1e-3) / 1e9
     us_per_gemv = ms * 1e3 / args.steps
 
-    # the dominant kernel alone, same rotation, for the roofline
-    dom = {"thresh": "thresh", "list": "gemv", "mask": "mask"}[path]
+    # the dominant kernel alone, same rotation, for the roofline: the GEMV
+    # kernel through its accumulating form (the same kernel adding its
+    # split-K sums into an fp32 buffer, so no epilogue kernel follows it);
+    # the mask path has no accumulating form and is timed as the whole call
+    dom = {"thresh": "thresh_acc", "list": "gemv_acc", "mask": "mask"}[path]
     nk = max(args.steps, 2 * R)
     kms = time_calls(lambda i: rep.kernel_only(i % R, dom), nk, period)
     k_us = kms * 1e3 / nk
     k_bytes = sum(rep.abytes[i % R] for i in range(nk)) / nk
-    if dom == "thresh":   # reads all of x, no index list
-        k_bytes = k_bytes - 6 * np.mean(rep.active) + 2 * K
+    if dom == "thresh_acc":   # reads all of x, no index list; fp32 y
+        k_bytes = k_bytes - 6 * np.mean(rep.active) + 2 * K + 2 * N
+    elif dom == "gemv_acc":   # fp32 y
+        k_bytes = k_bytes + 2 * N
     elif dom == "mask":   # K/8 bytes of mask instead of the 4a-byte index list
         k_bytes = k_bytes - 4 * np.mean(rep.active) + K // 8
     peak, peak_kind = measured_peak()
@@ -388,23 +400,31 @@ def run_ours(args, dist: Dist):
     src = source_hash("gemv.cu", "sgq_device.cuh")
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
-                "traffic": profiled_traffic(dom, src), "kernel": f"sgq_{dom}",
+                "traffic": profiled_traffic({"thresh_acc": "thresh", "gemv_acc": "gemv"}.get(dom, dom), src),
+                "kernel": {"thresh_acc": "gemv_kernel<ROWS_THRESH> (select fused)",
+                           "gemv_acc": "gemv_kernel<ROWS_LIST>",
+                           "mask": "sgq_gemv_mask call"}[dom],
                 "kernel_us": round(k_us, 3), "algorithmic_bytes": int(k_bytes),
                 "frac_of_8TBps": round(achieved / 8000.0, 4),
-                "timed": "the GEMV call on its stream (GEMV kernel + split-K epilogue kernel)"}
+                "timed": ("the GEMV kernel alone on its stream, launched through the "
+                          "accumulating entry point (sgq_gemv_thresh_acc / sgq_gemv_acc): the "
+                          "same kernel, its split-K sums added into fp32 y, no epilogue kernel; "
+                          "the bf16 call with its epilogue kernel is call_us")
+                         if dom != "mask" else "the sgq_gemv_mask call (GEMV + epilogue kernel)"}
 
     # comparison points on the same rotation: dense int4 GEMV, select alone
     nc = max(min(args.steps, 4000), 2 * period)
     dense_ms = time_calls(lambda i: rep.kernel_only(i % R, "dense"), nc, period)
     sel_ms = time_calls(lambda i: rep.kernel_only(i % R, "select"), nc, period)
     cmp_us = {}
-    for name in ("gemv", "thresh", "mask", "select_mask"):
+    for name in ("gemv", "thresh", "mask", "select_mask", "thresh_acc"):
         cms = time_calls(lambda i: rep.kernel_only(i % R, name), nc, period)
         cmp_us[name] = round(cms * 1e3 / nc, 3)
 
     e2e = run_e2e(rep, path, min(args.steps, 2000), args.warmup, dist)
     layer = None if args.no_ffn else run_layer()
     batch = None if args.no_ffn else run_batch()
+    nm = None if args.no_ffn else run_nm()
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": dist.world,
@@ -425,6 +445,7 @@ def run_ours(args, dist: Dist):
         "select_us": round(sel_ms * 1e3 / nc, 3),
         "call_us": {"gemv_list": cmp_us["gemv"], "gemv_thresh": cmp_us["thresh"],
                     "gemv_mask": cmp_us["mask"], "select_mask": cmp_us["select_mask"],
+                    "gemv_thresh_acc": cmp_us["thresh_acc"],
                     "note": "one C-ABI call each on the same rotation; a GEMV call is the "
                             "GEMV kernel plus its split-K epilogue kernel"},
         "e2e": e2e,
@@ -435,6 +456,8 @@ def run_ours(args, dist: Dist):
         line.update(layer)
     if batch is not None:
         line["batch_ffn"] = batch
+    if nm is not None:
+        line["nm_2of4"] = nm
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     return line
@@ -708,6 +731,46 @@ def run_batch(batches=(1, 2, 4, 8, 16), n_steps: int = 64):
                         "SiLU): per-row 50% thresholds, union active sets, fused gate/up GLU; "
                         "6 launches per FFN (two selects, two GEMV calls)",
             "rows": out, "rotation": f"{R} copies, {f.bytes_resident / 1e6:.0f} MB"}
+
+
+def run_nm(n_steps: int = 4000, sparsity: float = 0.5):
+    """The 8B down_proj with 2:4 weight sparsity (sgq_pack_nm) composed with
+    50% activation sparsity, fused threshold path, on its own rotation."""
+    W = wl.weight(N, K, 0)
+    qb, kb, sb = sgq.sgq_packed_sizes_nm(N, K, GROUP)
+    qw0, kp0, sz0 = sgq.alloc_packed_nm(N, K, GROUP)
+    sgq.sgq_pack_nm(W.cuda(), N, K, GROUP, qw0, kp0, sz0)
+    l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+    R = max(2, int(math.ceil(4 * l2 / (qb + kb + sb))) + 1)
+    cp = [(qw0, kp0, sz0)] + [(qw0.clone(), kp0.clone(), sz0.clone()) for _ in range(R - 1)]
+    xh = [wl.x_silu_gated(1, K, 1000 + r) for r in range(R)]
+    x = [v.cuda() for v in xh]
+    t = [wl.percentile_threshold(v[0], sparsity) for v in xh]
+    y = torch.empty(1, N, dtype=torch.bfloat16, device="cuda")
+    ws = sgq.alloc_workspace(N, K, 1)
+    idx, cnt = sgq.alloc_select(K)
+    ab = []
+    for r in range(R):
+        sgq.sgq_select(x[r], 1, K, [t[r]], idx, cnt)
+        a = int(cnt.item())
+        gr = int(np.unique(idx[:a].cpu().numpy() // GROUP).size)
+        ab.append(a * N // 4 + gr * (N // 2) * 4 + gr * N // 8 + 2 * K + 2 * N)
+
+    def call(i):
+        r = i % R
+        q, k_, s_ = cp[r]
+        sgq.sgq_gemv_nm_thresh(q, k_, s_, N, K, GROUP, x[r], t[r], y, None, ws)
+
+    period = R * max(1, 64 // R)
+    n = max(n_steps, 2 * period)
+    us = time_calls(call, n, period) * 1e3 / n
+    b = float(np.mean(ab))
+    return {"workload": "Llama-3-8B down_proj (K=14336, N=4096, g128) with static 2:4 weight "
+                        "sparsity along the outputs (sgq_pack_nm) and 50% activation sparsity, "
+                        "select fused; batch 1",
+            "us_per_gemv": round(us, 3), "active_bytes_per_gemv": int(b),
+            "GBps_active": round(b / (us * 1e-6) / 1e9, 1),
+            "rotation": f"{R} copies, {R * (qb + kb + sb) / 1e6:.0f} MB"}
 
 
 # ---------------------------------------------------------------------------

@@ -172,6 +172,22 @@ int sgq_gemv_thresh(const void *qweight, const void *sz, int N, int K, int group
                     void *workspace, size_t ws_bytes, int32_t *status, void *stream);
 
 /*
+ * Accumulating forms: y_acc += W_deq[:, S] x[S] into a caller-owned fp32
+ * buffer y_acc [B][N] (16-byte aligned), e.g. the fp32 residual stream of a
+ * decode step (the pages fuse no such epilogue; it is a deployment form of
+ * this library). The GEMV's split-K partial sums are added straight into
+ * y_acc with fp32 reductions, so there is no workspace, no bf16 rounding and
+ * no second (epilogue) kernel: one launch per call. The order of the fp32
+ * additions is not fixed, so the low bits of y_acc may differ from run to
+ * run. Rows as sgq_gemv (index list, B <= 16) or sgq_gemv_thresh (B = 1).
+ */
+int sgq_gemv_acc(const void *qweight, const void *sz, int N, int K, int group,
+                 const void *x, int B, const int32_t *idx, const int32_t *count,
+                 float *y_acc, int32_t *status, void *stream);
+int sgq_gemv_thresh_acc(const void *qweight, const void *sz, int N, int K, int group,
+                        const void *x, float t, float *y_acc, int32_t *status, void *stream);
+
+/*
  * The activation-sparse GEMV with the active set given as a bitmask (as
  * written by sgq_select_mask, or by any producer of the same format): the
  * same result as sgq_gemv over the ascending list of the set bits. Each CTA

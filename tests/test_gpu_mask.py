@@ -105,3 +105,33 @@ def test_gemv_mask_empty_gives_positive_zero():
     ws = sgq.alloc_workspace(N, K, 1)
     sgq.sgq_gemv_mask(qw, sz, N, K, g, case.x.to(DEV), 1, m, y, y32, ws)
     assert (y32 == 0).all() and not torch.signbit(y32).any() and bits(y).max() == 0
+
+
+# ---------------------------------------------------------------------------
+# accumulating forms (y_acc += the GEMV, one kernel)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("path,B", [("thresh", 1), ("list", 1), ("list", 4)])
+def test_gemv_acc_adds_into_fp32_buffer(path, B):
+    """y_acc starts at random r0; afterwards y_acc - r0 must be the GEMV within
+    its bound plus the fp32 roundings of adding into r0 (at most one per
+    split-K share and one for r0 itself: 64 ulps of |r0| + sum|wx| is ample)."""
+    case = wl.gemv_case(**wl.LLAMA8B_DOWN, B=B, sparsity=0.5, seed=430)
+    N, K, g = case.W.shape[0], case.W.shape[1], case.group
+    qw, sz, _ = gpu_pack(case.W, g)
+    x_d = case.x.to(DEV)
+    r0 = torch.randn(B, N, generator=torch.Generator().manual_seed(431)) * 3
+    y_acc = r0.clone().to(DEV)
+    if path == "thresh":
+        sgq.sgq_gemv_thresh_acc(qw, sz, N, K, g, x_d, case.t[0], y_acc)
+    else:
+        idx, cnt = sgq.alloc_select(K)
+        sgq.sgq_select(x_d, B, K, case.t, idx, cnt)
+        sgq.sgq_gemv_acc(qw, sz, N, K, g, x_d, B, idx, cnt, y_acc)
+    xb = bits(case.x)
+    oidx = oracle.select(xb, case.t)
+    q, s, z = oracle_codes(case.W, g)
+    y64, sa, _ = oracle.gemv(q, s, z, g, xb, oidx)
+    got = y_acc.cpu().double().numpy() - r0.double().numpy()
+    tol = 1e-3 * sa + 64 * 2.0 ** -24 * (np.abs(r0.double().numpy()) + sa)
+    assert np.all(np.abs(got - y64) <= tol)
