@@ -73,6 +73,27 @@ __device__ __forceinline__ int warp_max_exponent(float m)
     return ilogbf(m);
 }
 
+// Exclusive prefix, over runs, of the per-run counts in scan[] for the runs
+// 32c .. 32c + 31 (one per lane), plus the carry from the earlier chunks: a
+// warp scan instead of a serial walk over shared memory. Returns the lane's
+// exclusive prefix; *chunk_total receives the chunk's sum (every lane).
+__device__ __forceinline__ int chunk_prefix(const int *scan, int runs, int c, int carry,
+                                            int *chunk_total)
+{
+    const int lane = threadIdx.x & 31;
+    const int r = c * 32 + lane;
+    const int v = (r < runs) ? scan[r] : 0;
+    int incl = v;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d)
+            incl += t;
+    }
+    *chunk_total = __shfl_sync(0xffffffffu, incl, 31);
+    return carry + incl - v;
+}
+
 // Channel slice [c0, c1) of split s when channels are dealt out in runs of 8.
 __device__ __forceinline__ void channel_slice(const KParams &kp, int split, int &c0, int &c1)
 {
@@ -145,18 +166,22 @@ __device__ int build_rows(const KParams &kp, int split, int32_t *ridx, float *rx
         }
         __syncthreads();
         int total = 0;
-        for (int q = 0; q < runs; ++q)
-            total += scan[q];
-        for (int q = warp; q < runs; q += NT / 32) {
-            const uint32_t m = run_bits(q);
-            if ((m >> lane) & 1u) {
-                int pos = __popc(m & ((1u << lane) - 1u));
-                for (int r = 0; r < q; ++r)
-                    pos += scan[r];
-                ridx[pos] = c0 + q * 32 + lane;
-                if (FILL_X)
-                    rx[pos] = xs[q * 32 + lane];
+        for (int c = 0; c * 32 < runs; ++c) {
+            int ct;
+            const int excl = chunk_prefix(scan, runs, c, total, &ct);
+            // this warp's runs in the chunk (q is warp-uniform)
+            for (int q = c * 32 + ((warp - c * 32) % (NT / 32) + NT / 32) % (NT / 32);
+                 q < runs && q < c * 32 + 32; q += NT / 32) {
+                const int base = __shfl_sync(0xffffffffu, excl, q - c * 32);
+                const uint32_t m = run_bits(q);
+                if ((m >> lane) & 1u) {
+                    const int pos = base + __popc(m & ((1u << lane) - 1u));
+                    ridx[pos] = c0 + q * 32 + lane;
+                    if (FILL_X)
+                        rx[pos] = xs[q * 32 + lane];
+                }
             }
+            total += ct;
         }
         __syncthreads();
         return total;
@@ -188,18 +213,19 @@ __device__ int build_rows(const KParams &kp, int split, int32_t *ridx, float *rx
                 scan[q] = __popc(mask[u]);
         }
         __syncthreads();
-        int total = 0;
-        for (int q = 0; q < runs; ++q)
-            total += scan[q];
+        // runs <= 4 * NT / 32 <= 32 (the launcher keeps it so): one chunk
+        int total;
+        const int excl = chunk_prefix(scan, runs, 0, 0, &total);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            const int q = warp + u * (NT / 32);
-            if (q < runs && ((mask[u] >> lane) & 1u)) {
-                int pos = __popc(mask[u] & ((1u << lane) - 1u));
-                for (int r = 0; r < q; ++r)
-                    pos += scan[r];
-                ridx[pos] = c0 + q * 32 + lane;
-                rx[pos] = xv[u];
+            const int q = warp + u * (NT / 32); // warp-uniform
+            if (q < runs) {
+                const int base = __shfl_sync(0xffffffffu, excl, q);
+                if ((mask[u] >> lane) & 1u) {
+                    const int pos = base + __popc(mask[u] & ((1u << lane) - 1u));
+                    ridx[pos] = c0 + q * 32 + lane;
+                    rx[pos] = xv[u];
+                }
             }
         }
         __syncthreads();
