@@ -69,8 +69,11 @@ class Dist:
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
         self.pg = None
+        self.dev = "cuda"
 
     def init(self, backend="nccl"):
+        # reductions run on the device for NCCL, on the host for gloo
+        self.dev = "cuda" if backend == "nccl" else "cpu"
         if self.world > 1:
             import torch.distributed as dist
             dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120),
@@ -85,14 +88,14 @@ class Dist:
     def max(self, v: float) -> float:
         if not self.pg:
             return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        t = torch.tensor([v], dtype=torch.float64, device=self.dev)
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 
     def sum(self, v: float) -> float:
         if not self.pg:
             return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        t = torch.tensor([v], dtype=torch.float64, device=self.dev)
         self.pg.all_reduce(t, op=self.pg.ReduceOp.SUM)
         return float(t.item())
 
@@ -314,6 +317,13 @@ class GraphRunner:
             self._graph(rem, 0).replay()
 
 
+def whole_job(bytes_local: float, ms_local: float, dist: Dist):
+    """Whole-job GB/s: the bytes of every rank over the slowest rank's device
+    time (replicas: weak scaling). Returns (GB/s, max ms)."""
+    ms = dist.max(ms_local)
+    return dist.sum(bytes_local) / (ms * 1e-3) / 1e9, ms
+
+
 def time_calls(fn, n: int, period: int, dist: Dist | None = None, warm: int = 3):
     """Device time (ms) of exactly n calls of fn(i), via CUDA graphs."""
     stream = torch.cuda.Stream()
@@ -374,10 +384,7 @@ def run_ours(args, dist: Dist):
         torch.cuda.synchronize()
     dist.barrier()
     ms_local = e0.elapsed_time(e1)
-    ms = dist.max(ms_local)
-    step_bytes = sum(rep.abytes[i % R] for i in range(args.steps))
-    total_bytes = dist.sum(step_bytes)
-    value = total_bytes / (ms * 1e-3) / 1e9
+    value, ms = whole_job(sum(rep.abytes[i % R] for i in range(args.steps)), ms_local, dist)
     us_per_gemv = ms * 1e3 / args.steps
 
     # the dominant kernel alone, same rotation, for the roofline: the GEMV
