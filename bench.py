@@ -472,14 +472,17 @@ def run_ours(args, dist: Dist):
 
 def run_e2e(rep: Replica, path: str, steps: int, warmup: int, dist: Dist):
     """The same metric through the public API with host buffers: every step
-    copies x from pinned host memory, runs the path, and reads y back."""
+    copies x from pinned host memory, runs the path, reads y back into pinned
+    host memory and waits for it. Each step is one CUDA graph holding those
+    three operations (captured once per weight copy), so a step costs one
+    graph launch and one synchronize; the same steps issued as separate calls
+    are reported as us_per_gemv_eager."""
     xs = [x.pin_memory() for x in rep.x_host]
     yh = torch.empty(1, N, dtype=torch.bfloat16).pin_memory()
     xd = torch.empty(1, K, dtype=torch.bfloat16, device="cuda")
     R = rep.R
 
-    def one(i):
-        r = i % R
+    def body(r):
         xd.copy_(xs[r], non_blocking=True)
         if path == "list":
             sgq.sgq_select(xd, 1, K, [rep.t[r]], rep.sidx, rep.scnt)
@@ -493,23 +496,51 @@ def run_e2e(rep: Replica, path: str, steps: int, warmup: int, dist: Dist):
             sgq.sgq_gemv_thresh(rep.qw[r], rep.sz[r], N, K, GROUP, xd, rep.t[r], rep.y, None,
                                 rep.ws)
         yh.copy_(rep.y, non_blocking=True)
-        torch.cuda.current_stream().synchronize()
+
+    stream = torch.cuda.Stream()
+    graphs = []
+    with torch.cuda.stream(stream):
+        for r in range(R):
+            body(r)                      # warm the path on this stream before capture
+        stream.synchronize()
+        for r in range(R):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                body(r)
+            graphs.append(g)
+    torch.cuda.synchronize()
+
+    def step_graph(i):
+        graphs[i % R].replay()
+        stream.synchronize()
         return float(yh[0, 0])
 
-    for i in range(max(3, warmup)):
-        one(i)
-    torch.cuda.synchronize()
-    dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(steps):
-        one(i)
-    e1.record()
-    torch.cuda.synchronize()
-    ms = dist.max(e0.elapsed_time(e1))
+    def step_eager(i):
+        body(i % R)
+        stream.synchronize()
+        return float(yh[0, 0])
+
+    def timed(fn):
+        with torch.cuda.stream(stream):
+            for i in range(max(3, warmup)):
+                fn(i)
+        torch.cuda.synchronize()
+        dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for i in range(steps):
+                fn(i)
+            e1.record(stream)
+        torch.cuda.synchronize()
+        return dist.max(e0.elapsed_time(e1))
+
+    ms = timed(step_graph)
+    ms_eager = timed(step_eager)
     b = dist.sum(sum(rep.abytes[i % R] for i in range(steps)))
     return {"value": round(b / (ms * 1e-3) / 1e9, 1), "unit": UNIT,
             "us_per_gemv": round(ms * 1e3 / steps, 3), "steps": steps,
+            "us_per_gemv_eager": round(ms_eager * 1e3 / steps, 3),
             "h2d_bytes_per_step": 2 * K, "d2h_bytes_per_step": 2 * N}
 
 
