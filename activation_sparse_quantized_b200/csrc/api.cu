@@ -515,6 +515,85 @@ int sgq_gemv_glu_dense(const void *qweight, const void *sz, int I, int K, int gr
     return run_gemv_glu(p, I, act, ws_bytes, workspace, stream);
 }
 
+size_t sgq_ffn_workspace_bytes(int H, int I)
+{
+    if (H <= 0 || I <= 0 || I > (1 << 29))
+        return 0;
+    return sgq::gemv_workspace_bytes(2 * I, 1) + sgq::gemv_workspace_bytes(H, 1);
+}
+
+int sgq_ffn(const void *qweight_gu, const void *sz_gu, const void *qweight_d, const void *sz_d,
+            int H, int I, int group, const void *x, float t_in, int act, float t_h, void *y,
+            float *y_f32, void *h_out, void *workspace, size_t ws_bytes, int32_t *status,
+            void *stream)
+{
+    if (act != SGQ_ACT_SILU && act != SGQ_ACT_RELU)
+        return SGQ_ERR_ACT;
+    if (I <= 0 || I > (1 << 29) || H <= 0)
+        return SGQ_ERR_SHAPE;
+    int rc = check_weights(2 * I, H, group);
+    if (rc)
+        return rc;
+    rc = check_weights(H, I, group);
+    if (rc)
+        return rc;
+    if (H % 8 != 0 || I % 8 != 0)
+        return SGQ_ERR_SHAPE;
+    if (!qweight_gu || !sz_gu || !qweight_d || !sz_d || !x || !y || !workspace)
+        return SGQ_ERR_NULL;
+    if (!aligned16(qweight_gu) || !aligned16(sz_gu) || !aligned16(qweight_d) ||
+        !aligned16(sz_d) || !aligned16(x) || !aligned16(y) || !aligned16(workspace) ||
+        (y_f32 && !aligned16(y_f32)) || (h_out && !aligned16(h_out)))
+        return SGQ_ERR_ALIGN;
+    if (ws_bytes < sgq_ffn_workspace_bytes(H, I))
+        return SGQ_ERR_WORKSPACE;
+    const int sms = current_device_sms();
+    if (sms < 0)
+        return sms;
+    float *gu = static_cast<float *>(workspace);
+    float *wsd = gu + sgq::gemv_workspace_bytes(2 * I, 1) / sizeof(float);
+    // gate and up as one accumulating GEMV (select fused): fp32 sums into gu
+    sgq::GemvProblem p1{};
+    p1.qweight = static_cast<const uint8_t *>(qweight_gu);
+    p1.sz = static_cast<const uint32_t *>(sz_gu);
+    p1.x = static_cast<const uint16_t *>(x);
+    p1.status = status;
+    p1.N = 2 * I;
+    p1.K = H;
+    p1.group = group;
+    p1.B = 1;
+    p1.t = t_in;
+    p1.source = sgq::ROWS_THRESH;
+    p1.accumulate = true;
+    p1.ws_acc = gu;
+    cudaError_t e = sgq::launch_gemv(p1, sms, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+        return fail_cuda(e);
+    // the down projection: h = bf16(act(gate) * up) and its active channels
+    // in the prologue, then the GEMV and the epilogue kernel (which re-zeroes gu)
+    sgq::GemvProblem p2{};
+    p2.qweight = static_cast<const uint8_t *>(qweight_d);
+    p2.sz = static_cast<const uint32_t *>(sz_d);
+    p2.x = static_cast<const uint16_t *>(x); // not read (rows come from gu)
+    p2.y = static_cast<uint16_t *>(y);
+    p2.y_f32 = y_f32;
+    p2.status = status;
+    p2.N = H;
+    p2.K = I;
+    p2.group = group;
+    p2.B = 1;
+    p2.t = t_h;
+    p2.source = sgq::ROWS_GLU;
+    p2.gu = gu;
+    p2.glu_act = act;
+    p2.h_out = static_cast<uint16_t *>(h_out);
+    p2.zero_extra = gu;
+    p2.zero_extra_n = 2 * I;
+    p2.ws_acc = wsd;
+    e = sgq::launch_gemv(p2, sms, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SGQ_OK : fail_cuda(e);
+}
+
 int sgq_glu(const void *gate, const void *up, void *h, int B, int I, int act, void *stream)
 {
     if (act != SGQ_ACT_SILU && act != SGQ_ACT_RELU)

@@ -109,7 +109,7 @@ __device__ __forceinline__ void channel_slice(const KParams &kp, int split, int 
 // ---------------------------------------------------------------------------
 template <int SRC, int NT, bool FILL_X = false>
 __device__ int build_rows(const KParams &kp, int split, int32_t *ridx, float *rx, int *scan,
-                          float *xs = nullptr)
+                          float *xs = nullptr, bool write_h = false)
 {
     const GemvProblem &p = kp.p;
     const int tid = threadIdx.x;
@@ -204,7 +204,19 @@ __device__ int build_rows(const KParams &kp, int split, int32_t *ridx, float *rx
             float v = 0.f;
             bool act = false;
             if (q < runs && c < c1) {
-                v = bf16_bits_to_float(__ldg(p.x + c));
+                if (SRC == ROWS_GLU) {
+                    // x = h = bf16(act(gate) * up) from the consumed fp32 sums
+                    // (written by the previous kernel's reductions: read from L2)
+                    const float gt = ld_cg_f32(p.gu + c), up = ld_cg_f32(p.gu + p.K + c);
+                    const float hv = (p.glu_act == SGQ_ACT_SILU) ? act_mul<SGQ_ACT_SILU>(gt, up)
+                                                                 : act_mul<SGQ_ACT_RELU>(gt, up);
+                    const uint16_t hb = float_to_bf16_bits(hv);
+                    if (write_h && p.h_out)
+                        p.h_out[c] = hb;
+                    v = bf16_bits_to_float(hb);
+                } else {
+                    v = bf16_bits_to_float(__ldg(p.x + c));
+                }
                 act = fabsf(v) > p.t;
             }
             mask[u] = __ballot_sync(0xffffffffu, act);
@@ -273,6 +285,10 @@ __global__ void __launch_bounds__(256) finalize_kernel(GemvProblem p)
         if (p.y_f32)
             *reinterpret_cast<float4 *>(p.y_f32 + o) = v;
     }
+    // sums consumed by this GEMV's prologue (the gate/up sums of a fused FFN)
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < p.zero_extra_n / 4;
+         e += gridDim.x * blockDim.x)
+        st_cg_v4(p.zero_extra + 4 * e, make_float4(0.f, 0.f, 0.f, 0.f));
 }
 
 // ---------------------------------------------------------------------------
@@ -494,7 +510,7 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_kernel(const KParams kp)
     };
     if (SRC != ROWS_LIST) {
         int c0, c1;
-        if (SRC == ROWS_THRESH || SRC == ROWS_MASK) {
+        if (SRC == ROWS_THRESH || SRC == ROWS_MASK || SRC == ROWS_GLU) {
             channel_slice(kp, split, c0, c1);
         } else {
             c0 = (int)((long long)p.K * split / kp.k_splits);
@@ -512,7 +528,8 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_kernel(const KParams kp)
     // Rows (build_rows ends with a barrier). Invalid list entries stay -1: they
     // are read as row 0 with x = 0, so they add nothing.
     const int nr = build_rows<SRC, kThreads1, (BW == 1)>(kp, split, ridx, rx, scan,
-                                                         reinterpret_cast<float *>(smem + L.xs));
+                                                         reinterpret_cast<float *>(smem + L.xs),
+                                                         tile == 0);
     auto row = [&](int j) { return (SRC == ROWS_LIST) ? max(ridx[j], 0) : ridx[j]; };
 
     if (SRC == ROWS_LIST) {
@@ -546,7 +563,7 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_kernel(const KParams kp)
     // x of this warp's rows and batch rows (after the weights are in flight),
     // unless build_rows already read it (threshold; bitmask at batch 1).
     // Padded batch rows and invalid list entries get x = 0.
-    if (!(SRC == ROWS_THRESH || (SRC == ROWS_MASK && BW == 1))) {
+    if (!(SRC == ROWS_THRESH || SRC == ROWS_GLU || (SRC == ROWS_MASK && BW == 1))) {
         for (int e = lane; e < n * BW; e += 32) {
             const int j = e / BW, bb = e - j * BW;
             const int k = ridx[wa + j];
@@ -843,7 +860,7 @@ cudaError_t launch_gemv_and_finalize(Kern kern, int grid, int block, size_t smem
     cudaError_t err = launch_pdl(kern, grid, block, smem, stream, kp);
     if (err != cudaSuccess || kp.p.accumulate)
         return err;
-    const int quads = kp.p.B * (kp.p.N / 4);
+    const int quads = std::max(kp.p.B * (kp.p.N / 4), kp.p.zero_extra_n / 4);
     const int fgrid = std::max(1, std::min(ceil_div(quads, 256), 148));
     switch (kp.p.epilogue) {
     case EPI_GLU_SILU:
@@ -880,12 +897,14 @@ cudaError_t launch_gemv_t(KParams kp, int num_sms, cudaStream_t stream)
         kp.span_cap = std::min(G, ceil_div(p.K, (long long)kp.k_splits << kp.lg) + 2);
         L = smem1_layout(kp.span_cap, kp.rows_cap, bp, BW, NM);
         // the threshold path handles at most 4 runs of 32 channels per warp
-        const bool runs_ok = (SRC != ROWS_THRESH) || (kp.rows_cap <= 4 * kThreads1);
+        const bool fused_select = (SRC == ROWS_THRESH || SRC == ROWS_GLU);
+        const bool runs_ok = !fused_select || (kp.rows_cap <= 4 * kThreads1);
         if ((L.total <= kMaxSmem && runs_ok) || kp.k_splits >= p.K / 8)
             break;
         kp.k_splits *= 2;
     }
-    if (L.total > kMaxSmem || (SRC == ROWS_THRESH && kp.rows_cap > 4 * kThreads1))
+    if (L.total > kMaxSmem ||
+        ((SRC == ROWS_THRESH || SRC == ROWS_GLU) && kp.rows_cap > 4 * kThreads1))
         return cudaErrorInvalidConfiguration;
     return launch_gemv_and_finalize(gemv_kernel<SRC, BW, NM>, kp.n_tiles * kp.k_splits,
                                     kThreads1, L.total, stream, kp);
@@ -918,6 +937,7 @@ cudaError_t launch_gemv(const GemvProblem &p, int num_sms, cudaStream_t stream)
     case ROWS_LIST: return launch_src<ROWS_LIST>(kp, num_sms, stream);
     case ROWS_DENSE: return launch_src<ROWS_DENSE>(kp, num_sms, stream);
     case ROWS_MASK: return launch_src<ROWS_MASK>(kp, num_sms, stream);
+    case ROWS_GLU: return launch_gemv_t<ROWS_GLU, 1>(kp, num_sms, stream); // batch 1
     default:
         // the API admits the threshold path at B = 1 only
         if (p.keep)

@@ -112,6 +112,13 @@ __device__ __forceinline__ float4 ld_cg_v4(const float *gptr)
     return v;
 }
 
+__device__ __forceinline__ float ld_cg_f32(const float *gptr)
+{
+    float v;
+    asm volatile("ld.global.cg.f32 %0, [%1];\n" : "=f"(v) : "l"(gptr) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ void st_cg_v4(float *gptr, float4 v)
 {
     asm volatile("st.global.cg.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"l"(gptr), "f"(v.x),

@@ -19,6 +19,7 @@ enum RowSource : int {
     ROWS_DENSE = 1,  // every channel
     ROWS_THRESH = 2, // |x[k]| > t, found by each CTA for its own channel slice
     ROWS_MASK = 3,   // bit k of a device bitmask, decoded by each CTA for its own slice
+    ROWS_GLU = 4,    // x = bf16(act(gate) * up) from the fp32 sums of a gate/up GEMV, |x| > t
 };
 
 // What the epilogue writes from the fp32 sums of the N GEMV outputs.
@@ -45,6 +46,14 @@ struct GemvProblem {
     int source;
     int epilogue; // Epilogue; y (and y_f32) are [B][N/2] for the GLU epilogues
     bool accumulate; // add into ws_acc (the caller's fp32 [B][N]) and launch no epilogue kernel
+    // ROWS_GLU: gate = gu[k], up = gu[K + k] (fp32 sums, 2K floats), the activation,
+    // and an optional bf16 copy of x = h written once per channel
+    const float *gu;
+    int glu_act;
+    uint16_t *h_out;
+    // the epilogue kernel also zeroes zero_extra[0 .. zero_extra_n) (consumed sums)
+    float *zero_extra;
+    int zero_extra_n;
 };
 
 // Bytes of workspace (partial sums + tile counters) for N outputs, B rows.

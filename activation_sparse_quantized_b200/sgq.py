@@ -33,6 +33,7 @@ EXPORTS = (
     "sgq_layout_version", "sgq_gemv_thresh_noalloc", "sgq_gemv_glu", "sgq_gemv_glu_thresh",
     "sgq_gemv_glu_dense", "sgq_select_mask", "sgq_gemv_mask", "sgq_packed_sizes_nm",
     "sgq_pack_nm", "sgq_gemv_nm", "sgq_gemv_nm_thresh", "sgq_gemv_acc", "sgq_gemv_thresh_acc",
+    "sgq_ffn_workspace_bytes", "sgq_ffn",
 )
 
 
@@ -92,6 +93,8 @@ def _declare(lib):
         "sgq_gemv_nm_thresh": ([P, P, P, I, I, I, P, F, P, P, P, Z, P, P], I),
         "sgq_gemv_acc": ([P, P, I, I, I, P, I, P, P, P, P, P], I),
         "sgq_gemv_thresh_acc": ([P, P, I, I, I, P, F, P, P, P], I),
+        "sgq_ffn_workspace_bytes": ([I, I], Z),
+        "sgq_ffn": ([P, P, P, P, I, I, I, P, F, I, F, P, P, P, P, Z, P, P], I),
         "sgq_status_string": ([I], ctypes.c_char_p),
         "sgq_last_cuda_error": ([], I),
         "sgq_layout_version": ([], I),
@@ -256,6 +259,24 @@ def sgq_gemv_glu_dense(qweight, sz, I, K, group, x, B, act, h, h_f32, workspace,
         _ptr(qweight), _ptr(sz), I, K, group, _ptr(x), B, act, _ptr(h), _ptr(h_f32),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status),
         _stream(stream)))
+
+
+def sgq_ffn_workspace_bytes(H: int, I: int) -> int:
+    return load().sgq_ffn_workspace_bytes(H, I)
+
+
+def sgq_ffn(qweight_gu, sz_gu, qweight_d, sz_d, H, I, group, x, t_in, act, t_h, y, y_f32,
+            h_out, workspace, status=None, stream=None):
+    """The batch-1 decode FFN in three kernels (gate/up GEMV, down GEMV with the
+    GLU and the selection of h in its prologue, epilogue)."""
+    _check("sgq_ffn", load().sgq_ffn(
+        _ptr(qweight_gu), _ptr(sz_gu), _ptr(qweight_d), _ptr(sz_d), H, I, group, _ptr(x),
+        float(t_in), act, float(t_h), _ptr(y), _ptr(y_f32), _ptr(h_out), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream)))
+
+
+def alloc_ffn_workspace(H, I, device="cuda"):
+    return torch.zeros(sgq_ffn_workspace_bytes(H, I) // 4, dtype=torch.int32, device=device)
 
 
 def sgq_glu(gate, up, h, B, I, act, stream=None):

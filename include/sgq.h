@@ -292,6 +292,34 @@ int sgq_gemv_glu_dense(const void *qweight, const void *sz, int I, int K, int gr
                        void *workspace, size_t ws_bytes, int32_t *status, void *stream);
 
 /*
+ * The whole decode FFN at batch 1, three kernels:
+ *
+ *     h = bf16(act(W_g[:, S] x[S]) * (W_u[:, S] x[S])),  S = { k : |x_k| > t_in }
+ *     y = W_d[:, T] h[T],                                  T = { i : |h_i| > t_h }
+ *
+ * The gate/up GEMV (select fused) leaves its fp32 sums in the workspace; the
+ * down GEMV's prologue forms h from them for its own slice of the I channels
+ * (the same bf16 h as sgq_gemv_glu_thresh), selects T there and gathers only
+ * those rows ("SVD Contextual Sparsity Predictors for Fast LLM Inference",
+ * Abstract: with ReLU gating and t_h = 0, T is the nonzero neurons); h is not
+ * written to memory unless h_out is given. The epilogue kernel writes y and
+ * re-zeroes the workspace.
+ *
+ *   qweight_gu, sz_gu  sgq_pack of the stacked [W_g; W_u] (N = 2I, K = H).
+ *   qweight_d, sz_d    sgq_pack of W_d (N = H, K = I).
+ *   x                  bf16 [1][H]; y bf16 [1][H]; y_f32 optional fp32 [1][H].
+ *   h_out              optional bf16 [1][I] copy of h (NULL = not written).
+ *   workspace          sgq_ffn_workspace_bytes(H, I) bytes, zero-filled once.
+ * Requires H % 8 == 0 and I % 8 == 0 besides the sgq_pack conditions.
+ * Returns as sgq_gemv, plus SGQ_ERR_ACT.
+ */
+size_t sgq_ffn_workspace_bytes(int H, int I);
+int sgq_ffn(const void *qweight_gu, const void *sz_gu, const void *qweight_d, const void *sz_d,
+            int H, int I, int group, const void *x, float t_in, int act, float t_h, void *y,
+            float *y_f32, void *h_out, void *workspace, size_t ws_bytes, int32_t *status,
+            void *stream);
+
+/*
  * sgq_gemv_thresh without a workspace argument, for callers that cannot
  * allocate device memory (no cudaMalloc available to them, or none allowed
  * during the call). The pages have no counterpart of this entry point; it is a

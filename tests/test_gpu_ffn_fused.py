@@ -229,3 +229,63 @@ def test_qkv_stacked_single_gemv():
         y64, sa, _ = oracle.gemv(q, s, z, g, xb, idx)
         check_y(y[:, o:o + n], y32[:, o:o + n], y64, sa, f"stacked {name}")
         o += n
+
+
+# ---------------------------------------------------------------------------
+# sgq_ffn: the decode FFN in three kernels (h formed and selected in the down
+# projection's prologue)
+# ---------------------------------------------------------------------------
+
+def run_ffn_case(H, I, g, act, t_in_sparsity, t_h_sparsity, seed):
+    Wg, Wu = weights(I, H, seed)
+    Wd = wl.weight(H, I, seed + 2)
+    x = wl.x_gaussian(1, H, seed + 3)
+    t_in = wl.percentile_threshold(x[0], t_in_sparsity) if t_in_sparsity > 0 else -1.0
+    qgu, sgu, _ = gpu_pack(torch.cat([Wg, Wu], 0), g)
+    qd, sd, _ = gpu_pack(Wd, g)
+    # oracle h (fp64) for the threshold of h and the h check
+    _, h64, a64, u64, sag, sau = fused_expect(Wg, Wu, g, x, [t_in], act)
+    hb64 = np.abs(h64[0])
+    t_h = 0.0 if t_h_sparsity == 0 else float(np.quantile(hb64, t_h_sparsity))
+    ws = sgq.alloc_ffn_workspace(H, I)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    q, s, z = oracle_codes(Wd, g)
+    for call in range(2):                      # the workspace must come back to zero
+        y = torch.full((1, H), float("nan"), dtype=torch.bfloat16, device=DEV)
+        y32 = torch.full((1, H), float("nan"), dtype=torch.float32, device=DEV)
+        h = torch.full((1, I), float("nan"), dtype=torch.bfloat16, device=DEV)
+        sgq.sgq_ffn(qgu, sgu, qd, sd, H, I, g, x.to(DEV), t_in, act, t_h, y, y32, h, ws, status)
+        hbits = bits(h)
+        # h against the oracle's fp64 h (the GLU bound, bf16 part)
+        hv = bf16_values(hbits)
+        L = LIP[act]
+        eg, eu = 1e-3 * sag, 1e-3 * sau
+        tol = (L * eg * (np.abs(u64) + eu) + np.abs(a64) * eu
+               + 2.0 ** -20 * (np.abs(a64) + L * eg) * (np.abs(u64) + eu)) * 1.01 \
+            + 2.0 ** -8 * np.abs(h64) + 1e-37
+        assert np.all(np.abs(hv - h64) <= tol), f"ffn h call {call}"
+        # y against the oracle's down GEMV over the GPU's own h and t_h
+        idx = oracle.select(hbits, [t_h])
+        y64, sa, _ = oracle.gemv(q, s, z, g, hbits, idx)
+        check_y(y, y32, y64, sa, f"ffn y call {call}")
+        assert bool((ws == 0).all().item()) and int(status.item()) == 0
+    return idx.size / I
+
+
+def test_ffn_three_kernels_llama8b_silu():
+    shp = wl.LLAMA8B_LAYER["gate"]
+    frac = run_ffn_case(shp["K"], shp["N"], shp["group"], SILU, 0.5, 0.5, 380)
+    assert 0.45 < frac < 0.55
+
+
+def test_ffn_three_kernels_reglu_zeros():
+    """ReGLU: dense input, ReLU gating, t_h = 0: the down projection reads
+    exactly the nonzero neurons."""
+    cfg = wl.REGLU_FFN
+    frac = run_ffn_case(cfg["hidden"], cfg["inter"], cfg["group"], RELU, 0.0, 0.0, 390)
+    assert 0.4 < frac < 0.6
+
+
+@pytest.mark.parametrize("H,I,g", [(512, 1056, 32), (1024, 3136, 64)])
+def test_ffn_three_kernels_ragged(H, I, g):
+    run_ffn_case(H, I, g, SILU, 0.5, 0.7, 400)
