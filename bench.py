@@ -171,6 +171,26 @@ def measured_peak():
         return 6650.0, "fallback"
 
 
+def read_peak_gbs(nbytes: int = 2 << 30, reps: int = 10) -> float:
+    """A read-only streaming peak measured here: device time of a reduction
+    over a buffer much larger than L2 (torch's fp32 sum: one read of the
+    buffer, no conversion pass), the best of several runs."""
+    buf = torch.ones(nbytes // 4, dtype=torch.float32, device="cuda")
+    torch.sum(buf)
+    torch.cuda.synchronize()
+    best = 1e30
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        torch.sum(buf)
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    del buf
+    torch.cuda.empty_cache()
+    return nbytes / (best * 1e-3) / 1e9
+
+
 def source_hash(*names):
     h = hashlib.sha256()
     for n in names:
@@ -403,6 +423,7 @@ def run_ours(args, dist: Dist):
     elif dom == "mask":   # K/8 bytes of mask instead of the 4a-byte index list
         k_bytes = k_bytes - 4 * np.mean(rep.active) + K // 8
     peak, peak_kind = measured_peak()
+    rpk = read_peak_gbs()
     achieved = k_bytes / (k_us * 1e-6) / 1e9
     src = source_hash("gemv.cu", "sgq_device.cuh")
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
@@ -413,6 +434,7 @@ def run_ours(args, dist: Dist):
                            "mask": "sgq_gemv_mask call"}[dom],
                 "kernel_us": round(k_us, 3), "algorithmic_bytes": int(k_bytes),
                 "frac_of_8TBps": round(achieved / 8000.0, 4),
+                "read_peak_gbs": round(rpk, 1), "frac_of_read_peak": round(achieved / rpk, 4),
                 "timed": ("the GEMV kernel alone on its stream, launched through the "
                           "accumulating entry point (sgq_gemv_thresh_acc / sgq_gemv_acc): the "
                           "same kernel, its split-K sums added into fp32 y, no epilogue kernel; "
