@@ -289,3 +289,16 @@ def test_ffn_three_kernels_reglu_zeros():
 @pytest.mark.parametrize("H,I,g", [(512, 1056, 32), (1024, 3136, 64)])
 def test_ffn_three_kernels_ragged(H, I, g):
     run_ffn_case(H, I, g, SILU, 0.5, 0.7, 400)
+
+
+@pytest.mark.parametrize("B,act", [(2, RELU), (4, SILU)])
+def test_glu_fused_dense_batch(B, act):
+    """Dense gate/up at B > 1 (two batch rows per warp) with the GLU epilogue."""
+    I, K, g = 2048, 2048, 128
+    Wg, Wu = weights(I, K, 450)
+    x = wl.x_gaussian(B, K, 451)
+    gg = GpuGlu(Wg, Wu, g, B)
+    h, h32 = gg.run("dense", x.to(DEV), [-1.0] * B, act)
+    _, h64, a64, u64, sag, sau = fused_expect(Wg, Wu, g, x, [-1.0] * B, act, dense=True)
+    check_h(h, h32, h64, a64, u64, sag, sau, act, what=f"dense GLU B={B}")
+    assert bool((gg.ws == 0).all().item())

@@ -441,3 +441,27 @@ def test_ffn_pipeline_end_to_end(act):
     yv = bf16_values(bits(y))[0]
     tol = 1e-3 * sa[0] + 2.0 ** -7 * spread + 2.0 ** -8 * np.abs(y64[0])
     assert np.all(np.abs(yv - y64[0]) <= tol)
+
+
+@pytest.mark.parametrize("B", [2, 5, 16])
+def test_gemv_batch_bad_index_is_skipped(B):
+    """Invalid list entries at B > 1 (every batch group reads the same rows):
+    skipped for every row, flagged, and the workspace left zero. Per-row
+    sparsity 0.9 keeps the union (1 - 0.9^B of K) short of K, so the two planted
+    entries do not push the count past K (which would be clamped)."""
+    case = wl.gemv_case(N=2048, K=4096, group=128, B=B, sparsity=0.9, seed=440)
+    g = GpuGemv(case.W, case.group, B)
+    x_d = case.x.to(DEV)
+    xb = bits(case.x)
+    good = oracle.select(xb, case.t)
+    assert good.size + 2 <= case.K
+    bad = np.concatenate([good[:7], [-5], good[7:300], [case.K], good[300:]]).astype(np.int32)
+    idx = torch.from_numpy(bad).to(DEV)
+    cnt = torch.tensor([bad.size], dtype=torch.int32, device=DEV)
+    y, y32 = g.gemv(x_d, idx, cnt)
+    q, s, z = oracle_codes(case.W, case.group)
+    y64, sa, _ = oracle.gemv(q, s, z, case.group, xb, good)
+    check_y(y, y32, y64, sa, f"batch {B} bad index")
+    assert not (g.status.item() & sgq.SGQ_STATUS_BAD_COUNT)
+    assert g.status.item() & sgq.SGQ_STATUS_BAD_INDEX
+    assert g.workspace_is_zero()
