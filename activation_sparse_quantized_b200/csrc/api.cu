@@ -116,6 +116,23 @@ int sgq_last_cuda_error(void)
     return g_last_cuda_error;
 }
 
+int sgq_read_status(int32_t *dev_status, int32_t *host_out, int clear, void *stream)
+{
+    if (!dev_status || !host_out)
+        return SGQ_ERR_NULL;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(host_out, dev_status, sizeof(int32_t),
+                                    cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess)
+        return fail_cuda(e);
+    if (clear) {
+        e = cudaMemsetAsync(dev_status, 0, sizeof(int32_t), st);
+        if (e != cudaSuccess)
+            return fail_cuda(e);
+    }
+    return SGQ_OK;
+}
+
 const char *sgq_status_string(int code)
 {
     switch (code) {

@@ -33,7 +33,7 @@ EXPORTS = (
     "sgq_layout_version", "sgq_gemv_thresh_noalloc", "sgq_gemv_glu", "sgq_gemv_glu_thresh",
     "sgq_gemv_glu_dense", "sgq_select_mask", "sgq_gemv_mask", "sgq_packed_sizes_nm",
     "sgq_pack_nm", "sgq_gemv_nm", "sgq_gemv_nm_thresh", "sgq_gemv_acc", "sgq_gemv_thresh_acc",
-    "sgq_ffn_workspace_bytes", "sgq_ffn",
+    "sgq_ffn_workspace_bytes", "sgq_ffn", "sgq_read_status",
 )
 
 
@@ -94,6 +94,7 @@ def _declare(lib):
         "sgq_gemv_acc": ([P, P, I, I, I, P, I, P, P, P, P, P], I),
         "sgq_gemv_thresh_acc": ([P, P, I, I, I, P, F, P, P, P], I),
         "sgq_ffn_workspace_bytes": ([I, I], Z),
+        "sgq_read_status": ([P, P, I, P], I),
         "sgq_ffn": ([P, P, P, P, I, I, I, P, F, I, F, P, P, P, P, Z, P, P], I),
         "sgq_status_string": ([I], ctypes.c_char_p),
         "sgq_last_cuda_error": ([], I),
@@ -124,6 +125,16 @@ def _check(fn, rc):
 # --------------------------------------------------------------------------
 # The C entry points, one to one.
 # --------------------------------------------------------------------------
+
+def sgq_read_status(status, clear=True, stream=None) -> int:
+    """The SGQ_STATUS_* bits of a device status word (synchronises the stream
+    to return the value; the C call itself only enqueues the copy)."""
+    out = ctypes.c_int32(0)
+    _check("sgq_read_status", load().sgq_read_status(_ptr(status), ctypes.byref(out),
+                                                     1 if clear else 0, _stream(stream)))
+    (stream or torch.cuda.current_stream()).synchronize()
+    return out.value
+
 
 def sgq_layout_version() -> int:
     return load().sgq_layout_version()

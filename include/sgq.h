@@ -338,6 +338,15 @@ int sgq_gemv_thresh_noalloc(const void *qweight, const void *sz, int N, int K, i
                             const void *x, float t, void *y, float *y_f32, int32_t *status,
                             void *stream);
 
+/*
+ * Read the device status word (the SGQ_STATUS_* bits that calls OR into it):
+ * enqueues on `stream` a copy of *dev_status into *host_out (host memory;
+ * the value is there once the stream has reached this point, e.g. after the
+ * caller synchronises it), then, if `clear` is nonzero, sets *dev_status to 0.
+ * Does not synchronise.
+ */
+int sgq_read_status(int32_t *dev_status, int32_t *host_out, int clear, void *stream);
+
 /* Text for a return code (static string). */
 const char *sgq_status_string(int code);
 

@@ -112,6 +112,7 @@ def test_host_argument_checks(lib):
                                    fake, wsg, None, None) == -7
     assert lib.sgq_gemv_glu_dense(fake, fake, 14336, 4096, 96, fake, 1, 0, fake, None, fake,
                                   wsg, None, None) == -3
+    assert lib.sgq_read_status(None, None, 0, None) == -1
     # 2:4 layout: N % 64, null keep, sizes
     assert lib.sgq_pack_nm(fake, 4064, 14336, 128, fake, fake, fake, None, None) == -2
     assert lib.sgq_gemv_nm(fake, None, fake, 4096, 14336, 128, fake, fake, fake, fake, None,

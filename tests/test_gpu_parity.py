@@ -465,3 +465,12 @@ def test_gemv_batch_bad_index_is_skipped(B):
     assert not (g.status.item() & sgq.SGQ_STATUS_BAD_COUNT)
     assert g.status.item() & sgq.SGQ_STATUS_BAD_INDEX
     assert g.workspace_is_zero()
+
+
+def test_read_status_returns_and_clears_the_word():
+    W = wl.weight(64, 128, 8)
+    W[3, 9] = float("nan")
+    _, _, st = gpu_pack(W, 64)
+    assert sgq.sgq_read_status(st, clear=False) & sgq.SGQ_STATUS_NONFINITE_W
+    assert sgq.sgq_read_status(st, clear=True) & sgq.SGQ_STATUS_NONFINITE_W
+    assert sgq.sgq_read_status(st) == 0 and int(st.item()) == 0
