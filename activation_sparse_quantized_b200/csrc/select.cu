@@ -6,10 +6,11 @@
 // exactly the nonzero channels, the ReLU zeros of "SVD Contextual Sparsity
 // Predictors", Abstract). The list is written in ascending order.
 //
-// One CTA of 1024 threads walks the channels in tiles of 8 per thread:
-// 16-byte loads of each batch row, a per-thread 8-bit mask, a warp shuffle
-// scan and a cross-warp scan in shared memory, then each thread writes its
-// indices at its exclusive offset. The activation vector is small (2*B*K
+// One CTA of 1024 threads walks the channels in tiles of 16 per thread:
+// 16-byte loads of each batch row, a per-thread 16-bit mask, a warp shuffle
+// scan and a cross-warp scan in shared memory; each thread puts its indices at
+// its exclusive offset in a shared-memory copy of the tile, which the CTA then
+// writes out with coalesced stores. The activation vector is small (2*B*K
 // bytes), so one CTA keeps the whole list ordered without any inter-CTA wait.
 #include "sgq_device.cuh"
 #include "sgq_launch.h"
@@ -28,24 +29,35 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const uint16_t *__r
 {
     __shared__ int warp_excl[kSelWarps];
     __shared__ int tile_total;
+    extern __shared__ int s_idx[]; // one tile's indices, written out coalesced
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
     int offset = 0;
-    for (int base = 0; base < K; base += 8 * kSelThreads) {
-        const int c0 = base + tid * 8;
+    // tiles of 16 channels per thread: two 16-byte loads per batch row, both
+    // in flight before either is used (K <= 16384 is a single tile)
+    for (int base = 0; base < K; base += 16 * kSelThreads) {
+        const int c0 = base + tid * 16;
         uint32_t mask = 0;
-        if (c0 < K) {
-            for (int b = 0; b < B; ++b) {
-                uint4 v = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)b * K + c0));
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-                const float t = th.t[b];
+        for (int b = 0; b < B; ++b) {
+            uint4 v[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+                v[h] = (c0 + 8 * h < K)
+                           ? __ldg(reinterpret_cast<const uint4 *>(x + (size_t)b * K + c0 + 8 * h))
+                           : make_uint4(0u, 0u, 0u, 0u);
+            const float t = th.t[b];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                if (c0 + 8 * h >= K)
+                    continue;
+                const uint32_t w[4] = {v[h].x, v[h].y, v[h].z, v[h].w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     float lo = fabsf(__uint_as_float(w[e] << 16));
                     float hi = fabsf(__uint_as_float(w[e] & 0xffff0000u));
-                    mask |= (lo > t ? 1u : 0u) << (2 * e);
-                    mask |= (hi > t ? 1u : 0u) << (2 * e + 1);
+                    mask |= (lo > t ? 1u : 0u) << (8 * h + 2 * e);
+                    mask |= (hi > t ? 1u : 0u) << (8 * h + 2 * e + 1);
                 }
             }
         }
@@ -74,14 +86,18 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const uint16_t *__r
                 tile_total = wi;
         }
         __syncthreads();
-        int pos = offset + warp_excl[warp] + incl - cnt;
+        int pos = warp_excl[warp] + incl - cnt; // position inside the tile
         while (mask) {
             const int j = __ffs(mask) - 1;
-            idx[pos++] = c0 + j;
+            s_idx[pos++] = c0 + j;
             mask &= mask - 1;
         }
-        offset += tile_total;
-        __syncthreads(); // warp_excl / tile_total are rewritten by the next tile
+        __syncthreads();
+        const int tt = tile_total;
+        for (int i = tid; i < tt; i += kSelThreads)
+            idx[offset + i] = s_idx[i];
+        offset += tt;
+        __syncthreads(); // warp_excl / tile_total / s_idx are rewritten by the next tile
     }
     if (tid == 0)
         *count = offset;
@@ -92,9 +108,9 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const uint16_t *__r
 // Efficient LLM Inference", Abstract, and the shared-memory bitmap decoding of
 // "Unified Static-Dynamic Pruning for Efficient LLM Inference", Abstract, in
 // that page's similar-work list): bit k % 32 of word k / 32 is set when
-// channel k is active. Each thread forms the 8-bit mask of its 8 channels as
-// above; the lead lane of every 4 lanes gathers its neighbours' bytes with
-// three shuffles and stores one 32-bit word. The CTA also reduces the count.
+// channel k is active. Each thread forms the 16-bit mask of its 16 channels as
+// above; the even lane of every pair takes its neighbour's half with one
+// shuffle and stores one 32-bit word. The CTA also reduces the count.
 __global__ void __launch_bounds__(kSelThreads) select_mask_kernel(const uint16_t *__restrict__ x,
                                                                   int B, int K, Thresholds th,
                                                                   uint32_t *__restrict__ mask,
@@ -105,29 +121,35 @@ __global__ void __launch_bounds__(kSelThreads) select_mask_kernel(const uint16_t
     const int lane = tid & 31;
     const int warp = tid >> 5;
     int total = 0;
-    for (int base = 0; base < K; base += 8 * kSelThreads) {
-        const int c0 = base + tid * 8;
+    for (int base = 0; base < K; base += 16 * kSelThreads) {
+        const int c0 = base + tid * 16;
         uint32_t m = 0;
-        if (c0 < K) {
-            for (int b = 0; b < B; ++b) {
-                uint4 v = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)b * K + c0));
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-                const float t = th.t[b];
+        for (int b = 0; b < B; ++b) {
+            uint4 v[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+                v[h] = (c0 + 8 * h < K)
+                           ? __ldg(reinterpret_cast<const uint4 *>(x + (size_t)b * K + c0 + 8 * h))
+                           : make_uint4(0u, 0u, 0u, 0u);
+            const float t = th.t[b];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                if (c0 + 8 * h >= K)
+                    continue;
+                const uint32_t w[4] = {v[h].x, v[h].y, v[h].z, v[h].w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     float lo = fabsf(__uint_as_float(w[e] << 16));
                     float hi = fabsf(__uint_as_float(w[e] & 0xffff0000u));
-                    m |= (lo > t ? 1u : 0u) << (2 * e);
-                    m |= (hi > t ? 1u : 0u) << (2 * e + 1);
+                    m |= (lo > t ? 1u : 0u) << (8 * h + 2 * e);
+                    m |= (hi > t ? 1u : 0u) << (8 * h + 2 * e + 1);
                 }
             }
         }
         total += __popc(m);
-        const uint32_t b1 = __shfl_down_sync(0xffffffffu, m, 1);
-        const uint32_t b2 = __shfl_down_sync(0xffffffffu, m, 2);
-        const uint32_t b3 = __shfl_down_sync(0xffffffffu, m, 3);
-        if ((lane & 3) == 0 && c0 < K)
-            mask[c0 >> 5] = m | (b1 << 8) | (b2 << 16) | (b3 << 24);
+        const uint32_t m1 = __shfl_down_sync(0xffffffffu, m, 1);
+        if ((lane & 1) == 0 && c0 < K)
+            mask[c0 >> 5] = m | (m1 << 16);
     }
 #pragma unroll
     for (int d = 16; d > 0; d >>= 1)
@@ -150,7 +172,12 @@ __global__ void __launch_bounds__(kSelThreads) select_mask_kernel(const uint16_t
 cudaError_t launch_select(const uint16_t *x, int B, int K, const Thresholds &th, int32_t *idx,
                           int32_t *count, cudaStream_t stream)
 {
-    select_kernel<<<1, kSelThreads, 0, stream>>>(x, B, K, th, idx, count);
+    const size_t smem = sizeof(int) * 16 * kSelThreads; // 64 KB: one tile of indices
+    cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess)
+        return e;
+    select_kernel<<<1, kSelThreads, smem, stream>>>(x, B, K, th, idx, count);
     return cudaGetLastError();
 }
 
