@@ -41,6 +41,7 @@
 //  * Programmatic dependent launch: a GEMV lets the next kernel in the stream
 //    launch early and itself waits for the previous one before it reads x,
 //    idx or count or writes anything; only the packed weights are read before.
+#include "gemv_rows.cuh"
 #include "sgq_device.cuh"
 #include "sgq_launch.h"
 
@@ -49,201 +50,6 @@
 namespace sgq {
 
 namespace {
-
-constexpr int kTileN1 = 1024;            // B = 1: outputs per tile, 32 per lane
-constexpr int kRowBytes1 = kTileN1 / 2;  // bytes of one packed row per tile
-
-struct KParams {
-    GemvProblem p;
-    int n_tiles;
-    int k_splits;
-    int rows_cap;  // capacity of the per-CTA row arrays
-    int span_cap;  // groups of scale/zero staged in shared memory per CTA
-    int lg;        // log2(group)
-    int nb;        // batch groups of warps (1 for B = 1)
-};
-
-__device__ __forceinline__ int warp_max_exponent(float m)
-{
-#pragma unroll
-    for (int d = 16; d > 0; d >>= 1)
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, d));
-    if (!(m > 0.0f) || isinf(m))
-        return INT32_MIN; // all zero (or non-finite): no scaling
-    return ilogbf(m);
-}
-
-// Exclusive prefix, over runs, of the per-run counts in scan[] for the runs
-// 32c .. 32c + 31 (one per lane), plus the carry from the earlier chunks: a
-// warp scan instead of a serial walk over shared memory. Returns the lane's
-// exclusive prefix; *chunk_total receives the chunk's sum (every lane).
-__device__ __forceinline__ int chunk_prefix(const int *scan, int runs, int c, int carry,
-                                            int *chunk_total)
-{
-    const int lane = threadIdx.x & 31;
-    const int r = c * 32 + lane;
-    const int v = (r < runs) ? scan[r] : 0;
-    int incl = v;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, d);
-        if (lane >= d)
-            incl += t;
-    }
-    *chunk_total = __shfl_sync(0xffffffffu, incl, 31);
-    return carry + incl - v;
-}
-
-// Channel slice [c0, c1) of split s when channels are dealt out in runs of 8.
-__device__ __forceinline__ void channel_slice(const KParams &kp, int split, int &c0, int &c1)
-{
-    const int K8 = kp.p.K / 8;
-    c0 = (int)((long long)K8 * split / kp.k_splits) * 8;
-    c1 = (int)((long long)K8 * (split + 1) / kp.k_splits) * 8;
-}
-
-// ---------------------------------------------------------------------------
-// Row lists: fill ridx[0..nr) (and rx = x for ROWS_THRESH) for this CTA and
-// return nr. Entries outside [0, K) become -1 (their x is 0; they read row 0).
-// Must be called by all threads; ends with a barrier.
-// ---------------------------------------------------------------------------
-template <int SRC, int NT, bool FILL_X = false>
-__device__ int build_rows(const KParams &kp, int split, int32_t *ridx, float *rx, int *scan,
-                          float *xs = nullptr, bool write_h = false)
-{
-    const GemvProblem &p = kp.p;
-    const int tid = threadIdx.x;
-    if (SRC == ROWS_LIST) {
-        const int c = __ldg(p.count);
-        const int a = c < 0 ? 0 : (c > p.K ? p.K : c);
-        if (a != c && tid == 0 && blockIdx.x == 0)
-            set_status(p.status, SGQ_STATUS_BAD_COUNT);
-        const int r0 = (int)((long long)a * split / kp.k_splits);
-        const int r1 = (int)((long long)a * (split + 1) / kp.k_splits);
-        for (int j = tid; j < r1 - r0; j += NT) {
-            int k = __ldg(p.idx + r0 + j);
-            if ((unsigned)k >= (unsigned)p.K) {
-                set_status(p.status, SGQ_STATUS_BAD_INDEX);
-                k = -1;
-            }
-            ridx[j] = k;
-        }
-        __syncthreads();
-        return r1 - r0;
-    } else if (SRC == ROWS_DENSE) {
-        const int r0 = (int)((long long)p.K * split / kp.k_splits);
-        const int r1 = (int)((long long)p.K * (split + 1) / kp.k_splits);
-        for (int j = tid; j < r1 - r0; j += NT)
-            ridx[j] = r0 + j;
-        __syncthreads();
-        return r1 - r0;
-    } else if (SRC == ROWS_MASK) {
-        // Decode this CTA's channel slice of the bitmask: runs of 32 channels,
-        // one per lane, a ballot per run, the count of each run in scan[]; a
-        // second pass recomputes the ballots (the mask words stay in L1) and
-        // writes each active channel at its ascending position. With FILL_X
-        // (batch 1) the first pass also reads the slice of x, coalesced and
-        // alongside the mask words, into xs[], and the second copies the x of
-        // each active channel into rx[].
-        int c0, c1;
-        channel_slice(kp, split, c0, c1);
-        const int lane = tid & 31, warp = tid >> 5;
-        const int runs = (c1 - c0 + 31) / 32;
-        auto run_bits = [&](int q) -> uint32_t {
-            const int c = c0 + q * 32 + lane;
-            const bool act = (c < c1) && ((__ldg(p.mask + (c >> 5)) >> (c & 31)) & 1u);
-            return __ballot_sync(0xffffffffu, act);
-        };
-        for (int q = warp; q < runs; q += NT / 32) {
-            if (FILL_X) {
-                const int c = c0 + q * 32 + lane;
-                if (c < c1)
-                    xs[c - c0] = bf16_bits_to_float(__ldg(p.x + c));
-            }
-            const uint32_t m = run_bits(q);
-            if (lane == 0)
-                scan[q] = __popc(m);
-        }
-        __syncthreads();
-        int total = 0;
-        for (int c = 0; c * 32 < runs; ++c) {
-            int ct;
-            const int excl = chunk_prefix(scan, runs, c, total, &ct);
-            // this warp's runs in the chunk (q is warp-uniform)
-            for (int q = c * 32 + ((warp - c * 32) % (NT / 32) + NT / 32) % (NT / 32);
-                 q < runs && q < c * 32 + 32; q += NT / 32) {
-                const int base = __shfl_sync(0xffffffffu, excl, q - c * 32);
-                const uint32_t m = run_bits(q);
-                if ((m >> lane) & 1u) {
-                    const int pos = base + __popc(m & ((1u << lane) - 1u));
-                    ridx[pos] = c0 + q * 32 + lane;
-                    if (FILL_X)
-                        rx[pos] = xs[q * 32 + lane];
-                }
-            }
-            total += ct;
-        }
-        __syncthreads();
-        return total;
-    } else {
-        // Threshold this CTA's channel slice: each warp takes runs of 32
-        // channels, one per lane; a ballot gives each run's active channels,
-        // a count per run and a prefix over runs give the ascending positions.
-        int c0, c1;
-        channel_slice(kp, split, c0, c1);
-        const int lane = tid & 31, warp = tid >> 5;
-        const int runs = (c1 - c0 + 31) / 32;
-        uint32_t mask[4];
-        float xv[4];
-        // Runs of this warp: warp, warp + NT/32, ... (the launcher keeps
-        // runs <= 4 * NT / 32).
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int q = warp + u * (NT / 32);
-            const int c = c0 + q * 32 + lane;
-            float v = 0.f;
-            bool act = false;
-            if (q < runs && c < c1) {
-                if (SRC == ROWS_GLU) {
-                    // x = h = bf16(act(gate) * up) from the consumed fp32 sums
-                    // (written by the previous kernel's reductions: read from L2)
-                    const float gt = ld_cg_f32(p.gu + c), up = ld_cg_f32(p.gu + p.K + c);
-                    const float hv = (p.glu_act == SGQ_ACT_SILU) ? act_mul<SGQ_ACT_SILU>(gt, up)
-                                                                 : act_mul<SGQ_ACT_RELU>(gt, up);
-                    const uint16_t hb = float_to_bf16_bits(hv);
-                    if (write_h && p.h_out)
-                        p.h_out[c] = hb;
-                    v = bf16_bits_to_float(hb);
-                } else {
-                    v = bf16_bits_to_float(__ldg(p.x + c));
-                }
-                act = fabsf(v) > p.t;
-            }
-            mask[u] = __ballot_sync(0xffffffffu, act);
-            xv[u] = v;
-            if (lane == 0 && q < runs)
-                scan[q] = __popc(mask[u]);
-        }
-        __syncthreads();
-        // runs <= 4 * NT / 32 <= 32 (the launcher keeps it so): one chunk
-        int total;
-        const int excl = chunk_prefix(scan, runs, 0, 0, &total);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int q = warp + u * (NT / 32); // warp-uniform
-            if (q < runs) {
-                const int base = __shfl_sync(0xffffffffu, excl, q);
-                if ((mask[u] >> lane) & 1u) {
-                    const int pos = base + __popc(mask[u] & ((1u << lane) - 1u));
-                    ridx[pos] = c0 + q * 32 + lane;
-                    rx[pos] = xv[u];
-                }
-            }
-        }
-        __syncthreads();
-        return total;
-    }
-}
 
 // Split-K epilogue, a second (tiny) kernel launched right behind the GEMV with
 // programmatic dependent launch: it waits until the GEMV grid has completed
@@ -825,33 +631,6 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_kernel(const KParams kp)
 // Host-side configuration
 // ---------------------------------------------------------------------------
 
-constexpr size_t kMaxSmem = 227 * 1024;
-
-int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
-
-template <typename Kern, typename Arg>
-cudaError_t launch_pdl(Kern kern, int grid, int block, size_t smem, cudaStream_t stream,
-                       const Arg &arg)
-{
-    if (smem > 48 * 1024) {
-        cudaError_t err = cudaFuncSetAttribute(
-            kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (err != cudaSuccess)
-            return err;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3((unsigned)block);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, arg);
-}
-
 // The GEMV grid, then the split-K epilogue grid behind it.
 template <typename Kern>
 cudaError_t launch_gemv_and_finalize(Kern kern, int grid, int block, size_t smem,
@@ -860,16 +639,7 @@ cudaError_t launch_gemv_and_finalize(Kern kern, int grid, int block, size_t smem
     cudaError_t err = launch_pdl(kern, grid, block, smem, stream, kp);
     if (err != cudaSuccess || kp.p.accumulate)
         return err;
-    const int quads = std::max(kp.p.B * (kp.p.N / 4), kp.p.zero_extra_n / 4);
-    const int fgrid = std::max(1, std::min(ceil_div(quads, 256), 148));
-    switch (kp.p.epilogue) {
-    case EPI_GLU_SILU:
-        return launch_pdl(finalize_kernel<EPI_GLU_SILU>, fgrid, 256, 0, stream, kp.p);
-    case EPI_GLU_RELU:
-        return launch_pdl(finalize_kernel<EPI_GLU_RELU>, fgrid, 256, 0, stream, kp.p);
-    default:
-        return launch_pdl(finalize_kernel<EPI_PLAIN>, fgrid, 256, 0, stream, kp.p);
-    }
+    return launch_finalize(kp.p, stream);
 }
 
 // Batch groups of warps for B > 1: ceil(B / 2) rounded up to 1, 2, 4 or 8.
@@ -922,6 +692,17 @@ cudaError_t launch_src(KParams kp, int num_sms, cudaStream_t stream)
 
 } // namespace
 
+cudaError_t launch_finalize(const GemvProblem &p, cudaStream_t stream)
+{
+    const int quads = std::max(p.B * (p.N / 4), p.zero_extra_n / 4);
+    const int fgrid = std::max(1, std::min(ceil_div(quads, 256), 148));
+    switch (p.epilogue) {
+    case EPI_GLU_SILU: return launch_pdl(finalize_kernel<EPI_GLU_SILU>, fgrid, 256, 0, stream, p);
+    case EPI_GLU_RELU: return launch_pdl(finalize_kernel<EPI_GLU_RELU>, fgrid, 256, 0, stream, p);
+    default: return launch_pdl(finalize_kernel<EPI_PLAIN>, fgrid, 256, 0, stream, p);
+    }
+}
+
 size_t gemv_workspace_bytes(int N, int B)
 {
     const size_t acc = (size_t)B * N * sizeof(float);
@@ -933,6 +714,12 @@ cudaError_t launch_gemv(const GemvProblem &p, int num_sms, cudaStream_t stream)
     KParams kp{};
     kp.p = p;
     kp.lg = __builtin_ctz((unsigned)p.group);
+    // B > 8 over the plain layout: the tensor-core kernel. Up to 8 rows the
+    // CUDA-core kernel (two batch rows per warp, one FMA per code and row)
+    // measured as fast; above, its warps each carry every row of the CTA.
+    if (p.B > 8 && !p.keep &&
+        (p.source == ROWS_LIST || p.source == ROWS_DENSE || p.source == ROWS_MASK))
+        return launch_gemv_mma(p, num_sms, stream);
     switch (p.source) {
     case ROWS_LIST: return launch_src<ROWS_LIST>(kp, num_sms, stream);
     case ROWS_DENSE: return launch_src<ROWS_DENSE>(kp, num_sms, stream);

@@ -1,0 +1,736 @@
+// gemv_mma.cu -- the activation-sparse GEMV for batch 2..16, on the tensor cores.
+//
+//   y[b][n] = sum_{k in U} s[g(k)][n] * (q[k][n] - z[g(k)][n]) * x[b][k]
+//
+// U is the one active set of the batch (the union of the rows' active
+// channels, or the caller's index list or bitmask). Method: "Enabling Dynamic
+// Sparsity in Quantized LLM Inference", Abstract: a GEMV over the quantized
+// layout that reads only the weight runs of the active channels.
+//
+// With B batch rows every weight code is used B times. The CUDA-core kernel
+// (one FMA per code and batch row) is bound by FMA issue well before HBM once
+// B >= 2, so here each code is expanded once into an exact fp16 operand and
+// the products go to the tensor cores (tcgen05.mma kind::f16, fp32
+// accumulators in tensor memory):
+//  * Tiles of 1024 outputs (512 bytes of a packed row) and k_splits shares of
+//    the rows per tile, as in the batch-1 kernel, with the same row lists.
+//  * The CTA's rows are cut into runs of one quantization group, and each run
+//    into K-blocks of 16 rows (the MMA's K; a run's last block is padded with
+//    zero rows).
+//  * 8 warps; warp w expands slots 2w and 2w + 1 of every K-block. Its lanes
+//    stream their own 16-byte columns of those rows through per-lane cp.async
+//    rings (8 rows ahead) and turn each code, minus the group's zero, into the
+//    exact fp16 value (q - z) 2^-24 (2^-20 for the high nibble of a byte): one
+//    AND and one packed fp16 subtraction per two codes, the zero being held in
+//    the same subnormal form. A K-block's A operand (1024 outputs x 16 rows,
+//    M-major, 128-byte swizzle) and B operand (16 rows x 16 batch columns of
+//    x' = x 2^S_b in fp16, K-major) go to one of two stages.
+//  * One thread issues the K-block's 8 MMAs (M = 128 outputs, N = 16, K = 16)
+//    into the run's accumulators (two alternating sets of 8 x 16 columns of
+//    tensor memory), then commits them to the stage's "empty" barrier and, at
+//    a run's end, to the set's "ready" barrier.
+//  * A run later every thread reads its outputs' sums from tensor memory and
+//    folds them with the group's scale: acc += s 2^c D. The products are those
+//    of the batch-1 kernel (exact fp16 x fp16), summed in fp32.
+//  * Split-K partials go into the fp32 workspace with float reductions; the
+//    shared epilogue kernel turns the workspace into bf16 y.
+//
+// Every wait on a barrier is bounded; a wait that runs out sets
+// SGQ_STATUS_TIMEOUT and the kernel carries on to its end (y is then not
+// valid), freeing its tensor memory. The kernel takes more than half of an
+// SM's shared memory, so at most one of its CTAs is resident per SM and the
+// allocation of 256 tensor-memory columns never waits.
+#include "gemv_rows.cuh"
+#include "sgq_device.cuh"
+#include "sgq_launch.h"
+
+#include <algorithm>
+
+namespace sgq {
+
+namespace {
+
+constexpr int kMWarps = 8;                  // warps that expand rows and fold
+constexpr int kIssuer = kMWarps;            // one more warp issues the MMAs
+constexpr int kAllWarps = kMWarps + 1;
+constexpr int kMThreads = kAllWarps * 32;
+constexpr int kKb = 16;                     // rows per K-block (the fp16 MMA's K)
+constexpr int kMmaN = 16;                   // MMA N: batch columns, padded to 16
+constexpr int kMBlocks = kTileN1 / 128;     // MMA M-blocks per tile
+constexpr int kAStage = kKb * kTileN1 * 2;  // A operand of one K-block: 32 KB
+constexpr int kBStage = kKb * kMmaN * 2;    // B operand of one K-block: 512 B
+constexpr int kMaxStages = 4;               // operand stages (2..4, by shared memory)
+constexpr int kMRing = 8;                   // rows in flight per warp
+constexpr int kTmemCols = 256;              // two sets of kMBlocks x kMmaN columns
+constexpr int kMSpin = 1 << 22;             // polls of a barrier before giving up
+constexpr size_t kOneCtaSmem = 116 * 1024;  // more than half of the SM's shared memory
+
+static_assert(2 * kMBlocks * kMmaN <= kTmemCols, "two accumulator sets");
+
+// Instruction descriptor of tcgen05.mma kind::f16: fp32 D, fp16 A and B,
+// A M-major, B K-major, N = 16, M = 128.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 15) | ((uint32_t)(kMmaN >> 3) << 17) |
+                            ((uint32_t)(128 >> 4) << 24);
+
+// Shared-memory matrix descriptor (sm_100 form): start, leading and stride
+// byte offsets in 16-byte units, version 1, layout type (0 none, 2 128B swizzle).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo,
+                                              uint32_t layout)
+{
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46) |
+           ((uint64_t)(layout & 7u) << 61);
+}
+
+// Byte offset, inside a K-block's A stage, of the 16-byte chunk that lane l
+// writes for word j of its 16-byte column of slot k. The stage is 16 atoms
+// (64 outputs x 8 rows, 1 KB, 128-byte swizzle) along M times 2 along K. Lane
+// l = 8g + h puts word j into atom g + 4j, logical chunk h, so that the 8
+// lanes of each group g cover all 32 banks in every store.
+__device__ __forceinline__ uint32_t a_chunk_off(int lane, int j, int k)
+{
+    const int g = lane >> 3, h = lane & 7, r = k & 7;
+    return (uint32_t)((k >> 3) * (16 * 1024) + (g + 4 * j) * 1024 + r * 128 + ((h ^ r) << 4));
+}
+
+// Output (0..1023, within the tile) held by M slot m of the A operand: the
+// inverse of the placement above. Chunk element e of word j carries output
+// 8j + (e >> 1) + 4 (e & 1): an AND takes codes 8j + i and 8j + i + 4 into
+// the two halves of a register.
+__host__ __device__ constexpr int mma_out_of_slot(int m)
+{
+    return 32 * (8 * ((m >> 6) & 3) + ((m >> 3) & 7)) + 8 * (m >> 8) + ((m & 7) >> 1) +
+           4 * (m & 1);
+}
+
+// Byte offset of element (batch column c, slot k) in a K-block's B stage:
+// K-major, no swizzle, core matrices of 8 columns x 8 slots (16-byte rows),
+// 128 bytes apart along K and 256 along N.
+__device__ __forceinline__ uint32_t b_elem_off(int c, int k)
+{
+    return (uint32_t)((k & 7) * 2 + (c & 7) * 16 + (k >> 3) * 128 + (c >> 3) * 256);
+}
+
+struct SmemM {
+    size_t a, b, ring, rxh, ridx, rstart, rkb, scan, total;
+};
+
+__host__ __device__ inline size_t align16(size_t v) { return (v + 15) / 16 * 16; }
+
+// a: `stages` A stages (1024-aligned); b: B stages; ring: each expanding
+// warp's per-lane rings; rxh: x' of each row, [row][bp batch columns] fp16;
+// ridx: the CTA's rows; rstart / rkb: first row / first K-block of each run
+// (+1 entry); scan: per-32-row counts.
+__host__ __device__ inline SmemM smemm_layout(int rows_cap, int stages, int bp)
+{
+    SmemM s;
+    s.a = 0;
+    s.b = s.a + (size_t)stages * kAStage;
+    s.ring = s.b + (size_t)stages * kBStage;
+    s.rxh = s.ring + (size_t)kMWarps * kMRing * kRowBytes1;
+    s.ridx = align16(s.rxh + (size_t)rows_cap * bp * 2);
+    s.rstart = align16(s.ridx + (size_t)rows_cap * 4);
+    s.rkb = align16(s.rstart + (size_t)(rows_cap + 1) * 4);
+    s.scan = align16(s.rkb + (size_t)(rows_cap + 1) * 4);
+    s.total = align16(s.scan + (size_t)((rows_cap + 31) / 32 + 4) * 4);
+    return s;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Waits for the phase of the given parity to complete, at most kMSpin polls.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok = 0;
+    for (int it = 0; it < kMSpin && !ok; ++it)
+        asm volatile("{\n\t.reg .pred p;\n\t"
+                     "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                     "selp.u32 %0, 1, 0, p;\n\t}"
+                     : "=r"(ok)
+                     : "r"(smem_u32(bar)), "r"(parity)
+                     : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                        bool accumulate)
+{
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+                 "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"((uint32_t)accumulate)
+                 : "memory");
+}
+
+// The completion of every MMA this thread issued so far arrives once on bar.
+__device__ __forceinline__ void mma_commit(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+// 16 consecutive fp32 columns of this thread's tensor-memory lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t addr, float *d)
+{
+    uint32_t r[16];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,"
+                 "%12,%13,%14,%15}, [%16];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
+                   "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+                 : "r"(addr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int c = 0; c < 16; ++c)
+        d[c] = __uint_as_float(r[c]);
+}
+
+__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d)
+{
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+                 "r"(d)
+                 : "memory");
+}
+
+// Integer zero point (0..15) of an (s, z) fp16 pair.
+__device__ __forceinline__ uint32_t zero_of(uint32_t w)
+{
+    return (uint32_t)__float2int_rn(__half2float(__ushort_as_half((uint16_t)(w >> 16))));
+}
+
+template <int SRC>
+__global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp)
+{
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t bar_full[kMaxStages], bar_empty[kMaxStages];
+    __shared__ __align__(8) uint64_t bar_ready[2], bar_free[2];
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_nruns, s_nkb;
+    __shared__ unsigned s_xmax[kMmaN];
+    __shared__ int s_S[kMmaN];
+
+    const GemvProblem &p = kp.p;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nst = kp.stages, bp = kp.bp;
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const SmemM L = smemm_layout(kp.rows_cap, nst, bp);
+    uint8_t *ring = smem + L.ring;
+    uint16_t *rxh = reinterpret_cast<uint16_t *>(smem + L.rxh);
+    int32_t *ridx = reinterpret_cast<int32_t *>(smem + L.ridx);
+    int *rstart = reinterpret_cast<int *>(smem + L.rstart);
+    int *rkb = reinterpret_cast<int *>(smem + L.rkb);
+    int *scan = reinterpret_cast<int *>(smem + L.scan);
+    const uint32_t sA = smem_u32(smem + L.a), sB = smem_u32(smem + L.b);
+
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(&s_tmem)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (tid == 0) {
+        for (int s = 0; s < nst; ++s) {
+            mbar_init(bar_full + s, kMWarps);
+            mbar_init(bar_empty + s, 1);
+        }
+        for (int d = 0; d < 2; ++d) {
+            mbar_init(bar_ready + d, 1);
+            mbar_init(bar_free + d, kMWarps);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (tid < kMmaN)
+        s_xmax[tid] = 0u;
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+
+    grid_launch_dependents();
+    const int tile = blockIdx.x % kp.n_tiles;
+    const int split = blockIdx.x / kp.n_tiles;
+    const int n0 = tile * kTileN1;
+    const int lg = kp.lg;
+    const int nvalid_out = min(kTileN1, p.N - n0); // outputs of this tile
+    const bool lane_ok = 32 * lane < nvalid_out;
+    bool ok = true;
+
+    grid_dependency_wait(); // x, idx, count, mask may come from the previous kernel
+
+    // The CTA's rows (invalid list entries are -1: read as row 0 with x = 0).
+    const int nr = build_rows<SRC, kMThreads, false>(kp, split, ridx, nullptr, scan);
+    auto grp = [&](int j) { return max(ridx[j], 0) >> lg; };
+
+    // Runs of one group: starts by ballots over chunks of 32 rows, positions
+    // by a prefix over the chunks' counts.
+    const int chunks = (nr + 31) / 32;
+    for (int q = warp; q < chunks; q += kAllWarps) {
+        const int j = q * 32 + lane;
+        const bool st = (j < nr) && (j == 0 || grp(j) != grp(j - 1));
+        const uint32_t m = __ballot_sync(0xffffffffu, st);
+        if (lane == 0)
+            scan[q] = __popc(m);
+    }
+    __syncthreads();
+    {
+        int total = 0;
+        for (int c = 0; c * 32 < chunks; ++c) {
+            int ct;
+            const int excl = chunk_prefix(scan, chunks, c, total, &ct);
+            for (int q = c * 32 + ((warp - c * 32) % kAllWarps + kAllWarps) % kAllWarps;
+                 q < chunks && q < c * 32 + 32; q += kAllWarps) {
+                const int base = __shfl_sync(0xffffffffu, excl, q - c * 32);
+                const int j = q * 32 + lane;
+                const bool st = (j < nr) && (j == 0 || grp(j) != grp(j - 1));
+                const uint32_t m = __ballot_sync(0xffffffffu, st);
+                if (st)
+                    rstart[base + __popc(m & ((1u << lane) - 1u))] = j;
+            }
+            total += ct;
+        }
+        if (tid == 0) {
+            s_nruns = total;
+            rstart[total] = nr;
+        }
+    }
+    __syncthreads();
+    const int nruns = s_nruns;
+    // First K-block of each run: a prefix over the runs' K-block counts.
+    if (warp == 0) {
+        int carry = 0;
+        for (int c = 0; c * 32 < nruns; ++c) {
+            const int r = c * 32 + lane;
+            const int v = (r < nruns) ? (rstart[r + 1] - rstart[r] + kKb - 1) / kKb : 0;
+            int incl = v;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, incl, d);
+                if (lane >= d)
+                    incl += t;
+            }
+            if (r < nruns)
+                rkb[r] = carry + incl - v;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) {
+            rkb[nruns] = carry;
+            s_nkb = carry;
+        }
+    }
+    __syncthreads();
+    const int nkb = s_nkb;
+
+    // K-block kb: its run (a pointer advanced monotonically), the ridx
+    // position of its slot 0 and its valid slots.
+    auto kb_run = [&](int kb, int &run) {
+        while (kb >= rkb[run + 1])
+            ++run;
+    };
+
+    if (warp == kIssuer) {
+        // ---- the MMA issuer --------------------------------------------------
+        if (lane == 0) {
+            int run = 0;
+            for (int kb = 0; kb < nkb; ++kb) {
+                kb_run(kb, run);
+                const bool first = kb == rkb[run], last = kb == rkb[run + 1] - 1;
+                const int s = kb % nst;
+                if (!mbar_wait(bar_full + s, (uint32_t)((kb / nst) & 1)))
+                    ok = false;
+                tc_fence_after();
+                if (first && run >= 2) {
+                    if (!mbar_wait(bar_free + (run & 1), (uint32_t)(((run >> 1) - 1) & 1)))
+                        ok = false;
+                    tc_fence_after();
+                }
+                const uint32_t a_st = sA + (uint32_t)(s * kAStage);
+                const uint32_t dcol = tmem + (uint32_t)(128 * (run & 1));
+                const uint64_t bdesc = smem_desc(sB + (uint32_t)(s * kBStage), 128, 256, 0);
+                // Every M-block: a lane's outputs are spread over the M-blocks
+                // (lanes past N hold finite codes of column 0 and are dropped
+                // in the epilogue).
+#pragma unroll
+                for (int mb = 0; mb < kMBlocks; ++mb)
+                    mma_f16(dcol + (uint32_t)(kMmaN * mb),
+                            smem_desc(a_st + (uint32_t)(mb * 2048), 1024, 16 * 1024, 2), bdesc,
+                            !first);
+                mma_commit(bar_empty + s);
+                if (last)
+                    mma_commit(bar_ready + (run & 1));
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---- the expanding warps ---------------------------------------------
+        // This warp's rows: slots 2w, 2w + 1 of every K-block, in order;
+        // sequence position i = 2 kb + u. The ring runs kMRing positions ahead
+        // with its own run pointer.
+        const size_t row_bytes = (size_t)(p.N / 2);
+        const uint8_t *wcol = p.qweight + (lane_ok ? ((size_t)n0 / 2 + lane * 16) : 0);
+        uint8_t *myring = ring + (size_t)warp * kMRing * kRowBytes1 + lane * 16;
+        const int nseq = 2 * nkb;
+        int ring_run = 0;
+        auto seq_row = [&](int i) -> int { // ridx position, or -1 for a padding slot
+            const int kb = i >> 1;
+            kb_run(kb, ring_run);
+            const int slot = 2 * warp + (i & 1);
+            const int j = rstart[ring_run] + kKb * (kb - rkb[ring_run]) + slot;
+            return (j < rstart[ring_run + 1]) ? j : -1;
+        };
+#pragma unroll
+        for (int i = 0; i < kMRing; ++i) {
+            if (i < nseq) {
+                const int j = seq_row(i);
+                if (j >= 0)
+                    cp_async16(myring + i * kRowBytes1,
+                               wcol + (size_t)max(ridx[j], 0) * row_bytes);
+            }
+            cp_async_commit();
+        }
+
+        // Zero points of this lane's 32 outputs for one group, as subnormal
+        // fp16 pairs matching the AND results: word j, pairs = outputs
+        // (8j, 8j+4), (8j+1, 8j+5) << 4, (8j+2, 8j+6), (8j+3, 8j+7) << 4.
+        uint4 zraw[8];
+        auto load_sz = [&](int G) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.sz + (size_t)G * p.N + n0 +
+                                                               (lane_ok ? lane * 32 : 0));
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                zraw[c] = __ldg(src + c);
+        };
+        uint32_t zc[4][4];
+        auto unpack_z = [&]() {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t w[8] = {zraw[2 * j].x,     zraw[2 * j].y,     zraw[2 * j].z,
+                                       zraw[2 * j].w,     zraw[2 * j + 1].x, zraw[2 * j + 1].y,
+                                       zraw[2 * j + 1].z, zraw[2 * j + 1].w};
+                uint32_t z[8];
+#pragma unroll
+                for (int o = 0; o < 8; ++o)
+                    z[o] = lane_ok ? zero_of(w[o]) : 0u;
+                zc[j][0] = z[0] | (z[4] << 16);
+                zc[j][1] = (z[1] | (z[5] << 16)) << 4;
+                zc[j][2] = z[2] | (z[6] << 16);
+                zc[j][3] = (z[3] | (z[7] << 16)) << 4;
+            }
+        };
+        // Scales of this thread's 4 fold outputs (one per M-block of its half).
+        const int mb0 = 4 * (warp >> 2);
+        int fout[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            fout[i] = mma_out_of_slot(128 * (mb0 + i) + 32 * (warp & 3) + lane);
+        float sfold[4], snew[4];
+        auto load_s = [&](int G, float *sv) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                sv[i] = (fout[i] < nvalid_out)
+                            ? __half2float(__ushort_as_half((uint16_t)(
+                                  __ldg(p.sz + (size_t)G * p.N + n0 + fout[i]) & 0xffffu)))
+                            : 0.f;
+        };
+        if (nruns > 0) {
+            load_sz(grp(rstart[0]));
+            load_s(grp(rstart[0]), snew);
+        }
+
+        // x' = x 2^S_b in fp16 per batch row b, 2^14 <= max |x'| < 2^15 over
+        // the CTA's rows (as in the batch-1 kernel), staged as rxh[row][bp].
+        // Pass 1 gathers x of the rows (bf16 bits), 8 rows per item: one
+        // 16-byte load when the 8 rows are 8 consecutive aligned channels; it
+        // takes max |x| per b. Pass 2 converts in place, a row per item.
+        {
+            const int nch = (nr + 7) / 8;
+            const int items = p.B * nch;
+            int bcur = -1;
+            float m = 0.f;
+            for (int e0 = tid; e0 < items; e0 += 4 * kMWarps * 32) {
+                uint4 v[4];
+                int bi[4], ji[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int e = e0 + u * kMWarps * 32;
+                    bi[u] = -1;
+                    ji[u] = 0;
+                    v[u] = make_uint4(0u, 0u, 0u, 0u);
+                    if (e < items) {
+                        const int b = e / nch, j0 = (e - b * nch) * 8;
+                        bi[u] = b;
+                        ji[u] = j0;
+                        const uint16_t *xb = p.x + (size_t)b * p.K;
+                        const int k0 = ridx[j0];
+                        bool vec = (j0 + 8 <= nr) && k0 >= 0 && (k0 & 7) == 0;
+#pragma unroll
+                        for (int i = 1; i < 8; ++i)
+                            vec = vec && (ridx[min(j0 + i, nr - 1)] == k0 + i);
+                        if (vec) {
+                            v[u] = __ldg(reinterpret_cast<const uint4 *>(xb + k0));
+                        } else {
+                            uint32_t h[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const int k = (j0 + i < nr) ? ridx[j0 + i] : -1;
+                                h[i] = (k >= 0) ? (uint32_t)__ldg(xb + k) : 0u;
+                            }
+                            v[u] = make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16),
+                                              h[4] | (h[5] << 16), h[6] | (h[7] << 16));
+                        }
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    if (bi[u] < 0)
+                        continue;
+                    if (bi[u] != bcur) {
+                        if (bcur >= 0)
+                            atomicMax(s_xmax + bcur, __float_as_uint(m));
+                        bcur = bi[u];
+                        m = 0.f;
+                    }
+                    const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const uint16_t hb = (uint16_t)(w[i >> 1] >> (16 * (i & 1)));
+                        if (ji[u] + i < nr) {
+                            rxh[(ji[u] + i) * bp + bi[u]] = hb;
+                            m = fmaxf(m, fabsf(bf16_bits_to_float(hb)));
+                        }
+                    }
+                }
+            }
+            if (bcur >= 0)
+                atomicMax(s_xmax + bcur, __float_as_uint(m));
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kMWarps * 32) : "memory");
+        if (tid < kMmaN) {
+            const float mx = __uint_as_float(s_xmax[tid]);
+            s_S[tid] = (mx > 0.f && !isinf(mx)) ? 14 - ilogbf(mx) : 0;
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kMWarps * 32) : "memory");
+        for (int j = tid; j < nr; j += kMWarps * 32) {
+            uint16_t *row = rxh + (size_t)j * bp;
+            for (int b = 0; b < p.B; ++b) {
+                const int S = s_S[b];
+                row[b] = __half_as_ushort(__float2half_rn(
+                    (bf16_bits_to_float(row[b]) * pow2f(S - S / 2)) * pow2f(S / 2)));
+            }
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kMWarps * 32) : "memory");
+
+        float acc[4][kMmaN];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int c = 0; c < kMmaN; ++c)
+                acc[i][c] = 0.f;
+
+        // acc += s 2^c D for run r's accumulators (set r & 1).
+        auto fold = [&](int r) {
+            if (!mbar_wait(bar_ready + (r & 1), (uint32_t)((r >> 1) & 1)))
+                ok = false;
+            tc_fence_after();
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float d[kMmaN];
+                tmem_ld16(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + 128 * (r & 1) +
+                              kMmaN * (mb0 + i),
+                          d);
+                const float f = sfold[i] * ((fout[i] & 1) ? 1048576.f : 16777216.f);
+#pragma unroll
+                for (int c = 0; c < kMmaN; ++c)
+                    acc[i][c] = fmaf(f, d[c], acc[i][c]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar_free + (r & 1));
+        };
+
+        int run = 0;
+        for (int kb = 0; kb < nkb; ++kb) {
+            kb_run(kb, run);
+            const int s = kb % nst;
+            const int j0 = rstart[run] + kKb * (kb - rkb[run]);
+            const int nv = min(kKb, rstart[run + 1] - j0);
+            const bool first = kb == rkb[run];
+            if (first) {
+                unpack_z(); // this run's zero points (loaded a run ahead)
+                if (run + 1 < nruns)
+                    load_sz(grp(rstart[run + 1]));
+            }
+            // The stage's previous K-block has been multiplied.
+            if (kb >= nst && !mbar_wait(bar_empty + s, (uint32_t)((kb / nst - 1) & 1)))
+                ok = false;
+            const uint32_t a_st = sA + (uint32_t)(s * kAStage);
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int i = 2 * kb + u;
+                const int slot = 2 * warp + u;
+                cp_async_wait<kMRing - 1>();
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                const bool valid = slot < nv;
+                if (valid)
+                    v = *reinterpret_cast<const uint4 *>(myring + (i % kMRing) * kRowBytes1);
+                // refill the ring slot with the row kMRing positions ahead
+                if (i + kMRing < nseq) {
+                    const int j = seq_row(i + kMRing);
+                    if (j >= 0)
+                        cp_async16(myring + (i % kMRing) * kRowBytes1,
+                                   wcol + (size_t)max(ridx[j], 0) * row_bytes);
+                }
+                cp_async_commit();
+                const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint32_t t0 = 0u, t1 = 0u, t2 = 0u, t3 = 0u;
+                    if (valid) {
+                        const uint32_t w = wv[j], w8 = w >> 8;
+                        t0 = hsub2(w & 0x000F000Fu, zc[j][0]);
+                        t1 = hsub2(w & 0x00F000F0u, zc[j][1]);
+                        t2 = hsub2(w8 & 0x000F000Fu, zc[j][2]);
+                        t3 = hsub2(w8 & 0x00F000F0u, zc[j][3]);
+                    }
+                    st_shared_v4(a_st + a_chunk_off(lane, j, slot), t0, t1, t2, t3);
+                }
+            }
+            {
+                // B operand: x' of slots 2w, 2w + 1 for the 16 batch columns.
+                const int u = lane >> 4, c = lane & 15, slot = 2 * warp + u;
+                const uint16_t xv =
+                    (slot < nv && c < p.B) ? rxh[(j0 + slot) * bp + c] : (uint16_t)0;
+                asm volatile("st.shared.u16 [%0], %1;" ::"r"(sB + (uint32_t)(s * kBStage) +
+                                                             b_elem_off(c, slot)),
+                             "h"(xv)
+                             : "memory");
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar_full + s);
+
+            // The previous run ended with the previous K-block: fold it now,
+            // while this K-block is being multiplied.
+            if (first && run > 0) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    sfold[i] = snew[i];
+                load_s(grp(rstart[run]), snew); // this run's scales, for its fold
+                fold(run - 1);
+            }
+        }
+        if (nruns > 0) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                sfold[i] = snew[i];
+            fold(nruns - 1);
+        }
+        cp_async_wait_all();
+
+        // Split-K partials, back in real units (x 2^-S_b, two exact factors).
+        if (nkb > 0) {
+#pragma unroll
+            for (int c = 0; c < kMmaN; ++c) {
+                if (c < p.B) {
+                    const int E = -s_S[c];
+                    const float f1 = pow2f(E / 2), f2 = pow2f(E - E / 2);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        if (fout[i] < nvalid_out)
+                            atomicAdd(p.ws_acc + (size_t)c * p.N + n0 + fout[i],
+                                      (acc[i][c] * f1) * f2);
+                }
+            }
+        }
+    }
+    if (!ok)
+        set_status(p.status, SGQ_STATUS_TIMEOUT);
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"(kTmemCols)
+                     : "memory");
+}
+
+// Batch columns of the staged x: B rounded up to 2, 4, 8 or 16.
+int pad_batch(int B)
+{
+    int b = 2;
+    while (b < B)
+        b *= 2;
+    return b;
+}
+
+template <int SRC>
+cudaError_t launch_mma_t(KParams kp, int num_sms, cudaStream_t stream)
+{
+    const GemvProblem &p = kp.p;
+    kp.nb = 1;
+    kp.bp = pad_batch(p.B);
+    kp.n_tiles = ceil_div(p.N, kTileN1);
+    kp.k_splits = std::max(1, num_sms / kp.n_tiles);
+    kp.span_cap = 0;
+    SmemM L;
+    for (;;) {
+        kp.rows_cap = ceil_div(p.K, kp.k_splits) + 8;
+        // the most operand stages that fit, at least two
+        kp.stages = kMaxStages;
+        L = smemm_layout(kp.rows_cap, kp.stages, kp.bp);
+        while (kp.stages > 2 && L.total + 1024 > kMaxSmem) {
+            --kp.stages;
+            L = smemm_layout(kp.rows_cap, kp.stages, kp.bp);
+        }
+        if (L.total + 1024 <= kMaxSmem || kp.k_splits >= p.K / 8)
+            break;
+        kp.k_splits *= 2;
+    }
+    if (L.total + 1024 > kMaxSmem)
+        return cudaErrorInvalidConfiguration;
+    const size_t smem = std::max(L.total + 1024, kOneCtaSmem);
+    cudaError_t err = launch_pdl(gemv_mma_kernel<SRC>, kp.n_tiles * kp.k_splits, kMThreads,
+                                 smem, stream, kp);
+    if (err != cudaSuccess || p.accumulate)
+        return err;
+    return launch_finalize(p, stream);
+}
+
+} // namespace
+
+cudaError_t launch_gemv_mma(const GemvProblem &p, int num_sms, cudaStream_t stream)
+{
+    KParams kp{};
+    kp.p = p;
+    kp.lg = __builtin_ctz((unsigned)p.group);
+    switch (p.source) {
+    case ROWS_LIST: return launch_mma_t<ROWS_LIST>(kp, num_sms, stream);
+    case ROWS_DENSE: return launch_mma_t<ROWS_DENSE>(kp, num_sms, stream);
+    case ROWS_MASK: return launch_mma_t<ROWS_MASK>(kp, num_sms, stream);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+} // namespace sgq

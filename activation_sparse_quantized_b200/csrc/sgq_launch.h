@@ -68,6 +68,10 @@ cudaError_t launch_select(const uint16_t *x, int B, int K, const Thresholds &th,
 cudaError_t launch_select_mask(const uint16_t *x, int B, int K, const Thresholds &th,
                                uint32_t *mask, int32_t *count, cudaStream_t stream);
 cudaError_t launch_gemv(const GemvProblem &p, int num_sms, cudaStream_t stream);
+// B > 1 over the plain layout (gemv_mma.cu), then the split-K epilogue.
+cudaError_t launch_gemv_mma(const GemvProblem &p, int num_sms, cudaStream_t stream);
+// The split-K epilogue kernel alone (PDL-chained behind a GEMV grid).
+cudaError_t launch_finalize(const GemvProblem &p, cudaStream_t stream);
 // Records e as the last CUDA error of this thread; returns SGQ_ERR_CUDA.
 int record_cuda_error(cudaError_t e);
 

@@ -24,6 +24,7 @@ SGQ_ACT_RELU = 1
 SGQ_STATUS_NONFINITE_W = 1
 SGQ_STATUS_BAD_INDEX = 2
 SGQ_STATUS_BAD_COUNT = 4
+SGQ_STATUS_TIMEOUT = 8
 SGQ_MAX_BATCH = 16
 SGQ_NOALLOC_MAX_N = 65536
 

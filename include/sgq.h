@@ -63,6 +63,7 @@ extern "C" {
 #define SGQ_STATUS_NONFINITE_W  1  /* sgq_pack: W holds NaN or Inf (that group packed as zeros) */
 #define SGQ_STATUS_BAD_INDEX    2  /* sgq_gemv: an index outside [0, K) was skipped             */
 #define SGQ_STATUS_BAD_COUNT    4  /* sgq_gemv: *count outside [0, K]; clamped                  */
+#define SGQ_STATUS_TIMEOUT      8  /* a bounded wait inside a GEMV kernel ran out: y is not valid */
 
 /* Activations for sgq_glu. */
 #define SGQ_ACT_SILU 0

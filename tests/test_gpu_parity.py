@@ -237,7 +237,7 @@ def test_gemv_dense_matches_oracle_and_full_list():
     assert g.workspace_is_zero()
 
 
-@pytest.mark.parametrize("B", [2, 8])
+@pytest.mark.parametrize("B", [2, 8, 12])
 def test_gemv_dense_batch(B):
     case = wl.gemv_case(N=1024, K=4096, group=128, B=B, sparsity=0.0, seed=70)
     g = GpuGemv(case.W, 128, B)
@@ -245,6 +245,30 @@ def test_gemv_dense_batch(B):
     q, s, z = oracle_codes(case.W, 128)
     y64, sa, _ = oracle.gemv_dense(q, s, z, 128, bits(case.x))
     check_y(y, y32, y64, sa, f"dense B={B}")
+
+
+@pytest.mark.parametrize("B,g", [(9, 32), (12, 128), (16, 64)])
+def test_gemv_batch_unsorted_list_with_repeats(B, g):
+    """A caller's index list in no order, with repeated channels, at batch
+    sizes of the tensor-core kernel: the list is cut into runs of one group
+    wherever the group changes, and a repeated channel counts once per entry,
+    as in the oracle's sum over the list. N = 2080 leaves a ragged tile."""
+    N, K = 2080, 4096
+    case = wl.gemv_case(N=N, K=K, group=g, B=B, sparsity=0.0, seed=90 + B)
+    rng = np.random.default_rng(B)
+    idx = rng.permutation(K)[: K // 2]
+    idx = np.concatenate([idx, idx[:200]]).astype(np.int32)
+    rng.shuffle(idx)
+    gg = GpuGemv(case.W, g, B)
+    idx_d = torch.tensor(idx, dtype=torch.int32, device=DEV)
+    cnt = torch.tensor([idx.size], dtype=torch.int32, device=DEV)
+    y, y32 = gg.gemv(case.x.to(DEV), idx_d, cnt)
+    q, s, z = oracle_codes(case.W, g)
+    y64, sa, _ = oracle.gemv(q, s, z, g, bits(case.x), idx)
+    torch.cuda.synchronize()
+    check_y(y, y32, y64, sa, f"unsorted list B={B} g={g}")
+    assert gg.workspace_is_zero()
+    assert gg.status.item() == 0
 
 
 @pytest.mark.parametrize("sparsity", [0.0, 0.5, 0.9])
