@@ -50,7 +50,7 @@ namespace sgq {
 
 namespace {
 
-constexpr int kMWarps = 8;                  // warps that expand rows and fold
+constexpr int kMWarps = 16;                 // warps that expand rows (one slot each) and fold
 constexpr int kIssuer = kMWarps;            // one more warp issues the MMAs
 constexpr int kAllWarps = kMWarps + 1;
 constexpr int kMThreads = kAllWarps * 32;
@@ -60,12 +60,13 @@ constexpr int kMBlocks = kTileN1 / 128;     // MMA M-blocks per tile
 constexpr int kAStage = kKb * kTileN1 * 2;  // A operand of one K-block: 32 KB
 constexpr int kBStage = kKb * kMmaN * 2;    // B operand of one K-block: 512 B
 constexpr int kMaxStages = 4;               // operand stages (2..4, by shared memory)
-constexpr int kMRing = 8;                   // rows in flight per warp
-constexpr int kTmemCols = 256;              // two sets of kMBlocks x kMmaN columns
+constexpr int kMRing = 4;                   // rows in flight per expanding warp
+constexpr int kTmemCols = 512;              // two accumulator sets and the running totals
+constexpr int kTotCol = 256;                // first column of the totals
 constexpr int kMSpin = 1 << 22;             // polls of a barrier before giving up
 constexpr size_t kOneCtaSmem = 116 * 1024;  // more than half of the SM's shared memory
 
-static_assert(2 * kMBlocks * kMmaN <= kTmemCols, "two accumulator sets");
+static_assert(kTotCol + kMBlocks * kMmaN <= kTmemCols, "accumulators and totals");
 
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 D, fp16 A and B,
 // A M-major, B K-major, N = 16, M = 128.
@@ -197,6 +198,20 @@ __device__ __forceinline__ void tmem_ld16(uint32_t addr, float *d)
         d[c] = __uint_as_float(r[c]);
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t addr, const float *v)
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,"
+                 "%11,%12,%13,%14,%15,%16};" ::"r"(addr),
+                 "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+                 "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+                 "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+                 "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
+                 "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])),
+                 "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+                 "r"(__float_as_uint(v[15]))
+                 : "memory");
+}
+
 __device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b)
 {
     uint32_t d;
@@ -226,7 +241,6 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
     __shared__ __align__(8) uint64_t bar_ready[2], bar_free[2];
     __shared__ uint32_t s_tmem;
     __shared__ int s_nruns, s_nkb;
-    __shared__ unsigned s_xmax[kMmaN];
     __shared__ int s_S[kMmaN];
 
     const GemvProblem &p = kp.p;
@@ -260,8 +274,6 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (tid < kMmaN)
-        s_xmax[tid] = 0u;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -383,31 +395,36 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
         __syncwarp();
     } else {
         // ---- the expanding warps ---------------------------------------------
-        // This warp's rows: slots 2w, 2w + 1 of every K-block, in order;
-        // sequence position i = 2 kb + u. The ring runs kMRing positions ahead
-        // with its own run pointer.
+        // Warp w expands slot w of every K-block: its row stream is one row
+        // per K-block, through a per-lane ring kMRing K-blocks ahead (with its
+        // own run pointer).
+        constexpr int kEx = kMWarps * 32; // threads of the expanding warps
         const size_t row_bytes = (size_t)(p.N / 2);
         const uint8_t *wcol = p.qweight + (lane_ok ? ((size_t)n0 / 2 + lane * 16) : 0);
         uint8_t *myring = ring + (size_t)warp * kMRing * kRowBytes1 + lane * 16;
-        const int nseq = 2 * nkb;
         int ring_run = 0;
-        auto seq_row = [&](int i) -> int { // ridx position, or -1 for a padding slot
-            const int kb = i >> 1;
+        auto kb_row = [&](int kb) -> int { // ridx position of this warp's slot, or -1
             kb_run(kb, ring_run);
-            const int slot = 2 * warp + (i & 1);
-            const int j = rstart[ring_run] + kKb * (kb - rkb[ring_run]) + slot;
+            const int j = rstart[ring_run] + kKb * (kb - rkb[ring_run]) + warp;
             return (j < rstart[ring_run + 1]) ? j : -1;
         };
 #pragma unroll
         for (int i = 0; i < kMRing; ++i) {
-            if (i < nseq) {
-                const int j = seq_row(i);
+            if (i < nkb) {
+                const int j = kb_row(i);
                 if (j >= 0)
                     cp_async16(myring + i * kRowBytes1,
                                wcol + (size_t)max(ridx[j], 0) * row_bytes);
             }
             cp_async_commit();
         }
+        // This lane's four A chunks of slot `warp` (stage-relative) and its B
+        // element (lanes 0..15: batch column = lane).
+        uint32_t aoff[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            aoff[j] = a_chunk_off(lane, j, warp);
+        const uint32_t boff = b_elem_off(lane & 15, warp);
 
         // Zero points of this lane's 32 outputs for one group, as subnormal
         // fp16 pairs matching the AND results: word j, pairs = outputs
@@ -437,20 +454,21 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
                 zc[j][3] = (z[3] | (z[7] << 16)) << 4;
             }
         };
-        // Scales of this thread's 4 fold outputs (one per M-block of its half).
-        const int mb0 = 4 * (warp >> 2);
-        int fout[4];
+        // Fold outputs of this thread: its tensor-memory lane (quadrant
+        // warp % 4) in M-blocks 2 (warp / 4) and 2 (warp / 4) + 1.
+        const int mbA = 2 * (warp >> 2);
+        const uint32_t tlane = (uint32_t)(32 * (warp & 3)) << 16;
+        int fout[2];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            fout[i] = mma_out_of_slot(128 * (mb0 + i) + 32 * (warp & 3) + lane);
-        float sfold[4], snew[4];
-        auto load_s = [&](int G, float *sv) {
+        for (int i = 0; i < 2; ++i)
+            fout[i] = mma_out_of_slot(128 * (mbA + i) + 32 * (warp & 3) + lane);
+        // (s, z) words of the fold outputs for a group, kept raw until the fold
+        // so that the loads stay in flight.
+        uint32_t sfold[2], snew[2];
+        auto load_s = [&](int G, uint32_t *sv) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                sv[i] = (fout[i] < nvalid_out)
-                            ? __half2float(__ushort_as_half((uint16_t)(
-                                  __ldg(p.sz + (size_t)G * p.N + n0 + fout[i]) & 0xffffu)))
-                            : 0.f;
+            for (int i = 0; i < 2; ++i)
+                sv[i] = (fout[i] < nvalid_out) ? __ldg(p.sz + (size_t)G * p.N + n0 + fout[i]) : 0u;
         };
         if (nruns > 0) {
             load_sz(grp(rstart[0]));
@@ -459,110 +477,76 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
 
         // x' = x 2^S_b in fp16 per batch row b, 2^14 <= max |x'| < 2^15 over
         // the CTA's rows (as in the batch-1 kernel), staged as rxh[row][bp].
-        // Pass 1 gathers x of the rows (bf16 bits), 8 rows per item: one
-        // 16-byte load when the 8 rows are 8 consecutive aligned channels; it
-        // takes max |x| per b. Pass 2 converts in place, a row per item.
-        {
-            const int nch = (nr + 7) / 8;
-            const int items = p.B * nch;
-            int bcur = -1;
+        // Warp w owns batch row b = w: its lanes gather x of the rows, 8 rows
+        // per item (one 16-byte load when the 8 rows are 8 consecutive aligned
+        // channels), the warp reduces max |x|, then converts its column.
+        if (warp < p.B) {
+            const int b = warp;
+            const uint16_t *xb = p.x + (size_t)b * p.K;
             float m = 0.f;
-            for (int e0 = tid; e0 < items; e0 += 4 * kMWarps * 32) {
-                uint4 v[4];
-                int bi[4], ji[4];
+            for (int j0 = 8 * lane; j0 < nr; j0 += 8 * 32) {
+                const int k0 = ridx[j0];
+                bool vec = (j0 + 8 <= nr) && k0 >= 0 && (k0 & 7) == 0;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int e = e0 + u * kMWarps * 32;
-                    bi[u] = -1;
-                    ji[u] = 0;
-                    v[u] = make_uint4(0u, 0u, 0u, 0u);
-                    if (e < items) {
-                        const int b = e / nch, j0 = (e - b * nch) * 8;
-                        bi[u] = b;
-                        ji[u] = j0;
-                        const uint16_t *xb = p.x + (size_t)b * p.K;
-                        const int k0 = ridx[j0];
-                        bool vec = (j0 + 8 <= nr) && k0 >= 0 && (k0 & 7) == 0;
+                for (int i = 1; i < 8; ++i)
+                    vec = vec && (ridx[min(j0 + i, nr - 1)] == k0 + i);
+                uint32_t h[8];
+                if (vec) {
+                    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(xb + k0));
+                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                        for (int i = 1; i < 8; ++i)
-                            vec = vec && (ridx[min(j0 + i, nr - 1)] == k0 + i);
-                        if (vec) {
-                            v[u] = __ldg(reinterpret_cast<const uint4 *>(xb + k0));
-                        } else {
-                            uint32_t h[8];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                const int k = (j0 + i < nr) ? ridx[j0 + i] : -1;
-                                h[i] = (k >= 0) ? (uint32_t)__ldg(xb + k) : 0u;
-                            }
-                            v[u] = make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16),
-                                              h[4] | (h[5] << 16), h[6] | (h[7] << 16));
-                        }
-                    }
-                }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    if (bi[u] < 0)
-                        continue;
-                    if (bi[u] != bcur) {
-                        if (bcur >= 0)
-                            atomicMax(s_xmax + bcur, __float_as_uint(m));
-                        bcur = bi[u];
-                        m = 0.f;
-                    }
-                    const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+                    for (int i = 0; i < 8; ++i)
+                        h[i] = (w[i >> 1] >> (16 * (i & 1))) & 0xffffu;
+                } else {
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        const uint16_t hb = (uint16_t)(w[i >> 1] >> (16 * (i & 1)));
-                        if (ji[u] + i < nr) {
-                            rxh[(ji[u] + i) * bp + bi[u]] = hb;
-                            m = fmaxf(m, fabsf(bf16_bits_to_float(hb)));
-                        }
+                        const int k = (j0 + i < nr) ? ridx[j0 + i] : -1;
+                        h[i] = (k >= 0) ? (uint32_t)__ldg(xb + k) : 0u;
                     }
                 }
-            }
-            if (bcur >= 0)
-                atomicMax(s_xmax + bcur, __float_as_uint(m));
-        }
-        asm volatile("bar.sync 1, %0;" ::"n"(kMWarps * 32) : "memory");
-        if (tid < kMmaN) {
-            const float mx = __uint_as_float(s_xmax[tid]);
-            s_S[tid] = (mx > 0.f && !isinf(mx)) ? 14 - ilogbf(mx) : 0;
-        }
-        asm volatile("bar.sync 1, %0;" ::"n"(kMWarps * 32) : "memory");
-        for (int j = tid; j < nr; j += kMWarps * 32) {
-            uint16_t *row = rxh + (size_t)j * bp;
-            for (int b = 0; b < p.B; ++b) {
-                const int S = s_S[b];
-                row[b] = __half_as_ushort(__float2half_rn(
-                    (bf16_bits_to_float(row[b]) * pow2f(S - S / 2)) * pow2f(S / 2)));
-            }
-        }
-        asm volatile("bar.sync 1, %0;" ::"n"(kMWarps * 32) : "memory");
-
-        float acc[4][kMmaN];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int c = 0; c < kMmaN; ++c)
-                acc[i][c] = 0.f;
+                for (int i = 0; i < 8; ++i)
+                    if (j0 + i < nr) {
+                        rxh[(j0 + i) * bp + b] = (uint16_t)h[i];
+                        m = fmaxf(m, fabsf(bf16_bits_to_float((uint16_t)h[i])));
+                    }
+            }
+            const int e = warp_max_exponent(m);
+            const int S = (e == INT32_MIN) ? 0 : 14 - e;
+            if (lane == 0)
+                s_S[b] = S;
+            const float fa = pow2f(S - S / 2), fb = pow2f(S / 2);
+            for (int j = lane; j < nr; j += 32)
+                rxh[j * bp + b] = __half_as_ushort(
+                    __float2half_rn((bf16_bits_to_float(rxh[j * bp + b]) * fa) * fb));
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kEx) : "memory");
 
-        // acc += s 2^c D for run r's accumulators (set r & 1).
+        // totals += s 2^c D for run r's accumulators (set r & 1); the totals
+        // stay in tensor memory (columns kTotCol..), written by run 0.
         auto fold = [&](int r) {
             if (!mbar_wait(bar_ready + (r & 1), (uint32_t)((r >> 1) & 1)))
                 ok = false;
             tc_fence_after();
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float d[kMmaN];
-                tmem_ld16(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + 128 * (r & 1) +
-                              kMmaN * (mb0 + i),
-                          d);
-                const float f = sfold[i] * ((fout[i] & 1) ? 1048576.f : 16777216.f);
+            for (int i = 0; i < 2; ++i) {
+                float d[kMmaN], t[kMmaN];
+                tmem_ld16(tmem + tlane + 128 * (r & 1) + kMmaN * (mbA + i), d);
+                const float f = __half2float(__ushort_as_half((uint16_t)(sfold[i] & 0xffffu))) *
+                                ((fout[i] & 1) ? 1048576.f : 16777216.f);
+                if (r == 0) {
 #pragma unroll
-                for (int c = 0; c < kMmaN; ++c)
-                    acc[i][c] = fmaf(f, d[c], acc[i][c]);
+                    for (int c = 0; c < kMmaN; ++c)
+                        t[c] = f * d[c];
+                } else {
+                    tmem_ld16(tmem + tlane + kTotCol + kMmaN * (mbA + i), t);
+#pragma unroll
+                    for (int c = 0; c < kMmaN; ++c)
+                        t[c] = fmaf(f, d[c], t[c]);
+                }
+                tmem_st16(tmem + tlane + kTotCol + kMmaN * (mbA + i), t);
             }
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -574,7 +558,7 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
             kb_run(kb, run);
             const int s = kb % nst;
             const int j0 = rstart[run] + kKb * (kb - rkb[run]);
-            const int nv = min(kKb, rstart[run + 1] - j0);
+            const bool valid = warp < rstart[run + 1] - j0;
             const bool first = kb == rkb[run];
             if (first) {
                 unpack_z(); // this run's zero points (loaded a run ahead)
@@ -585,44 +569,36 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
             if (kb >= nst && !mbar_wait(bar_empty + s, (uint32_t)((kb / nst - 1) & 1)))
                 ok = false;
             const uint32_t a_st = sA + (uint32_t)(s * kAStage);
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int i = 2 * kb + u;
-                const int slot = 2 * warp + u;
-                cp_async_wait<kMRing - 1>();
-                uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                const bool valid = slot < nv;
-                if (valid)
-                    v = *reinterpret_cast<const uint4 *>(myring + (i % kMRing) * kRowBytes1);
-                // refill the ring slot with the row kMRing positions ahead
-                if (i + kMRing < nseq) {
-                    const int j = seq_row(i + kMRing);
-                    if (j >= 0)
-                        cp_async16(myring + (i % kMRing) * kRowBytes1,
-                                   wcol + (size_t)max(ridx[j], 0) * row_bytes);
-                }
-                cp_async_commit();
-                const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    uint32_t t0 = 0u, t1 = 0u, t2 = 0u, t3 = 0u;
-                    if (valid) {
-                        const uint32_t w = wv[j], w8 = w >> 8;
-                        t0 = hsub2(w & 0x000F000Fu, zc[j][0]);
-                        t1 = hsub2(w & 0x00F000F0u, zc[j][1]);
-                        t2 = hsub2(w8 & 0x000F000Fu, zc[j][2]);
-                        t3 = hsub2(w8 & 0x00F000F0u, zc[j][3]);
-                    }
-                    st_shared_v4(a_st + a_chunk_off(lane, j, slot), t0, t1, t2, t3);
-                }
+            cp_async_wait<kMRing - 1>();
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (valid)
+                v = *reinterpret_cast<const uint4 *>(myring + (kb % kMRing) * kRowBytes1);
+            // refill the ring slot with this warp's row kMRing K-blocks ahead
+            if (kb + kMRing < nkb) {
+                const int j = kb_row(kb + kMRing);
+                if (j >= 0)
+                    cp_async16(myring + (kb % kMRing) * kRowBytes1,
+                               wcol + (size_t)max(ridx[j], 0) * row_bytes);
             }
-            {
-                // B operand: x' of slots 2w, 2w + 1 for the 16 batch columns.
-                const int u = lane >> 4, c = lane & 15, slot = 2 * warp + u;
+            cp_async_commit();
+            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                uint32_t t0 = 0u, t1 = 0u, t2 = 0u, t3 = 0u;
+                if (valid) {
+                    const uint32_t w = wv[j], w8 = w >> 8;
+                    t0 = hsub2(w & 0x000F000Fu, zc[j][0]);
+                    t1 = hsub2(w & 0x00F000F0u, zc[j][1]);
+                    t2 = hsub2(w8 & 0x000F000Fu, zc[j][2]);
+                    t3 = hsub2(w8 & 0x00F000F0u, zc[j][3]);
+                }
+                st_shared_v4(a_st + aoff[j], t0, t1, t2, t3);
+            }
+            if (lane < kMmaN) {
+                // B operand: x' of slot `warp` for batch column `lane`.
                 const uint16_t xv =
-                    (slot < nv && c < p.B) ? rxh[(j0 + slot) * bp + c] : (uint16_t)0;
-                asm volatile("st.shared.u16 [%0], %1;" ::"r"(sB + (uint32_t)(s * kBStage) +
-                                                             b_elem_off(c, slot)),
+                    (valid && lane < p.B) ? rxh[(j0 + warp) * bp + lane] : (uint16_t)0;
+                asm volatile("st.shared.u16 [%0], %1;" ::"r"(sB + (uint32_t)(s * kBStage) + boff),
                              "h"(xv)
                              : "memory");
             }
@@ -635,7 +611,7 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
             // while this K-block is being multiplied.
             if (first && run > 0) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
+                for (int i = 0; i < 2; ++i)
                     sfold[i] = snew[i];
                 load_s(grp(rstart[run]), snew); // this run's scales, for its fold
                 fold(run - 1);
@@ -643,24 +619,29 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
         }
         if (nruns > 0) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < 2; ++i)
                 sfold[i] = snew[i];
             fold(nruns - 1);
         }
         cp_async_wait_all();
 
-        // Split-K partials, back in real units (x 2^-S_b, two exact factors).
+        // Split-K partials from the totals, back in real units (x 2^-S_b,
+        // two exact factors).
         if (nkb > 0) {
+            tc_fence_after();
 #pragma unroll
-            for (int c = 0; c < kMmaN; ++c) {
-                if (c < p.B) {
-                    const int E = -s_S[c];
-                    const float f1 = pow2f(E / 2), f2 = pow2f(E - E / 2);
+            for (int i = 0; i < 2; ++i) {
+                float t[kMmaN];
+                tmem_ld16(tmem + tlane + kTotCol + kMmaN * (mbA + i), t);
+                if (fout[i] < nvalid_out) {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        if (fout[i] < nvalid_out)
+                    for (int c = 0; c < kMmaN; ++c) {
+                        if (c < p.B) {
+                            const int E = -s_S[c];
                             atomicAdd(p.ws_acc + (size_t)c * p.N + n0 + fout[i],
-                                      (acc[i][c] * f1) * f2);
+                                      (t[c] * pow2f(E / 2)) * pow2f(E - E / 2));
+                        }
+                    }
                 }
             }
         }
