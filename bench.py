@@ -425,7 +425,7 @@ def run_ours(args, dist: Dist):
     peak, peak_kind = measured_peak()
     rpk = read_peak_gbs()
     achieved = k_bytes / (k_us * 1e-6) / 1e9
-    src = source_hash("gemv.cu", "sgq_device.cuh")
+    src = source_hash("gemv.cu", "gemv_rows.cuh", "sgq_device.cuh")
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
                 "traffic": profiled_traffic({"thresh_acc": "thresh", "gemv_acc": "gemv"}.get(dom, dom), src),
