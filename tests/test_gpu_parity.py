@@ -338,6 +338,31 @@ def test_gemv_all_masked_gives_positive_zero():
     assert g.workspace_is_zero()
 
 
+@pytest.mark.parametrize("B", [12, 16])
+def test_gemv_batch_all_masked_gives_positive_zero(B):
+    """The tensor-core kernel with no active channel: no run, no MMA; y = +0
+    and the workspace stays zero."""
+    case = wl.gemv_case(N=2048, K=1024, group=128, B=B, sparsity=0.5, seed=9)
+    g = GpuGemv(case.W, 128, B)
+    x_d = case.x.to(DEV)
+    g.select(x_d, [float("inf")] * B)
+    assert int(g.count.item()) == 0
+    y, y32 = g.gemv(x_d)
+    assert bits(y).max() == 0 and not torch.signbit(y32).any()
+    assert (y32 == 0).all()
+    assert g.workspace_is_zero()
+    assert g.status.item() == 0
+
+
+@pytest.mark.parametrize("N,K,g,B", [(96, 32, 32, 10), (992, 64, 32, 16), (1056, 128, 64, 9)])
+def test_gemv_batch_tiny_shapes(N, K, g, B):
+    """The tensor-core kernel on one group, one partial tile, or a tile of
+    1024 plus 32 outputs, dense and at 50% sparsity."""
+    for sp in (0.0, 0.5):
+        case = wl.gemv_case(N=N, K=K, group=g, B=B, sparsity=sp, seed=N + K + B)
+        run_list_case(case, what=f"tiny N={N} K={K} g={g} B={B} sparsity={sp}")
+
+
 def test_gemv_nan_channel_never_active():
     case = wl.gemv_case(**wl.TINY, sparsity=0.0, seed=12)
     x = case.x.clone()
