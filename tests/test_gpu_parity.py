@@ -290,10 +290,13 @@ def test_gemv_thresh_ragged(N, K, g):
     check_y(y, y32, y64, sa, "thresh ragged")
 
 
-def test_gemv_exact_integer_case_bitwise():
+@pytest.mark.parametrize("B", [1, 3, 12])
+def test_gemv_exact_integer_case_bitwise(B):
     """Power-of-two scales and small-integer x: every partial sum on both sides
-    is exact, so fp32 y equals the oracle's fp64 y and bf16 y matches bitwise."""
-    rng = np.random.default_rng(80)
+    is exact, so fp32 y equals the oracle's fp64 y and bf16 y matches bitwise
+    (B = 3: the CUDA-core batch kernel; B = 12: the tensor-core kernel, whose
+    products and fp32 sums are exact here too)."""
+    rng = np.random.default_rng(80 + B)
     N, K, g = 2048, 1024, 64
     G = K // g
     q = rng.integers(0, 16, (N, K))
@@ -301,26 +304,27 @@ def test_gemv_exact_integer_case_bitwise():
     s = 2.0 ** rng.integers(-3, 3, (N, G))
     z = rng.integers(0, 16, (N, G))
     W = torch.from_numpy((np.repeat(s, g, 1) * (q - np.repeat(z, g, 1))).astype(np.float16))
-    x = torch.from_numpy(rng.integers(-8, 9, (1, K)).astype(np.float32)).to(torch.bfloat16)
-    gg = GpuGemv(W, g)
+    x = torch.from_numpy(rng.integers(-8, 9, (B, K)).astype(np.float32)).to(torch.bfloat16)
+    gg = GpuGemv(W, g, B)
     x_d = x.to(DEV)
-    gg.select(x_d, [0.0])
+    gg.select(x_d, [0.0] * B)
     y, y32 = gg.gemv(x_d)
-    _, y64, _, yb = oracle_expect(W, g, x, [0.0])
+    _, y64, _, yb = oracle_expect(W, g, x, [0.0] * B)
     assert np.array_equal(y32.cpu().double().numpy(), y64)
     assert np.array_equal(bits(y), yb)
 
 
-def test_gemv_power_of_two_scaling():
-    case = wl.gemv_case(N=2048, K=4096, group=128, sparsity=0.5, seed=81, act="silu")
-    g = GpuGemv(case.W, 128)
+@pytest.mark.parametrize("B", [1, 12])
+def test_gemv_power_of_two_scaling(B):
+    case = wl.gemv_case(N=2048, K=4096, group=128, B=B, sparsity=0.5, seed=81, act="silu")
+    g = GpuGemv(case.W, 128, B)
     x_d = case.x.to(DEV)
     g.select(x_d, case.t)
     _, y0 = g.gemv(x_d)
     _, _, sa, _ = oracle_expect(case.W, 128, case.x, case.t)
     for j in (-20, 7):
         x2 = (case.x.float() * 2.0 ** j).to(torch.bfloat16).to(DEV)
-        g.select(x2, [case.t[0] * 2.0 ** j])
+        g.select(x2, [t * 2.0 ** j for t in case.t])
         _, y2 = g.gemv(x2)
         err = np.abs(y2.cpu().double().numpy() * 2.0 ** -j - y0.cpu().double().numpy())
         assert np.all(err <= 2e-3 * sa)
