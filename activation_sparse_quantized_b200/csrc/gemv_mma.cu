@@ -35,11 +35,13 @@
 //  * Split-K partials go into the fp32 workspace with float reductions; the
 //    shared epilogue kernel turns the workspace into bf16 y.
 //
-// Every wait on a barrier is bounded; a wait that runs out sets
-// SGQ_STATUS_TIMEOUT and the kernel carries on to its end (y is then not
-// valid), freeing its tensor memory. The kernel takes more than half of an
-// SM's shared memory, so at most one of its CTAs is resident per SM and the
-// allocation of 256 tensor-memory columns never waits.
+// Every wait on a barrier is bounded by 0.2 s of wall time; a wait that runs
+// out sets SGQ_STATUS_TIMEOUT, the thread waits on nothing further and the
+// kernel runs to its end (y is then not valid). Before the tensor memory is
+// freed, the issuing thread waits (bounded too) for a commit that covers every
+// MMA of the CTA. The kernel takes more than half of an SM's shared memory, so
+// at most one of its CTAs is resident per SM and the allocation of all 512
+// tensor-memory columns never waits.
 #include "gemv_rows.cuh"
 #include "sgq_device.cuh"
 #include "sgq_launch.h"
@@ -63,7 +65,7 @@ constexpr int kMaxStages = 4;               // operand stages (2..4, by shared m
 constexpr int kMRing = 4;                   // rows in flight per expanding warp
 constexpr int kTmemCols = 512;              // two accumulator sets and the running totals
 constexpr int kTotCol = 256;                // first column of the totals
-constexpr int kMSpin = 1 << 22;             // polls of a barrier before giving up
+constexpr unsigned long long kWaitNs = 200000000ull; // a barrier wait gives up after 0.2 s
 constexpr size_t kOneCtaSmem = 116 * 1024;  // more than half of the SM's shared memory
 
 static_assert(kTotCol + kMBlocks * kMmaN <= kTmemCols, "accumulators and totals");
@@ -148,18 +150,38 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Waits for the phase of the given parity to complete, at most kMSpin polls.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
+__device__ __forceinline__ unsigned long long global_ns()
 {
-    uint32_t ok = 0;
-    for (int it = 0; it < kMSpin && !ok; ++it)
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Waits for the phase of the given parity to complete, for at most kWaitNs of
+// wall time; a thread whose earlier wait gave up (ok == false) does not wait
+// again, so that a broken hand-off ends the kernel within a fraction of a
+// second. Returns ok.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, bool ok)
+{
+    if (!ok)
+        return false;
+    unsigned long long t0 = 0;
+    for (;;) {
+        uint32_t done;
         asm volatile("{\n\t.reg .pred p;\n\t"
                      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
                      "selp.u32 %0, 1, 0, p;\n\t}"
-                     : "=r"(ok)
+                     : "=r"(done)
                      : "r"(smem_u32(bar)), "r"(parity)
                      : "memory");
-    return ok != 0;
+        if (done)
+            return true;
+        const unsigned long long t = global_ns();
+        if (t0 == 0)
+            t0 = t;
+        else if (t - t0 > kWaitNs)
+            return false;
+    }
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -238,7 +260,7 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t bar_full[kMaxStages], bar_empty[kMaxStages];
-    __shared__ __align__(8) uint64_t bar_ready[2], bar_free[2];
+    __shared__ __align__(8) uint64_t bar_ready[2], bar_free[2], bar_done;
     __shared__ uint32_t s_tmem;
     __shared__ int s_nruns, s_nkb;
     __shared__ int s_S[kMmaN];
@@ -272,6 +294,7 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
             mbar_init(bar_ready + d, 1);
             mbar_init(bar_free + d, kMWarps);
         }
+        mbar_init(&bar_done, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     tc_fence_before();
@@ -368,12 +391,10 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
                 kb_run(kb, run);
                 const bool first = kb == rkb[run], last = kb == rkb[run + 1] - 1;
                 const int s = kb % nst;
-                if (!mbar_wait(bar_full + s, (uint32_t)((kb / nst) & 1)))
-                    ok = false;
+                ok = mbar_wait(bar_full + s, (uint32_t)((kb / nst) & 1), ok);
                 tc_fence_after();
                 if (first && run >= 2) {
-                    if (!mbar_wait(bar_free + (run & 1), (uint32_t)(((run >> 1) - 1) & 1)))
-                        ok = false;
+                    ok = mbar_wait(bar_free + (run & 1), (uint32_t)(((run >> 1) - 1) & 1), ok);
                     tc_fence_after();
                 }
                 const uint32_t a_st = sA + (uint32_t)(s * kAStage);
@@ -391,6 +412,10 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
                 if (last)
                     mma_commit(bar_ready + (run & 1));
             }
+            // every MMA of this CTA has completed when bar_done's phase 0 does
+            mma_commit(&bar_done);
+            // (the tensor memory is freed only after that, below)
+            ok = mbar_wait(&bar_done, 0u, true) && ok;
         }
         __syncwarp();
     } else {
@@ -525,8 +550,7 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
         // totals += s 2^c D for run r's accumulators (set r & 1); the totals
         // stay in tensor memory (columns kTotCol..), written by run 0.
         auto fold = [&](int r) {
-            if (!mbar_wait(bar_ready + (r & 1), (uint32_t)((r >> 1) & 1)))
-                ok = false;
+            ok = mbar_wait(bar_ready + (r & 1), (uint32_t)((r >> 1) & 1), ok);
             tc_fence_after();
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
@@ -566,8 +590,8 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
                     load_sz(grp(rstart[run + 1]));
             }
             // The stage's previous K-block has been multiplied.
-            if (kb >= nst && !mbar_wait(bar_empty + s, (uint32_t)((kb / nst - 1) & 1)))
-                ok = false;
+            if (kb >= nst)
+                ok = mbar_wait(bar_empty + s, (uint32_t)((kb / nst - 1) & 1), ok);
             const uint32_t a_st = sA + (uint32_t)(s * kAStage);
             cp_async_wait<kMRing - 1>();
             uint4 v = make_uint4(0u, 0u, 0u, 0u);
