@@ -299,6 +299,31 @@ int sgq_gemv(const void *qweight, const void *sz, int N, int K, int group, const
     return run_gemv(p, ws_bytes, workspace, stream);
 }
 
+int sgq_debug_gemv_withhold(const void *qweight, const void *sz, int N, int K, int group,
+                            const void *x, int B, const int32_t *idx, const int32_t *count,
+                            void *y, float *y_f32, void *workspace, size_t ws_bytes,
+                            int32_t *status, void *stream)
+{
+    if (B <= 8 || B > SGQ_MAX_BATCH)
+        return SGQ_ERR_SHAPE;
+    sgq::GemvProblem p{};
+    p.qweight = static_cast<const uint8_t *>(qweight);
+    p.sz = static_cast<const uint32_t *>(sz);
+    p.x = static_cast<const uint16_t *>(x);
+    p.idx = idx;
+    p.count = count;
+    p.y = static_cast<uint16_t *>(y);
+    p.y_f32 = y_f32;
+    p.status = status;
+    p.N = N;
+    p.K = K;
+    p.group = group;
+    p.B = B;
+    p.source = sgq::ROWS_LIST;
+    p.debug_withhold_ready = 1;
+    return run_gemv(p, ws_bytes, workspace, stream);
+}
+
 int sgq_gemv_thresh(const void *qweight, const void *sz, int N, int K, int group, const void *x,
                     float t, void *y, float *y_f32, void *workspace, size_t ws_bytes,
                     int32_t *status, void *stream)

@@ -409,7 +409,7 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
                             smem_desc(a_st + (uint32_t)(mb * 2048), 1024, 16 * 1024, 2), bdesc,
                             !first);
                 mma_commit(bar_empty + s);
-                if (last)
+                if (last && !(p.debug_withhold_ready && run == nruns - 1))
                     mma_commit(bar_ready + (run & 1));
             }
             // every MMA of this CTA has completed when bar_done's phase 0 does

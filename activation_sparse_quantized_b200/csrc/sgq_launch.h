@@ -54,6 +54,9 @@ struct GemvProblem {
     // the epilogue kernel also zeroes zero_extra[0 .. zero_extra_n) (consumed sums)
     float *zero_extra;
     int zero_extra_n;
+    // test hook (tensor-core batch kernel): withhold the last run's "ready"
+    // commit, so that the waits on it run out and set SGQ_STATUS_TIMEOUT
+    int debug_withhold_ready;
 };
 
 // Bytes of workspace (partial sums + tile counters) for N outputs, B rows.

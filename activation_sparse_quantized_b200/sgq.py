@@ -34,7 +34,7 @@ EXPORTS = (
     "sgq_layout_version", "sgq_gemv_thresh_noalloc", "sgq_gemv_glu", "sgq_gemv_glu_thresh",
     "sgq_gemv_glu_dense", "sgq_select_mask", "sgq_gemv_mask", "sgq_packed_sizes_nm",
     "sgq_pack_nm", "sgq_gemv_nm", "sgq_gemv_nm_thresh", "sgq_gemv_acc", "sgq_gemv_thresh_acc",
-    "sgq_ffn_workspace_bytes", "sgq_ffn", "sgq_read_status",
+    "sgq_ffn_workspace_bytes", "sgq_ffn", "sgq_read_status", "sgq_debug_gemv_withhold",
 )
 
 
@@ -78,6 +78,7 @@ def _declare(lib):
         "sgq_select": ([P, I, I, P, P, P, P], I),
         "sgq_gemv_workspace_bytes": ([I, I, I], Z),
         "sgq_gemv": ([P, P, I, I, I, P, I, P, P, P, P, P, Z, P, P], I),
+        "sgq_debug_gemv_withhold": ([P, P, I, I, I, P, I, P, P, P, P, P, Z, P, P], I),
         "sgq_gemv_thresh": ([P, P, I, I, I, P, F, P, P, P, Z, P, P], I),
         "sgq_gemv_dense": ([P, P, I, I, I, P, I, P, P, P, Z, P, P], I),
         "sgq_gemv_thresh_noalloc": ([P, P, I, I, I, P, F, P, P, P, P], I),
@@ -220,6 +221,16 @@ def sgq_gemv_workspace_bytes(N: int, K: int, B: int) -> int:
 def sgq_gemv(qweight, sz, N, K, group, x, B, idx, count, y, y_f32, workspace, status=None,
              stream=None):
     _check("sgq_gemv", load().sgq_gemv(
+        _ptr(qweight), _ptr(sz), N, K, group, _ptr(x), B, _ptr(idx), _ptr(count), _ptr(y),
+        _ptr(y_f32), _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status),
+        _stream(stream)))
+
+
+def sgq_debug_gemv_withhold(qweight, sz, N, K, group, x, B, idx, count, y, y_f32, workspace,
+                            status, stream=None):
+    """Test hook: sgq_gemv (B = 9..16) whose last group run is never released,
+    so the kernel's bounded waits run out and set SGQ_STATUS_TIMEOUT."""
+    _check("sgq_debug_gemv_withhold", load().sgq_debug_gemv_withhold(
         _ptr(qweight), _ptr(sz), N, K, group, _ptr(x), B, _ptr(idx), _ptr(count), _ptr(y),
         _ptr(y_f32), _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status),
         _stream(stream)))

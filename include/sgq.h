@@ -357,6 +357,20 @@ int sgq_last_cuda_error(void);
 /* SGQ_LAYOUT_VERSION of the packed format this build reads and writes. */
 int sgq_layout_version(void);
 
+/*
+ * Test hook for the device-side wait limits (not for production use):
+ * sgq_gemv with B = 9..16 (the tensor-core kernel) in which the MMA issuer
+ * withholds the commit that releases the last group run's accumulators. The
+ * CTAs' waits on it give up after 0.2 s, SGQ_STATUS_TIMEOUT is set in *status
+ * (status must be non-NULL to see it), y is not valid, and the kernel still
+ * frees its tensor memory only after its MMAs have completed; the context
+ * stays usable. Arguments as sgq_gemv; B outside 9..16 returns SGQ_ERR_SHAPE.
+ */
+int sgq_debug_gemv_withhold(const void *qweight, const void *sz, int N, int K, int group,
+                            const void *x, int B, const int32_t *idx, const int32_t *count,
+                            void *y, float *y_f32, void *workspace, size_t ws_bytes,
+                            int32_t *status, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -520,6 +520,35 @@ def test_gemv_batch_bad_index_is_skipped(B):
     assert g.workspace_is_zero()
 
 
+def test_batch_kernel_wait_limit_sets_timeout_and_context_survives():
+    """Fault injection from the host: the tensor-core kernel's issuer withholds
+    the release of the last group run, so the waits on it run out (0.2 s);
+    the status word carries SGQ_STATUS_TIMEOUT, the call returns, and the
+    next ordinary call on the same context and workspace is correct."""
+    B = 12
+    case = wl.gemv_case(N=2048, K=2048, group=128, B=B, sparsity=0.5, seed=95)
+    g = GpuGemv(case.W, 128, B)
+    x_d = case.x.to(DEV)
+    g.select(x_d, case.t)
+    y, y32 = g.outputs(B)
+    sgq.sgq_debug_gemv_withhold(g.qw, g.sz, g.N, g.K, 128, x_d, B, g.idx, g.count, y, y32,
+                                g.ws, g.status)
+    torch.cuda.synchronize()
+    assert g.status.item() & sgq.SGQ_STATUS_TIMEOUT
+    # the partial sums of the broken call are still in the workspace: clear it
+    g.ws.zero_()
+    g.status.zero_()
+    y, y32 = g.gemv(x_d)
+    idx, y64, sa, _ = oracle_expect(case.W, 128, case.x, case.t)
+    torch.cuda.synchronize()
+    check_y(y, y32, y64, sa, "after a timed-out call")
+    assert g.status.item() == 0
+    assert g.workspace_is_zero()
+    with pytest.raises(sgq.SgqError):
+        sgq.sgq_debug_gemv_withhold(g.qw, g.sz, g.N, g.K, 128, x_d, 4, g.idx, g.count, y, y32,
+                                    g.ws, g.status)
+
+
 def test_read_status_returns_and_clears_the_word():
     W = wl.weight(64, 128, 8)
     W[3, 9] = float("nan")
