@@ -1,4 +1,4 @@
-// gemv_mma.cu -- the activation-sparse GEMV for batch 2..16, on the tensor cores.
+// gemv_mma.cu -- the activation-sparse GEMV for batch 9..16, on the tensor cores.
 //
 //   y[b][n] = sum_{k in U} s[g(k)][n] * (q[k][n] - z[g(k)][n]) * x[b][k]
 //
@@ -8,30 +8,33 @@
 // layout that reads only the weight runs of the active channels.
 //
 // With B batch rows every weight code is used B times. The CUDA-core kernel
-// (one FMA per code and batch row) is bound by FMA issue well before HBM once
-// B >= 2, so here each code is expanded once into an exact fp16 operand and
-// the products go to the tensor cores (tcgen05.mma kind::f16, fp32
-// accumulators in tensor memory):
+// (one FMA per code and batch row) is bound by FMA issue well before HBM from
+// B of about 4, and above 8 rows each of its warps carries every row of its
+// CTA; there each code is expanded once into an exact fp16 operand and the
+// products go to the tensor cores (tcgen05.mma kind::f16, fp32 accumulators
+// in tensor memory):
 //  * Tiles of 1024 outputs (512 bytes of a packed row) and k_splits shares of
 //    the rows per tile, as in the batch-1 kernel, with the same row lists.
 //  * The CTA's rows are cut into runs of one quantization group, and each run
 //    into K-blocks of 16 rows (the MMA's K; a run's last block is padded with
 //    zero rows).
-//  * 8 warps; warp w expands slots 2w and 2w + 1 of every K-block. Its lanes
-//    stream their own 16-byte columns of those rows through per-lane cp.async
-//    rings (8 rows ahead) and turn each code, minus the group's zero, into the
-//    exact fp16 value (q - z) 2^-24 (2^-20 for the high nibble of a byte): one
-//    AND and one packed fp16 subtraction per two codes, the zero being held in
-//    the same subnormal form. A K-block's A operand (1024 outputs x 16 rows,
-//    M-major, 128-byte swizzle) and B operand (16 rows x 16 batch columns of
-//    x' = x 2^S_b in fp16, K-major) go to one of two stages.
-//  * One thread issues the K-block's 8 MMAs (M = 128 outputs, N = 16, K = 16)
-//    into the run's accumulators (two alternating sets of 8 x 16 columns of
-//    tensor memory), then commits them to the stage's "empty" barrier and, at
-//    a run's end, to the set's "ready" barrier.
-//  * A run later every thread reads its outputs' sums from tensor memory and
-//    folds them with the group's scale: acc += s 2^c D. The products are those
-//    of the batch-1 kernel (exact fp16 x fp16), summed in fp32.
+//  * 16 expanding warps; warp w expands slot w of every K-block. Its lanes
+//    stream their own 16-byte columns of its rows through per-lane cp.async
+//    rings (4 K-blocks ahead) and turn each code, minus the group's zero,
+//    into the exact fp16 value (q - z) 2^-24 (2^-20 for the high nibble of a
+//    byte): one AND and one packed fp16 subtraction per two codes, the zero
+//    being held in the same subnormal form. A K-block's A operand (1024
+//    outputs x 16 rows, M-major, 128-byte swizzle) and B operand (16 rows x
+//    16 batch columns of x' = x 2^S_b in fp16, K-major) go to one of 2..4
+//    stages.
+//  * A 17th warp issues the K-block's 8 MMAs (M = 128 outputs, N = 16,
+//    K = 16) into the run's accumulators (two alternating sets of 8 x 16
+//    columns of tensor memory), then commits them to the stage's "empty"
+//    barrier and, at a run's end, to the set's "ready" barrier.
+//  * A run later the expanding warps read their outputs' sums from tensor
+//    memory and fold them with the group's scale into running totals, also
+//    in tensor memory: total += s 2^c D. The products are those of the
+//    batch-1 kernel (exact fp16 x fp16), summed in fp32.
 //  * Split-K partials go into the fp32 workspace with float reductions; the
 //    shared epilogue kernel turns the workspace into bf16 y.
 //
