@@ -123,10 +123,15 @@ struct SmemM {
 
 __host__ __device__ inline size_t align16(size_t v) { return (v + 15) / 16 * 16; }
 
+// Row stride of the staged x' (batch-major): an odd multiple of 8 rows, so
+// that a lane's 8 rows are one 16-byte access and the 16 batch columns of one
+// row fall into distinct bank pairs.
+__host__ __device__ inline int rxh_stride(int rows_cap) { return (((rows_cap + 7) / 8) | 1) * 8; }
+
 // a: `stages` A stages (1024-aligned); b: B stages; ring: each expanding
-// warp's per-lane rings; rxh: x' of each row, [row][bp batch columns] fp16;
-// ridx: the CTA's rows; rstart / rkb: first row / first K-block of each run
-// (+1 entry); scan: per-32-row counts.
+// warp's per-lane rings; rxh: x' of the CTA's rows, [bp batch rows][stride]
+// fp16; ridx: the CTA's rows; rstart / rkb: first row / first K-block of each
+// run (+1 entry); scan: per-32-row counts.
 __host__ __device__ inline SmemM smemm_layout(int rows_cap, int stages, int bp)
 {
     SmemM s;
@@ -134,7 +139,7 @@ __host__ __device__ inline SmemM smemm_layout(int rows_cap, int stages, int bp)
     s.b = s.a + (size_t)stages * kAStage;
     s.ring = s.b + (size_t)stages * kBStage;
     s.rxh = s.ring + (size_t)kMWarps * kMRing * kRowBytes1;
-    s.ridx = align16(s.rxh + (size_t)rows_cap * bp * 2);
+    s.ridx = align16(s.rxh + (size_t)bp * rxh_stride(rows_cap) * 2);
     s.rstart = align16(s.ridx + (size_t)rows_cap * 4);
     s.rkb = align16(s.rstart + (size_t)(rows_cap + 1) * 4);
     s.scan = align16(s.rkb + (size_t)(rows_cap + 1) * 4);
@@ -427,6 +432,80 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
         // per K-block, through a per-lane ring kMRing K-blocks ahead (with its
         // own run pointer).
         constexpr int kEx = kMWarps * 32; // threads of the expanding warps
+        // x' = x 2^S_b in fp16 per batch row b, 2^14 <= max |x'| < 2^15 over
+        // the CTA's rows (as in the batch-1 kernel), staged batch-major in
+        // rxh. Warp w owns batch row b = w: each lane gathers chunks of 8 rows
+        // (one 16-byte load when the 8 rows are 8 consecutive aligned
+        // channels), four chunks in flight, before any weight row is
+        // requested; the warp reduces max |x|, then converts its row in place.
+        const int rs = rxh_stride(kp.rows_cap);
+        if (warp < p.B) {
+            const int b = warp;
+            uint16_t *xr = rxh + (size_t)b * rs;
+            const uint16_t *xb = p.x + (size_t)b * p.K;
+            const int nch = (nr + 7) / 8;
+            float m = 0.f;
+            for (int c0 = lane; c0 < nch; c0 += 4 * 32) {
+                uint4 v[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int c = c0 + 32 * u;
+                    v[u] = make_uint4(0u, 0u, 0u, 0u);
+                    if (c < nch) {
+                        const int j0 = 8 * c;
+                        const int k0 = ridx[j0];
+                        bool vec = (j0 + 8 <= nr) && k0 >= 0 && (k0 & 7) == 0;
+#pragma unroll
+                        for (int i = 1; i < 8; ++i)
+                            vec = vec && (ridx[min(j0 + i, nr - 1)] == k0 + i);
+                        if (vec) {
+                            v[u] = __ldg(reinterpret_cast<const uint4 *>(xb + k0));
+                        } else {
+                            uint32_t h[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const int k = (j0 + i < nr) ? ridx[j0 + i] : -1;
+                                h[i] = (k >= 0) ? (uint32_t)__ldg(xb + k) : 0u;
+                            }
+                            v[u] = make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16),
+                                              h[4] | (h[5] << 16), h[6] | (h[7] << 16));
+                        }
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int c = c0 + 32 * u;
+                    if (c < nch) {
+                        *reinterpret_cast<uint4 *>(xr + 8 * c) = v[u];
+                        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            m = fmaxf(m, fabsf(bf16_bits_to_float(
+                                             (uint16_t)(w[i >> 1] >> (16 * (i & 1))))));
+                    }
+                }
+            }
+            const int e = warp_max_exponent(m);
+            const int S = (e == INT32_MIN) ? 0 : 14 - e;
+            if (lane == 0)
+                s_S[b] = S;
+            const float fa = pow2f(S - S / 2), fb = pow2f(S / 2);
+            __syncwarp();
+            for (int c = lane; c < nch; c += 32) {
+                uint4 v = *reinterpret_cast<const uint4 *>(xr + 8 * c);
+                uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t lo = __half_as_ushort(__float2half_rn(
+                        (bf16_bits_to_float((uint16_t)(w[i] & 0xffffu)) * fa) * fb));
+                    const uint32_t hi = __half_as_ushort(__float2half_rn(
+                        (bf16_bits_to_float((uint16_t)(w[i] >> 16)) * fa) * fb));
+                    w[i] = lo | (hi << 16);
+                }
+                *reinterpret_cast<uint4 *>(xr + 8 * c) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        }
+
         const size_t row_bytes = (size_t)(p.N / 2);
         const uint8_t *wcol = p.qweight + (lane_ok ? ((size_t)n0 / 2 + lane * 16) : 0);
         uint8_t *myring = ring + (size_t)warp * kMRing * kRowBytes1 + lane * 16;
@@ -503,53 +582,6 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
             load_s(grp(rstart[0]), snew);
         }
 
-        // x' = x 2^S_b in fp16 per batch row b, 2^14 <= max |x'| < 2^15 over
-        // the CTA's rows (as in the batch-1 kernel), staged as rxh[row][bp].
-        // Warp w owns batch row b = w: its lanes gather x of the rows, 8 rows
-        // per item (one 16-byte load when the 8 rows are 8 consecutive aligned
-        // channels), the warp reduces max |x|, then converts its column.
-        if (warp < p.B) {
-            const int b = warp;
-            const uint16_t *xb = p.x + (size_t)b * p.K;
-            float m = 0.f;
-            for (int j0 = 8 * lane; j0 < nr; j0 += 8 * 32) {
-                const int k0 = ridx[j0];
-                bool vec = (j0 + 8 <= nr) && k0 >= 0 && (k0 & 7) == 0;
-#pragma unroll
-                for (int i = 1; i < 8; ++i)
-                    vec = vec && (ridx[min(j0 + i, nr - 1)] == k0 + i);
-                uint32_t h[8];
-                if (vec) {
-                    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(xb + k0));
-                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        h[i] = (w[i >> 1] >> (16 * (i & 1))) & 0xffffu;
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int k = (j0 + i < nr) ? ridx[j0 + i] : -1;
-                        h[i] = (k >= 0) ? (uint32_t)__ldg(xb + k) : 0u;
-                    }
-                }
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    if (j0 + i < nr) {
-                        rxh[(j0 + i) * bp + b] = (uint16_t)h[i];
-                        m = fmaxf(m, fabsf(bf16_bits_to_float((uint16_t)h[i])));
-                    }
-            }
-            const int e = warp_max_exponent(m);
-            const int S = (e == INT32_MIN) ? 0 : 14 - e;
-            if (lane == 0)
-                s_S[b] = S;
-            const float fa = pow2f(S - S / 2), fb = pow2f(S / 2);
-            for (int j = lane; j < nr; j += 32)
-                rxh[j * bp + b] = __half_as_ushort(
-                    __float2half_rn((bf16_bits_to_float(rxh[j * bp + b]) * fa) * fb));
-        }
-        asm volatile("bar.sync 1, %0;" ::"n"(kEx) : "memory");
-
         // totals += s 2^c D for run r's accumulators (set r & 1); the totals
         // stay in tensor memory (columns kTotCol..), written by run 0.
         auto fold = [&](int r) {
@@ -579,6 +611,9 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
             if (lane == 0)
                 mbar_arrive(bar_free + (r & 1));
         };
+
+        // every batch row's x' (written by its warp above) is in place
+        asm volatile("bar.sync 1, %0;" ::"n"(kEx) : "memory");
 
         int run = 0;
         for (int kb = 0; kb < nkb; ++kb) {
@@ -624,7 +659,7 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
             if (lane < kMmaN) {
                 // B operand: x' of slot `warp` for batch column `lane`.
                 const uint16_t xv =
-                    (valid && lane < p.B) ? rxh[(j0 + warp) * bp + lane] : (uint16_t)0;
+                    (valid && lane < p.B) ? rxh[(size_t)lane * rs + j0 + warp] : (uint16_t)0;
                 asm volatile("st.shared.u16 [%0], %1;" ::"r"(sB + (uint32_t)(s * kBStage) + boff),
                              "h"(xv)
                              : "memory");
