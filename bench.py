@@ -935,7 +935,24 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-ffn", action="store_true",
                     help="skip the secondary FFN / decode-layer leg (fused vs unfused)")
+    ap.add_argument("--profile-batch", type=int, default=0, metavar="B",
+                    help="profiling aid: run only the Qwen3-32B FFN at batch B for --steps "
+                         "FFNs and exit (prints one line of timing, no JSON contract line)")
     args = ap.parse_args(argv)
+    if args.profile_batch:
+        torch.cuda.set_device(0)
+        f = BatchFfnReplica()
+        f.setup(args.profile_batch)
+        for i in range(max(3, args.warmup)):
+            f.ffn(i % f.R)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for i in range(args.steps):
+            f.ffn(i % f.R)
+        torch.cuda.synchronize()
+        print(f"Qwen3-32B FFN batch {args.profile_batch}: "
+              f"{(time.perf_counter() - t0) * 1e6 / args.steps:.1f} us per FFN (host clock)")
+        return 0
     if args.warmup < 3:
         args.warmup = 3
     dist = Dist()
