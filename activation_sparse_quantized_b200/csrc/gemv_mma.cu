@@ -263,6 +263,65 @@ __device__ __forceinline__ uint32_t zero_of(uint32_t w)
     return (uint32_t)__float2int_rn(__half2float(__ushort_as_half((uint16_t)(w >> 16))));
 }
 
+// Rows of one segment into ridx (ascending positions of the caller's list, or
+// of the active channels), returns their number. Index list: entries
+// [lo, hi) of idx (outside [0, K) -> -1, flagged); dense: channels
+// [8 lo, 8 hi); bitmask: the active channels of [8 lo, 8 hi), by ballots over
+// runs of 32 channels and a prefix over the runs' counts. All threads; ends
+// with a barrier.
+template <int SRC>
+__device__ int segment_rows(const GemvProblem &p, int lo, int hi, int32_t *ridx, int *scan)
+{
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (SRC == ROWS_LIST) {
+        for (int j = tid; j < hi - lo; j += kMThreads) {
+            int k = __ldg(p.idx + lo + j);
+            if ((unsigned)k >= (unsigned)p.K) {
+                set_status(p.status, SGQ_STATUS_BAD_INDEX);
+                k = -1;
+            }
+            ridx[j] = k;
+        }
+        __syncthreads();
+        return hi - lo;
+    } else if (SRC == ROWS_DENSE) {
+        const int c0 = 8 * lo, n = 8 * (hi - lo);
+        for (int j = tid; j < n; j += kMThreads)
+            ridx[j] = c0 + j;
+        __syncthreads();
+        return n;
+    } else {
+        const int c0 = 8 * lo, c1 = 8 * hi;
+        const int runs = (c1 - c0 + 31) / 32;
+        auto run_bits = [&](int q) -> uint32_t {
+            const int c = c0 + q * 32 + lane;
+            const bool act = (c < c1) && ((__ldg(p.mask + (c >> 5)) >> (c & 31)) & 1u);
+            return __ballot_sync(0xffffffffu, act);
+        };
+        for (int q = warp; q < runs; q += kAllWarps) {
+            const uint32_t m = run_bits(q);
+            if (lane == 0)
+                scan[q] = __popc(m);
+        }
+        __syncthreads();
+        int total = 0;
+        for (int c = 0; c * 32 < runs; ++c) {
+            int ct;
+            const int excl = chunk_prefix(scan, runs, c, total, &ct);
+            for (int q = c * 32 + ((warp - c * 32) % kAllWarps + kAllWarps) % kAllWarps;
+                 q < runs && q < c * 32 + 32; q += kAllWarps) {
+                const int base = __shfl_sync(0xffffffffu, excl, q - c * 32);
+                const uint32_t m = run_bits(q);
+                if ((m >> lane) & 1u)
+                    ridx[base + __popc(m & ((1u << lane) - 1u))] = c0 + q * 32 + lane;
+            }
+            total += ct;
+        }
+        __syncthreads();
+        return total;
+    }
+}
+
 template <int SRC>
 __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp)
 {
@@ -311,402 +370,434 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
     const uint32_t tmem = s_tmem;
 
     grid_launch_dependents();
-    const int tile = blockIdx.x % kp.n_tiles;
-    const int split = blockIdx.x / kp.n_tiles;
-    const int n0 = tile * kTileN1;
     const int lg = kp.lg;
-    const int nvalid_out = min(kTileN1, p.N - n0); // outputs of this tile
-    const bool lane_ok = 32 * lane < nvalid_out;
     bool ok = true;
 
     grid_dependency_wait(); // x, idx, count, mask may come from the previous kernel
 
-    // The CTA's rows (invalid list entries are -1: read as row 0 with x = 0).
-    const int nr = build_rows<SRC, kMThreads, false>(kp, split, ridx, nullptr, scan);
-    auto grp = [&](int j) { return max(ridx[j], 0) >> lg; };
-
-    // Runs of one group: starts by ballots over chunks of 32 rows, positions
-    // by a prefix over the chunks' counts.
-    const int chunks = (nr + 31) / 32;
-    for (int q = warp; q < chunks; q += kAllWarps) {
-        const int j = q * 32 + lane;
-        const bool st = (j < nr) && (j == 0 || grp(j) != grp(j - 1));
-        const uint32_t m = __ballot_sync(0xffffffffu, st);
-        if (lane == 0)
-            scan[q] = __popc(m);
+    // This CTA's equal share [u0, u1) of the (tile, row) work: units of one
+    // list entry (index list) or of 8 channels (dense, bitmask) per tile, so
+    // that every SM gets the same amount whatever the number of tiles. A share
+    // may end one tile and start the next: each part is a segment, processed
+    // in turn, each adding into the workspace. Barrier phases and the
+    // accumulator sets run on CTA-wide K-block and run counters.
+    int per_tile;
+    if (SRC == ROWS_LIST) {
+        const int c = __ldg(p.count);
+        per_tile = c < 0 ? 0 : (c > p.K ? p.K : c);
+        if (per_tile != c && tid == 0 && blockIdx.x == 0)
+            set_status(p.status, SGQ_STATUS_BAD_COUNT);
+    } else {
+        per_tile = p.K / 8;
     }
-    __syncthreads();
-    {
-        int total = 0;
-        for (int c = 0; c * 32 < chunks; ++c) {
-            int ct;
-            const int excl = chunk_prefix(scan, chunks, c, total, &ct);
-            for (int q = c * 32 + ((warp - c * 32) % kAllWarps + kAllWarps) % kAllWarps;
-                 q < chunks && q < c * 32 + 32; q += kAllWarps) {
-                const int base = __shfl_sync(0xffffffffu, excl, q - c * 32);
-                const int j = q * 32 + lane;
-                const bool st = (j < nr) && (j == 0 || grp(j) != grp(j - 1));
-                const uint32_t m = __ballot_sync(0xffffffffu, st);
-                if (st)
-                    rstart[base + __popc(m & ((1u << lane) - 1u))] = j;
+    const long long W = (long long)kp.n_tiles * per_tile; // < 2^31 (checked by the launcher)
+    const int u0 = (int)(W * blockIdx.x / gridDim.x);
+    const int u1 = (int)(W * (blockIdx.x + 1) / gridDim.x);
+    int kb_base = 0, run_base = 0;
+    for (int u = u0; u < u1;) {
+        const int tile = u / per_tile;
+        const int lo = u - tile * per_tile;
+        const int hi = min(per_tile, u1 - tile * per_tile);
+        u = tile * per_tile + hi;
+        const int n0 = tile * kTileN1;
+        const int nvalid_out = min(kTileN1, p.N - n0); // outputs of this tile
+        const bool lane_ok = 32 * lane < nvalid_out;
+        __syncthreads(); // the previous segment's readers of the row arrays are done
+
+        // The segment's rows (invalid list entries are -1: read as row 0, x = 0).
+        const int nr = segment_rows<SRC>(p, lo, hi, ridx, scan);
+        auto grp = [&](int j) { return max(ridx[j], 0) >> lg; };
+
+        // Runs of one group: starts by ballots over chunks of 32 rows, positions
+        // by a prefix over the chunks' counts.
+        const int chunks = (nr + 31) / 32;
+        for (int q = warp; q < chunks; q += kAllWarps) {
+            const int j = q * 32 + lane;
+            const bool st = (j < nr) && (j == 0 || grp(j) != grp(j - 1));
+            const uint32_t m = __ballot_sync(0xffffffffu, st);
+            if (lane == 0)
+                scan[q] = __popc(m);
+        }
+        __syncthreads();
+        {
+            int total = 0;
+            for (int c = 0; c * 32 < chunks; ++c) {
+                int ct;
+                const int excl = chunk_prefix(scan, chunks, c, total, &ct);
+                for (int q = c * 32 + ((warp - c * 32) % kAllWarps + kAllWarps) % kAllWarps;
+                     q < chunks && q < c * 32 + 32; q += kAllWarps) {
+                    const int base = __shfl_sync(0xffffffffu, excl, q - c * 32);
+                    const int j = q * 32 + lane;
+                    const bool st = (j < nr) && (j == 0 || grp(j) != grp(j - 1));
+                    const uint32_t m = __ballot_sync(0xffffffffu, st);
+                    if (st)
+                        rstart[base + __popc(m & ((1u << lane) - 1u))] = j;
+                }
+                total += ct;
             }
-            total += ct;
-        }
-        if (tid == 0) {
-            s_nruns = total;
-            rstart[total] = nr;
-        }
-    }
-    __syncthreads();
-    const int nruns = s_nruns;
-    // First K-block of each run: a prefix over the runs' K-block counts.
-    if (warp == 0) {
-        int carry = 0;
-        for (int c = 0; c * 32 < nruns; ++c) {
-            const int r = c * 32 + lane;
-            const int v = (r < nruns) ? (rstart[r + 1] - rstart[r] + kKb - 1) / kKb : 0;
-            int incl = v;
-#pragma unroll
-            for (int d = 1; d < 32; d <<= 1) {
-                const int t = __shfl_up_sync(0xffffffffu, incl, d);
-                if (lane >= d)
-                    incl += t;
+            if (tid == 0) {
+                s_nruns = total;
+                rstart[total] = nr;
             }
-            if (r < nruns)
-                rkb[r] = carry + incl - v;
-            carry += __shfl_sync(0xffffffffu, incl, 31);
         }
-        if (lane == 0) {
-            rkb[nruns] = carry;
-            s_nkb = carry;
+        __syncthreads();
+        const int nruns = s_nruns;
+        // First K-block of each run: a prefix over the runs' K-block counts.
+        if (warp == 0) {
+            int carry = 0;
+            for (int c = 0; c * 32 < nruns; ++c) {
+                const int r = c * 32 + lane;
+                const int v = (r < nruns) ? (rstart[r + 1] - rstart[r] + kKb - 1) / kKb : 0;
+                int incl = v;
+    #pragma unroll
+                for (int d = 1; d < 32; d <<= 1) {
+                    const int t = __shfl_up_sync(0xffffffffu, incl, d);
+                    if (lane >= d)
+                        incl += t;
+                }
+                if (r < nruns)
+                    rkb[r] = carry + incl - v;
+                carry += __shfl_sync(0xffffffffu, incl, 31);
+            }
+            if (lane == 0) {
+                rkb[nruns] = carry;
+                s_nkb = carry;
+            }
         }
-    }
-    __syncthreads();
-    const int nkb = s_nkb;
+        __syncthreads();
+        const int nkb = s_nkb;
 
-    // K-block kb: its run (a pointer advanced monotonically), the ridx
-    // position of its slot 0 and its valid slots.
-    auto kb_run = [&](int kb, int &run) {
-        while (kb >= rkb[run + 1])
-            ++run;
-    };
+        // K-block kb: its run (a pointer advanced monotonically), the ridx
+        // position of its slot 0 and its valid slots.
+        auto kb_run = [&](int kb, int &run) {
+            while (kb >= rkb[run + 1])
+                ++run;
+        };
 
-    if (warp == kIssuer) {
-        // ---- the MMA issuer --------------------------------------------------
-        if (lane == 0) {
+        if (warp == kIssuer) {
+            // ---- the MMA issuer --------------------------------------------------
+            if (lane == 0) {
+                int run = 0;
+                for (int kb = 0; kb < nkb; ++kb) {
+                    kb_run(kb, run);
+                    const bool first = kb == rkb[run], last = kb == rkb[run + 1] - 1;
+                    const int kg = kb_base + kb, rg = run_base + run;
+                    const int s = kg % nst;
+                    ok = mbar_wait(bar_full + s, (uint32_t)((kg / nst) & 1), ok);
+                    tc_fence_after();
+                    if (first && rg >= 2) {
+                        ok = mbar_wait(bar_free + (rg & 1), (uint32_t)(((rg >> 1) - 1) & 1), ok);
+                        tc_fence_after();
+                    }
+                    const uint32_t a_st = sA + (uint32_t)(s * kAStage);
+                    const uint32_t dcol = tmem + (uint32_t)(128 * (rg & 1));
+                    const uint64_t bdesc = smem_desc(sB + (uint32_t)(s * kBStage), 128, 256, 0);
+                    // Every M-block: a lane's outputs are spread over the M-blocks
+                    // (lanes past N hold finite codes of column 0 and are dropped
+                    // in the epilogue).
+    #pragma unroll
+                    for (int mb = 0; mb < kMBlocks; ++mb)
+                        mma_f16(dcol + (uint32_t)(kMmaN * mb),
+                                smem_desc(a_st + (uint32_t)(mb * 2048), 1024, 16 * 1024, 2), bdesc,
+                                !first);
+                    mma_commit(bar_empty + s);
+                    if (last && !(p.debug_withhold_ready && run == nruns - 1))
+                        mma_commit(bar_ready + (rg & 1));
+                }
+            }
+            __syncwarp();
+        } else {
+            // ---- the expanding warps ---------------------------------------------
+            // Warp w expands slot w of every K-block: its row stream is one row
+            // per K-block, through a per-lane ring kMRing K-blocks ahead (with its
+            // own run pointer).
+            constexpr int kEx = kMWarps * 32; // threads of the expanding warps
+            // x' = x 2^S_b in fp16 per batch row b, 2^14 <= max |x'| < 2^15 over
+            // the CTA's rows (as in the batch-1 kernel), staged batch-major in
+            // rxh. Warp w owns batch row b = w: each lane gathers chunks of 8 rows
+            // (one 16-byte load when the 8 rows are 8 consecutive aligned
+            // channels), four chunks in flight, before any weight row is
+            // requested; the warp reduces max |x|, then converts its row in place.
+            const int rs = rxh_stride(kp.rows_cap);
+            if (warp < p.B) {
+                const int b = warp;
+                uint16_t *xr = rxh + (size_t)b * rs;
+                const uint16_t *xb = p.x + (size_t)b * p.K;
+                const int nch = (nr + 7) / 8;
+                float m = 0.f;
+                for (int c0 = lane; c0 < nch; c0 += 4 * 32) {
+                    uint4 v[4];
+    #pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int c = c0 + 32 * u;
+                        v[u] = make_uint4(0u, 0u, 0u, 0u);
+                        if (c < nch) {
+                            const int j0 = 8 * c;
+                            const int k0 = ridx[j0];
+                            bool vec = (j0 + 8 <= nr) && k0 >= 0 && (k0 & 7) == 0;
+    #pragma unroll
+                            for (int i = 1; i < 8; ++i)
+                                vec = vec && (ridx[min(j0 + i, nr - 1)] == k0 + i);
+                            if (vec) {
+                                v[u] = __ldg(reinterpret_cast<const uint4 *>(xb + k0));
+                            } else {
+                                uint32_t h[8];
+    #pragma unroll
+                                for (int i = 0; i < 8; ++i) {
+                                    const int k = (j0 + i < nr) ? ridx[j0 + i] : -1;
+                                    h[i] = (k >= 0) ? (uint32_t)__ldg(xb + k) : 0u;
+                                }
+                                v[u] = make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16),
+                                                  h[4] | (h[5] << 16), h[6] | (h[7] << 16));
+                            }
+                        }
+                    }
+    #pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int c = c0 + 32 * u;
+                        if (c < nch) {
+                            *reinterpret_cast<uint4 *>(xr + 8 * c) = v[u];
+                            const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+    #pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                m = fmaxf(m, fabsf(bf16_bits_to_float(
+                                                 (uint16_t)(w[i >> 1] >> (16 * (i & 1))))));
+                        }
+                    }
+                }
+                const int e = warp_max_exponent(m);
+                const int S = (e == INT32_MIN) ? 0 : 14 - e;
+                if (lane == 0)
+                    s_S[b] = S;
+                const float fa = pow2f(S - S / 2), fb = pow2f(S / 2);
+                __syncwarp();
+                for (int c = lane; c < nch; c += 32) {
+                    uint4 v = *reinterpret_cast<const uint4 *>(xr + 8 * c);
+                    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    #pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t lo = __half_as_ushort(__float2half_rn(
+                            (bf16_bits_to_float((uint16_t)(w[i] & 0xffffu)) * fa) * fb));
+                        const uint32_t hi = __half_as_ushort(__float2half_rn(
+                            (bf16_bits_to_float((uint16_t)(w[i] >> 16)) * fa) * fb));
+                        w[i] = lo | (hi << 16);
+                    }
+                    *reinterpret_cast<uint4 *>(xr + 8 * c) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+
+            const size_t row_bytes = (size_t)(p.N / 2);
+            const uint8_t *wcol = p.qweight + (lane_ok ? ((size_t)n0 / 2 + lane * 16) : 0);
+            uint8_t *myring = ring + (size_t)warp * kMRing * kRowBytes1 + lane * 16;
+            int ring_run = 0;
+            auto kb_row = [&](int kb) -> int { // ridx position of this warp's slot, or -1
+                kb_run(kb, ring_run);
+                const int j = rstart[ring_run] + kKb * (kb - rkb[ring_run]) + warp;
+                return (j < rstart[ring_run + 1]) ? j : -1;
+            };
+    #pragma unroll
+            for (int i = 0; i < kMRing; ++i) {
+                if (i < nkb) {
+                    const int j = kb_row(i);
+                    if (j >= 0)
+                        cp_async16(myring + i * kRowBytes1,
+                                   wcol + (size_t)max(ridx[j], 0) * row_bytes);
+                }
+                cp_async_commit();
+            }
+            // This lane's four A chunks of slot `warp` (stage-relative) and its B
+            // element (lanes 0..15: batch column = lane).
+            uint32_t aoff[4];
+    #pragma unroll
+            for (int j = 0; j < 4; ++j)
+                aoff[j] = a_chunk_off(lane, j, warp);
+            const uint32_t boff = b_elem_off(lane & 15, warp);
+
+            // Zero points of this lane's 32 outputs for one group, as subnormal
+            // fp16 pairs matching the AND results: word j, pairs = outputs
+            // (8j, 8j+4), (8j+1, 8j+5) << 4, (8j+2, 8j+6), (8j+3, 8j+7) << 4.
+            uint4 zraw[8];
+            auto load_sz = [&](int G) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(p.sz + (size_t)G * p.N + n0 +
+                                                                   (lane_ok ? lane * 32 : 0));
+    #pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    zraw[c] = __ldg(src + c);
+            };
+            uint32_t zc[4][4];
+            auto unpack_z = [&]() {
+    #pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t w[8] = {zraw[2 * j].x,     zraw[2 * j].y,     zraw[2 * j].z,
+                                           zraw[2 * j].w,     zraw[2 * j + 1].x, zraw[2 * j + 1].y,
+                                           zraw[2 * j + 1].z, zraw[2 * j + 1].w};
+                    uint32_t z[8];
+    #pragma unroll
+                    for (int o = 0; o < 8; ++o)
+                        z[o] = lane_ok ? zero_of(w[o]) : 0u;
+                    zc[j][0] = z[0] | (z[4] << 16);
+                    zc[j][1] = (z[1] | (z[5] << 16)) << 4;
+                    zc[j][2] = z[2] | (z[6] << 16);
+                    zc[j][3] = (z[3] | (z[7] << 16)) << 4;
+                }
+            };
+            // Fold outputs of this thread: its tensor-memory lane (quadrant
+            // warp % 4) in M-blocks 2 (warp / 4) and 2 (warp / 4) + 1.
+            const int mbA = 2 * (warp >> 2);
+            const uint32_t tlane = (uint32_t)(32 * (warp & 3)) << 16;
+            int fout[2];
+    #pragma unroll
+            for (int i = 0; i < 2; ++i)
+                fout[i] = mma_out_of_slot(128 * (mbA + i) + 32 * (warp & 3) + lane);
+            // (s, z) words of the fold outputs for a group, kept raw until the fold
+            // so that the loads stay in flight.
+            uint32_t sfold[2], snew[2];
+            auto load_s = [&](int G, uint32_t *sv) {
+    #pragma unroll
+                for (int i = 0; i < 2; ++i)
+                    sv[i] = (fout[i] < nvalid_out) ? __ldg(p.sz + (size_t)G * p.N + n0 + fout[i]) : 0u;
+            };
+            if (nruns > 0) {
+                load_sz(grp(rstart[0]));
+                load_s(grp(rstart[0]), snew);
+            }
+
+            // totals += s 2^c D for run r's accumulators (set r & 1); the totals
+            // stay in tensor memory (columns kTotCol..), written by run 0.
+            auto fold = [&](int r) { // r: run of this segment
+                const int rg = run_base + r;
+                ok = mbar_wait(bar_ready + (rg & 1), (uint32_t)((rg >> 1) & 1), ok);
+                tc_fence_after();
+    #pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    float d[kMmaN], t[kMmaN];
+                    tmem_ld16(tmem + tlane + 128 * (rg & 1) + kMmaN * (mbA + i), d);
+                    const float f = __half2float(__ushort_as_half((uint16_t)(sfold[i] & 0xffffu))) *
+                                    ((fout[i] & 1) ? 1048576.f : 16777216.f);
+                    if (r == 0) {
+    #pragma unroll
+                        for (int c = 0; c < kMmaN; ++c)
+                            t[c] = f * d[c];
+                    } else {
+                        tmem_ld16(tmem + tlane + kTotCol + kMmaN * (mbA + i), t);
+    #pragma unroll
+                        for (int c = 0; c < kMmaN; ++c)
+                            t[c] = fmaf(f, d[c], t[c]);
+                    }
+                    tmem_st16(tmem + tlane + kTotCol + kMmaN * (mbA + i), t);
+                }
+                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(bar_free + (rg & 1));
+            };
+
+            // every batch row's x' (written by its warp above) is in place
+            asm volatile("bar.sync 1, %0;" ::"n"(kEx) : "memory");
+
             int run = 0;
             for (int kb = 0; kb < nkb; ++kb) {
                 kb_run(kb, run);
-                const bool first = kb == rkb[run], last = kb == rkb[run + 1] - 1;
-                const int s = kb % nst;
-                ok = mbar_wait(bar_full + s, (uint32_t)((kb / nst) & 1), ok);
-                tc_fence_after();
-                if (first && run >= 2) {
-                    ok = mbar_wait(bar_free + (run & 1), (uint32_t)(((run >> 1) - 1) & 1), ok);
-                    tc_fence_after();
+                const int kg = kb_base + kb;
+                const int s = kg % nst;
+                const int j0 = rstart[run] + kKb * (kb - rkb[run]);
+                const bool valid = warp < rstart[run + 1] - j0;
+                const bool first = kb == rkb[run];
+                if (first) {
+                    unpack_z(); // this run's zero points (loaded a run ahead)
+                    if (run + 1 < nruns)
+                        load_sz(grp(rstart[run + 1]));
                 }
+                // The stage's previous K-block has been multiplied.
+                if (kg >= nst)
+                    ok = mbar_wait(bar_empty + s, (uint32_t)((kg / nst - 1) & 1), ok);
                 const uint32_t a_st = sA + (uint32_t)(s * kAStage);
-                const uint32_t dcol = tmem + (uint32_t)(128 * (run & 1));
-                const uint64_t bdesc = smem_desc(sB + (uint32_t)(s * kBStage), 128, 256, 0);
-                // Every M-block: a lane's outputs are spread over the M-blocks
-                // (lanes past N hold finite codes of column 0 and are dropped
-                // in the epilogue).
-#pragma unroll
-                for (int mb = 0; mb < kMBlocks; ++mb)
-                    mma_f16(dcol + (uint32_t)(kMmaN * mb),
-                            smem_desc(a_st + (uint32_t)(mb * 2048), 1024, 16 * 1024, 2), bdesc,
-                            !first);
-                mma_commit(bar_empty + s);
-                if (last && !(p.debug_withhold_ready && run == nruns - 1))
-                    mma_commit(bar_ready + (run & 1));
-            }
-            // every MMA of this CTA has completed when bar_done's phase 0 does
-            mma_commit(&bar_done);
-            // (the tensor memory is freed only after that, below)
-            ok = mbar_wait(&bar_done, 0u, true) && ok;
-        }
-        __syncwarp();
-    } else {
-        // ---- the expanding warps ---------------------------------------------
-        // Warp w expands slot w of every K-block: its row stream is one row
-        // per K-block, through a per-lane ring kMRing K-blocks ahead (with its
-        // own run pointer).
-        constexpr int kEx = kMWarps * 32; // threads of the expanding warps
-        // x' = x 2^S_b in fp16 per batch row b, 2^14 <= max |x'| < 2^15 over
-        // the CTA's rows (as in the batch-1 kernel), staged batch-major in
-        // rxh. Warp w owns batch row b = w: each lane gathers chunks of 8 rows
-        // (one 16-byte load when the 8 rows are 8 consecutive aligned
-        // channels), four chunks in flight, before any weight row is
-        // requested; the warp reduces max |x|, then converts its row in place.
-        const int rs = rxh_stride(kp.rows_cap);
-        if (warp < p.B) {
-            const int b = warp;
-            uint16_t *xr = rxh + (size_t)b * rs;
-            const uint16_t *xb = p.x + (size_t)b * p.K;
-            const int nch = (nr + 7) / 8;
-            float m = 0.f;
-            for (int c0 = lane; c0 < nch; c0 += 4 * 32) {
-                uint4 v[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int c = c0 + 32 * u;
-                    v[u] = make_uint4(0u, 0u, 0u, 0u);
-                    if (c < nch) {
-                        const int j0 = 8 * c;
-                        const int k0 = ridx[j0];
-                        bool vec = (j0 + 8 <= nr) && k0 >= 0 && (k0 & 7) == 0;
-#pragma unroll
-                        for (int i = 1; i < 8; ++i)
-                            vec = vec && (ridx[min(j0 + i, nr - 1)] == k0 + i);
-                        if (vec) {
-                            v[u] = __ldg(reinterpret_cast<const uint4 *>(xb + k0));
-                        } else {
-                            uint32_t h[8];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                const int k = (j0 + i < nr) ? ridx[j0 + i] : -1;
-                                h[i] = (k >= 0) ? (uint32_t)__ldg(xb + k) : 0u;
-                            }
-                            v[u] = make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16),
-                                              h[4] | (h[5] << 16), h[6] | (h[7] << 16));
-                        }
+                cp_async_wait<kMRing - 1>();
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (valid)
+                    v = *reinterpret_cast<const uint4 *>(myring + (kb % kMRing) * kRowBytes1);
+                // refill the ring slot with this warp's row kMRing K-blocks ahead
+                if (kb + kMRing < nkb) {
+                    const int j = kb_row(kb + kMRing);
+                    if (j >= 0)
+                        cp_async16(myring + (kb % kMRing) * kRowBytes1,
+                                   wcol + (size_t)max(ridx[j], 0) * row_bytes);
+                }
+                cp_async_commit();
+                const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+    #pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint32_t t0 = 0u, t1 = 0u, t2 = 0u, t3 = 0u;
+                    if (valid) {
+                        const uint32_t w = wv[j], w8 = w >> 8;
+                        t0 = hsub2(w & 0x000F000Fu, zc[j][0]);
+                        t1 = hsub2(w & 0x00F000F0u, zc[j][1]);
+                        t2 = hsub2(w8 & 0x000F000Fu, zc[j][2]);
+                        t3 = hsub2(w8 & 0x00F000F0u, zc[j][3]);
                     }
+                    st_shared_v4(a_st + aoff[j], t0, t1, t2, t3);
                 }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int c = c0 + 32 * u;
-                    if (c < nch) {
-                        *reinterpret_cast<uint4 *>(xr + 8 * c) = v[u];
-                        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            m = fmaxf(m, fabsf(bf16_bits_to_float(
-                                             (uint16_t)(w[i >> 1] >> (16 * (i & 1))))));
-                    }
+                if (lane < kMmaN) {
+                    // B operand: x' of slot `warp` for batch column `lane`.
+                    const uint16_t xv =
+                        (valid && lane < p.B) ? rxh[(size_t)lane * rs + j0 + warp] : (uint16_t)0;
+                    asm volatile("st.shared.u16 [%0], %1;" ::"r"(sB + (uint32_t)(s * kBStage) + boff),
+                                 "h"(xv)
+                                 : "memory");
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(bar_full + s);
+
+                // The previous run ended with the previous K-block: fold it now,
+                // while this K-block is being multiplied.
+                if (first && run > 0) {
+    #pragma unroll
+                    for (int i = 0; i < 2; ++i)
+                        sfold[i] = snew[i];
+                    load_s(grp(rstart[run]), snew); // this run's scales, for its fold
+                    fold(run - 1);
                 }
             }
-            const int e = warp_max_exponent(m);
-            const int S = (e == INT32_MIN) ? 0 : 14 - e;
-            if (lane == 0)
-                s_S[b] = S;
-            const float fa = pow2f(S - S / 2), fb = pow2f(S / 2);
-            __syncwarp();
-            for (int c = lane; c < nch; c += 32) {
-                uint4 v = *reinterpret_cast<const uint4 *>(xr + 8 * c);
-                uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t lo = __half_as_ushort(__float2half_rn(
-                        (bf16_bits_to_float((uint16_t)(w[i] & 0xffffu)) * fa) * fb));
-                    const uint32_t hi = __half_as_ushort(__float2half_rn(
-                        (bf16_bits_to_float((uint16_t)(w[i] >> 16)) * fa) * fb));
-                    w[i] = lo | (hi << 16);
-                }
-                *reinterpret_cast<uint4 *>(xr + 8 * c) = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-        }
-
-        const size_t row_bytes = (size_t)(p.N / 2);
-        const uint8_t *wcol = p.qweight + (lane_ok ? ((size_t)n0 / 2 + lane * 16) : 0);
-        uint8_t *myring = ring + (size_t)warp * kMRing * kRowBytes1 + lane * 16;
-        int ring_run = 0;
-        auto kb_row = [&](int kb) -> int { // ridx position of this warp's slot, or -1
-            kb_run(kb, ring_run);
-            const int j = rstart[ring_run] + kKb * (kb - rkb[ring_run]) + warp;
-            return (j < rstart[ring_run + 1]) ? j : -1;
-        };
-#pragma unroll
-        for (int i = 0; i < kMRing; ++i) {
-            if (i < nkb) {
-                const int j = kb_row(i);
-                if (j >= 0)
-                    cp_async16(myring + i * kRowBytes1,
-                               wcol + (size_t)max(ridx[j], 0) * row_bytes);
-            }
-            cp_async_commit();
-        }
-        // This lane's four A chunks of slot `warp` (stage-relative) and its B
-        // element (lanes 0..15: batch column = lane).
-        uint32_t aoff[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-            aoff[j] = a_chunk_off(lane, j, warp);
-        const uint32_t boff = b_elem_off(lane & 15, warp);
-
-        // Zero points of this lane's 32 outputs for one group, as subnormal
-        // fp16 pairs matching the AND results: word j, pairs = outputs
-        // (8j, 8j+4), (8j+1, 8j+5) << 4, (8j+2, 8j+6), (8j+3, 8j+7) << 4.
-        uint4 zraw[8];
-        auto load_sz = [&](int G) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(p.sz + (size_t)G * p.N + n0 +
-                                                               (lane_ok ? lane * 32 : 0));
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                zraw[c] = __ldg(src + c);
-        };
-        uint32_t zc[4][4];
-        auto unpack_z = [&]() {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const uint32_t w[8] = {zraw[2 * j].x,     zraw[2 * j].y,     zraw[2 * j].z,
-                                       zraw[2 * j].w,     zraw[2 * j + 1].x, zraw[2 * j + 1].y,
-                                       zraw[2 * j + 1].z, zraw[2 * j + 1].w};
-                uint32_t z[8];
-#pragma unroll
-                for (int o = 0; o < 8; ++o)
-                    z[o] = lane_ok ? zero_of(w[o]) : 0u;
-                zc[j][0] = z[0] | (z[4] << 16);
-                zc[j][1] = (z[1] | (z[5] << 16)) << 4;
-                zc[j][2] = z[2] | (z[6] << 16);
-                zc[j][3] = (z[3] | (z[7] << 16)) << 4;
-            }
-        };
-        // Fold outputs of this thread: its tensor-memory lane (quadrant
-        // warp % 4) in M-blocks 2 (warp / 4) and 2 (warp / 4) + 1.
-        const int mbA = 2 * (warp >> 2);
-        const uint32_t tlane = (uint32_t)(32 * (warp & 3)) << 16;
-        int fout[2];
-#pragma unroll
-        for (int i = 0; i < 2; ++i)
-            fout[i] = mma_out_of_slot(128 * (mbA + i) + 32 * (warp & 3) + lane);
-        // (s, z) words of the fold outputs for a group, kept raw until the fold
-        // so that the loads stay in flight.
-        uint32_t sfold[2], snew[2];
-        auto load_s = [&](int G, uint32_t *sv) {
-#pragma unroll
-            for (int i = 0; i < 2; ++i)
-                sv[i] = (fout[i] < nvalid_out) ? __ldg(p.sz + (size_t)G * p.N + n0 + fout[i]) : 0u;
-        };
-        if (nruns > 0) {
-            load_sz(grp(rstart[0]));
-            load_s(grp(rstart[0]), snew);
-        }
-
-        // totals += s 2^c D for run r's accumulators (set r & 1); the totals
-        // stay in tensor memory (columns kTotCol..), written by run 0.
-        auto fold = [&](int r) {
-            ok = mbar_wait(bar_ready + (r & 1), (uint32_t)((r >> 1) & 1), ok);
-            tc_fence_after();
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                float d[kMmaN], t[kMmaN];
-                tmem_ld16(tmem + tlane + 128 * (r & 1) + kMmaN * (mbA + i), d);
-                const float f = __half2float(__ushort_as_half((uint16_t)(sfold[i] & 0xffffu))) *
-                                ((fout[i] & 1) ? 1048576.f : 16777216.f);
-                if (r == 0) {
-#pragma unroll
-                    for (int c = 0; c < kMmaN; ++c)
-                        t[c] = f * d[c];
-                } else {
-                    tmem_ld16(tmem + tlane + kTotCol + kMmaN * (mbA + i), t);
-#pragma unroll
-                    for (int c = 0; c < kMmaN; ++c)
-                        t[c] = fmaf(f, d[c], t[c]);
-                }
-                tmem_st16(tmem + tlane + kTotCol + kMmaN * (mbA + i), t);
-            }
-            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(bar_free + (r & 1));
-        };
-
-        // every batch row's x' (written by its warp above) is in place
-        asm volatile("bar.sync 1, %0;" ::"n"(kEx) : "memory");
-
-        int run = 0;
-        for (int kb = 0; kb < nkb; ++kb) {
-            kb_run(kb, run);
-            const int s = kb % nst;
-            const int j0 = rstart[run] + kKb * (kb - rkb[run]);
-            const bool valid = warp < rstart[run + 1] - j0;
-            const bool first = kb == rkb[run];
-            if (first) {
-                unpack_z(); // this run's zero points (loaded a run ahead)
-                if (run + 1 < nruns)
-                    load_sz(grp(rstart[run + 1]));
-            }
-            // The stage's previous K-block has been multiplied.
-            if (kb >= nst)
-                ok = mbar_wait(bar_empty + s, (uint32_t)((kb / nst - 1) & 1), ok);
-            const uint32_t a_st = sA + (uint32_t)(s * kAStage);
-            cp_async_wait<kMRing - 1>();
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (valid)
-                v = *reinterpret_cast<const uint4 *>(myring + (kb % kMRing) * kRowBytes1);
-            // refill the ring slot with this warp's row kMRing K-blocks ahead
-            if (kb + kMRing < nkb) {
-                const int j = kb_row(kb + kMRing);
-                if (j >= 0)
-                    cp_async16(myring + (kb % kMRing) * kRowBytes1,
-                               wcol + (size_t)max(ridx[j], 0) * row_bytes);
-            }
-            cp_async_commit();
-            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                uint32_t t0 = 0u, t1 = 0u, t2 = 0u, t3 = 0u;
-                if (valid) {
-                    const uint32_t w = wv[j], w8 = w >> 8;
-                    t0 = hsub2(w & 0x000F000Fu, zc[j][0]);
-                    t1 = hsub2(w & 0x00F000F0u, zc[j][1]);
-                    t2 = hsub2(w8 & 0x000F000Fu, zc[j][2]);
-                    t3 = hsub2(w8 & 0x00F000F0u, zc[j][3]);
-                }
-                st_shared_v4(a_st + aoff[j], t0, t1, t2, t3);
-            }
-            if (lane < kMmaN) {
-                // B operand: x' of slot `warp` for batch column `lane`.
-                const uint16_t xv =
-                    (valid && lane < p.B) ? rxh[(size_t)lane * rs + j0 + warp] : (uint16_t)0;
-                asm volatile("st.shared.u16 [%0], %1;" ::"r"(sB + (uint32_t)(s * kBStage) + boff),
-                             "h"(xv)
-                             : "memory");
-            }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(bar_full + s);
-
-            // The previous run ended with the previous K-block: fold it now,
-            // while this K-block is being multiplied.
-            if (first && run > 0) {
-#pragma unroll
+            if (nruns > 0) {
+    #pragma unroll
                 for (int i = 0; i < 2; ++i)
                     sfold[i] = snew[i];
-                load_s(grp(rstart[run]), snew); // this run's scales, for its fold
-                fold(run - 1);
+                fold(nruns - 1);
             }
-        }
-        if (nruns > 0) {
-#pragma unroll
-            for (int i = 0; i < 2; ++i)
-                sfold[i] = snew[i];
-            fold(nruns - 1);
-        }
-        cp_async_wait_all();
+            cp_async_wait_all();
 
-        // Split-K partials from the totals, back in real units (x 2^-S_b,
-        // two exact factors).
-        if (nkb > 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                float t[kMmaN];
-                tmem_ld16(tmem + tlane + kTotCol + kMmaN * (mbA + i), t);
-                if (fout[i] < nvalid_out) {
-#pragma unroll
-                    for (int c = 0; c < kMmaN; ++c) {
-                        if (c < p.B) {
-                            const int E = -s_S[c];
-                            atomicAdd(p.ws_acc + (size_t)c * p.N + n0 + fout[i],
-                                      (t[c] * pow2f(E / 2)) * pow2f(E - E / 2));
+            // Split-K partials from the totals, back in real units (x 2^-S_b,
+            // two exact factors).
+            if (nkb > 0) {
+                tc_fence_after();
+    #pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    float t[kMmaN];
+                    tmem_ld16(tmem + tlane + kTotCol + kMmaN * (mbA + i), t);
+                    if (fout[i] < nvalid_out) {
+    #pragma unroll
+                        for (int c = 0; c < kMmaN; ++c) {
+                            if (c < p.B) {
+                                const int E = -s_S[c];
+                                atomicAdd(p.ws_acc + (size_t)c * p.N + n0 + fout[i],
+                                          (t[c] * pow2f(E / 2)) * pow2f(E - E / 2));
+                            }
                         }
                     }
                 }
             }
         }
+        kb_base += nkb;
+        run_base += nruns;
+    }
+    if (warp == kIssuer && lane == 0) {
+        // every MMA of this CTA has completed when bar_done's phase 0 does
+        // (the tensor memory is freed only after that, below)
+        mma_commit(&bar_done);
+        ok = mbar_wait(&bar_done, 0u, true) && ok;
     }
     if (!ok)
         set_status(p.status, SGQ_STATUS_TIMEOUT);
@@ -735,11 +826,24 @@ cudaError_t launch_mma_t(KParams kp, int num_sms, cudaStream_t stream)
     kp.nb = 1;
     kp.bp = pad_batch(p.B);
     kp.n_tiles = ceil_div(p.N, kTileN1);
-    kp.k_splits = std::max(1, num_sms / kp.n_tiles);
+    kp.k_splits = 1; // unused: the grid shares the (tile, row) space evenly
     kp.span_cap = 0;
+    // Each CTA an equal share of n_tiles x K/8 units of 8 rows; a segment
+    // holds at most one share's rows. When a whole number of shares per tile
+    // fills at least 90% of the SMs, shares stay inside tiles (a CTA that
+    // spans two tiles pays the prologue and the tail twice, and the slowest
+    // CTA sets the time); otherwise one share per SM. More CTAs (waves) only
+    // if a share's rows do not fit shared memory.
+    const long long units = (long long)kp.n_tiles * (p.K / 8);
+    if ((long long)kp.n_tiles * p.K >= (1ll << 31))
+        return cudaErrorInvalidValue; // the kernel's work units are 32-bit
+    int grid = num_sms;
+    if (kp.n_tiles <= num_sms && 10 * kp.n_tiles * (num_sms / kp.n_tiles) >= 9 * num_sms)
+        grid = kp.n_tiles * (num_sms / kp.n_tiles);
     SmemM L;
     for (;;) {
-        kp.rows_cap = ceil_div(p.K, kp.k_splits) + 8;
+        kp.rows_cap = (int)(8 * ((units + grid - 1) / grid + 1) + 8);
+        kp.rows_cap = std::min(kp.rows_cap, p.K + 8);
         // the most operand stages that fit, at least two
         kp.stages = kMaxStages;
         L = smemm_layout(kp.rows_cap, kp.stages, kp.bp);
@@ -747,15 +851,14 @@ cudaError_t launch_mma_t(KParams kp, int num_sms, cudaStream_t stream)
             --kp.stages;
             L = smemm_layout(kp.rows_cap, kp.stages, kp.bp);
         }
-        if (L.total + 1024 <= kMaxSmem || kp.k_splits >= p.K / 8)
+        if (L.total + 1024 <= kMaxSmem || (long long)grid >= units)
             break;
-        kp.k_splits *= 2;
+        grid *= 2;
     }
     if (L.total + 1024 > kMaxSmem)
         return cudaErrorInvalidConfiguration;
     const size_t smem = std::max(L.total + 1024, kOneCtaSmem);
-    cudaError_t err = launch_pdl(gemv_mma_kernel<SRC>, kp.n_tiles * kp.k_splits, kMThreads,
-                                 smem, stream, kp);
+    cudaError_t err = launch_pdl(gemv_mma_kernel<SRC>, grid, kMThreads, smem, stream, kp);
     if (err != cudaSuccess || p.accumulate)
         return err;
     return launch_finalize(p, stream);
