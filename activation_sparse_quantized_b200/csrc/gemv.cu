@@ -270,7 +270,11 @@ __device__ __forceinline__ int part_chunk16(int l, int c)
 // NM: the 2:4 layout (batch 1): the codes of a row are the kept outputs'
 // slots, 1024 slots = 2048 outputs per tile, 64 outputs per lane; the fold
 // adds each slot's sum to its output through the group's keep nibbles.
-template <int SRC, int BW, bool NM = false>
+// SEG (index list only): instead of (tile, split) from the block index, the
+// CTA takes an equal share of the (tile, list entry) space, which may end one
+// tile and start the next; each part (segment) runs the whole body in turn,
+// adding into the workspace.
+template <int SRC, int BW, bool NM = false, bool SEG = false>
 __global__ void __launch_bounds__(kThreads1, 1) gemv_kernel(const KParams kp)
 {
     static_assert(!NM || BW == 1, "the 2:4 layout is batch 1 only");
@@ -289,341 +293,371 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_kernel(const KParams kp)
     const int rcap = kp.rows_cap;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int tile = blockIdx.x % kp.n_tiles;
-    const int split = blockIdx.x / kp.n_tiles;
-    const int n0 = tile * TO;           // first output of the tile
-    const int s0 = tile * kTileN1;      // first code slot of the tile
-    const int SN = NM ? p.N / 2 : p.N;  // code slots (and (s, z) pairs) per row and group
-    const int lg = kp.lg;
-    const size_t row_stride = (size_t)(SN / 2);
-    const bool lane_ok = (n0 + lane * OPL) < p.N;
-
-    grid_launch_dependents();
-
-    // Scale/zero of the CTA's groups, staged asynchronously (the oldest
-    // cp.async group of every thread). With a fixed channel slice (threshold /
-    // mask / dense) the groups are known now, so the copies start before
-    // waiting on the previous kernel; with an index list they follow the list.
-    int G0 = 0, span = 0;
-    auto stage_sz = [&]() {
-        for (int c = tid; c < span * (kTileN1 / 4); c += kThreads1) {
-            const int g = c >> 8, q = c & 255; // q: chunk of 4 slots in the tile
-            if (s0 + 4 * q < SN)
-                cp_async16(smem + L.szs + ((size_t)g * 256 + part_chunk(q >> 3, q & 7)) * 16,
-                           p.sz + (size_t)(G0 + g) * SN + s0 + 4 * q);
-        }
-        cp_async_commit();
-    };
-    if (SRC != ROWS_LIST) {
-        int c0, c1;
-        if (SRC == ROWS_THRESH || SRC == ROWS_MASK || SRC == ROWS_GLU) {
-            channel_slice(kp, split, c0, c1);
+    // (tile, split), or with SEG the CTA's share of the list over the tiles
+    int su = 0, su1 = 1, per_tile = 1;
+    if constexpr (SEG) {
+        grid_launch_dependents();
+        grid_dependency_wait(); // x, idx, count may come from the previous kernel
+        const int c = __ldg(p.count);
+        per_tile = c < 0 ? 0 : (c > p.K ? p.K : c);
+        if (per_tile != c && tid == 0 && blockIdx.x == 0)
+            set_status(p.status, SGQ_STATUS_BAD_COUNT);
+        const long long W = (long long)kp.n_tiles * per_tile;
+        su = (int)(W * blockIdx.x / gridDim.x);
+        su1 = (int)(W * (blockIdx.x + 1) / gridDim.x);
+    }
+    while (su < su1) {
+        int tile, split = 0, seg_lo = 0, seg_hi = 0;
+        if constexpr (SEG) {
+            tile = su / per_tile;
+            seg_lo = su - tile * per_tile;
+            seg_hi = min(per_tile, su1 - tile * per_tile);
+            su = tile * per_tile + seg_hi;
+            __syncthreads(); // the previous segment is done with shared memory
         } else {
-            c0 = (int)((long long)p.K * split / kp.k_splits);
-            c1 = (int)((long long)p.K * (split + 1) / kp.k_splits);
+            tile = blockIdx.x % kp.n_tiles;
+            split = blockIdx.x / kp.n_tiles;
+            su = su1;
         }
-        if (c1 > c0) {
-            G0 = c0 >> lg;
-            span = min(((c1 - 1) >> lg) - G0 + 1, kp.span_cap);
+        (void)seg_lo;
+        (void)seg_hi;
+        const int n0 = tile * TO;           // first output of the tile
+        const int s0 = tile * kTileN1;      // first code slot of the tile
+        const int SN = NM ? p.N / 2 : p.N;  // code slots (and (s, z) pairs) per row and group
+        const int lg = kp.lg;
+        const size_t row_stride = (size_t)(SN / 2);
+        const bool lane_ok = (n0 + lane * OPL) < p.N;
+
+        if constexpr (!SEG)
+            grid_launch_dependents();
+
+        // Scale/zero of the CTA's groups, staged asynchronously (the oldest
+        // cp.async group of every thread). With a fixed channel slice (threshold /
+        // mask / dense) the groups are known now, so the copies start before
+        // waiting on the previous kernel; with an index list they follow the list.
+        int G0 = 0, span = 0;
+        auto stage_sz = [&]() {
+            for (int c = tid; c < span * (kTileN1 / 4); c += kThreads1) {
+                const int g = c >> 8, q = c & 255; // q: chunk of 4 slots in the tile
+                if (s0 + 4 * q < SN)
+                    cp_async16(smem + L.szs + ((size_t)g * 256 + part_chunk(q >> 3, q & 7)) * 16,
+                               p.sz + (size_t)(G0 + g) * SN + s0 + 4 * q);
+            }
+            cp_async_commit();
+        };
+        if (SRC != ROWS_LIST) {
+            int c0, c1;
+            if (SRC == ROWS_THRESH || SRC == ROWS_MASK || SRC == ROWS_GLU) {
+                channel_slice(kp, split, c0, c1);
+            } else {
+                c0 = (int)((long long)p.K * split / kp.k_splits);
+                c1 = (int)((long long)p.K * (split + 1) / kp.k_splits);
+            }
+            if (c1 > c0) {
+                G0 = c0 >> lg;
+                span = min(((c1 - 1) >> lg) - G0 + 1, kp.span_cap);
+            }
+            stage_sz();
         }
-        stage_sz();
-    }
 
-    grid_dependency_wait(); // x, idx, count, mask may come from the previous kernel
+        if constexpr (!SEG)
+            grid_dependency_wait(); // x, idx, count, mask may come from the previous kernel
 
-    // Rows (build_rows ends with a barrier). Invalid list entries stay -1: they
-    // are read as row 0 with x = 0, so they add nothing.
-    const int nr = build_rows<SRC, kThreads1, (BW == 1)>(kp, split, ridx, rx, scan,
-                                                         reinterpret_cast<float *>(smem + L.xs),
-                                                         tile == 0);
-    auto row = [&](int j) { return (SRC == ROWS_LIST) ? max(ridx[j], 0) : ridx[j]; };
+        // Rows (build_rows ends with a barrier). Invalid list entries stay -1: they
+        // are read as row 0 with x = 0, so they add nothing.
+        const int nr = build_rows<SRC, kThreads1, (BW == 1)>(
+            kp, split, ridx, rx, scan, reinterpret_cast<float *>(smem + L.xs), tile == 0,
+            SEG ? seg_lo : -1, SEG ? seg_hi : -1);
+        auto row = [&](int j) { return (SRC == ROWS_LIST) ? max(ridx[j], 0) : ridx[j]; };
 
-    if (SRC == ROWS_LIST) {
-        if (nr > 0) {
-            const int kf = row(0), kl = row(nr - 1);
-            G0 = kf >> lg;
-            span = min(max((kl >> lg) - G0 + 1, 1), kp.span_cap);
+        if (SRC == ROWS_LIST) {
+            if (nr > 0) {
+                const int kf = row(0), kl = row(nr - 1);
+                G0 = kf >> lg;
+                span = min(max((kl >> lg) - G0 + 1, 1), kp.span_cap);
+            }
+            stage_sz(); // stays the oldest cp.async group
         }
-        stage_sz(); // stays the oldest cp.async group
-    }
 
-    // This warp's batch rows and its contiguous slice of the CTA's rows.
-    const int wpg = (BW == 1) ? kWarps1 : kWarps1 / kp.nb;
-    const int b0 = (BW == 1) ? 0 : (warp / wpg) * BW;
-    const int wq = (BW == 1) ? warp : warp % wpg;
-    const int nbw = (BW == 1) ? 1 : max(0, min(BW, p.B - b0)); // real batch rows of this warp
-    const int wa = (int)((long long)nr * wq / wpg);
-    const int n = (nbw > 0) ? (int)((long long)nr * (wq + 1) / wpg) - wa : 0;
+        // This warp's batch rows and its contiguous slice of the CTA's rows.
+        const int wpg = (BW == 1) ? kWarps1 : kWarps1 / kp.nb;
+        const int b0 = (BW == 1) ? 0 : (warp / wpg) * BW;
+        const int wq = (BW == 1) ? warp : warp % wpg;
+        const int nbw = (BW == 1) ? 1 : max(0, min(BW, p.B - b0)); // real batch rows of this warp
+        const int wa = (int)((long long)nr * wq / wpg);
+        const int n = (nbw > 0) ? (int)((long long)nr * (wq + 1) / wpg) - wa : 0;
 
-    // Ring prologue. Lanes past N read column 0 (valid memory, result unused).
-    const uint8_t *wcol = p.qweight + (lane_ok ? ((size_t)s0 / 2 + lane * 16) : 0);
-    uint8_t *region = ring + (size_t)warp * warp_region_bytes(BW, NM);
-    uint8_t *myring = region + lane * 16;
-#pragma unroll
-    for (int s = 0; s < kStages1; ++s) {
-        if (s < n)
-            cp_async16(myring + s * kRowBytes1, wcol + (size_t)row(wa + s) * row_stride);
-        cp_async_commit();
-    }
+        // Ring prologue. Lanes past N read column 0 (valid memory, result unused).
+        const uint8_t *wcol = p.qweight + (lane_ok ? ((size_t)s0 / 2 + lane * 16) : 0);
+        uint8_t *region = ring + (size_t)warp * warp_region_bytes(BW, NM);
+        uint8_t *myring = region + lane * 16;
+    #pragma unroll
+        for (int s = 0; s < kStages1; ++s) {
+            if (s < n)
+                cp_async16(myring + s * kRowBytes1, wcol + (size_t)row(wa + s) * row_stride);
+            cp_async_commit();
+        }
 
-    // x of this warp's rows and batch rows (after the weights are in flight),
-    // unless build_rows already read it (threshold; bitmask at batch 1).
-    // Padded batch rows and invalid list entries get x = 0.
-    if (!(SRC == ROWS_THRESH || SRC == ROWS_GLU || (SRC == ROWS_MASK && BW == 1))) {
-        for (int e = lane; e < n * BW; e += 32) {
-            const int j = e / BW, bb = e - j * BW;
-            const int k = ridx[wa + j];
-            rx[(b0 + bb) * rcap + wa + j] =
-                (k >= 0 && bb < nbw) ? bf16_bits_to_float(__ldg(p.x + (size_t)(b0 + bb) * p.K + k))
-                                     : 0.f;
+        // x of this warp's rows and batch rows (after the weights are in flight),
+        // unless build_rows already read it (threshold; bitmask at batch 1).
+        // Padded batch rows and invalid list entries get x = 0.
+        if (!(SRC == ROWS_THRESH || SRC == ROWS_GLU || (SRC == ROWS_MASK && BW == 1))) {
+            for (int e = lane; e < n * BW; e += 32) {
+                const int j = e / BW, bb = e - j * BW;
+                const int k = ridx[wa + j];
+                rx[(b0 + bb) * rcap + wa + j] =
+                    (k >= 0 && bb < nbw) ? bf16_bits_to_float(__ldg(p.x + (size_t)(b0 + bb) * p.K + k))
+                                         : 0.f;
+            }
+            __syncwarp();
+        }
+
+        // Per batch row: x' = x 2^S in fp16 with 2^14 <= max |x'| < 2^15 over the
+        // warp's rows: exact for every |x| >= 2^-28 max |x| (fp16 normals);
+        // smaller x round on the fp16 subnormal grid, an error below
+        // 2^-39 max |x'|. Each product q 2^-24 x' (or q 2^-20 x') is then exact in
+        // fp32.
+        int S[BW];
+    #pragma unroll
+        for (int bb = 0; bb < BW; ++bb) {
+            const float *xr = rx + (b0 + bb) * rcap;
+            uint16_t *hr = rxh + (b0 + bb) * rcap;
+            float m = 0.f;
+            for (int j = lane; j < n; j += 32)
+                m = fmaxf(m, fabsf(xr[wa + j]));
+            const int e = warp_max_exponent(m);
+            S[bb] = (e == INT32_MIN) ? 0 : 14 - e;
+            const float fa = pow2f(S[bb] - S[bb] / 2), fb = pow2f(S[bb] / 2);
+            for (int j = lane; j < n; j += 32)
+                hr[wa + j] = __half_as_ushort(__float2half_rn((xr[wa + j] * fa) * fb));
         }
         __syncwarp();
-    }
+        // The staged scale/zero (every thread's oldest cp.async group) have landed
+        // and are visible to every warp before the first fold.
+        cp_async_wait<kStages1>();
+        __syncthreads();
 
-    // Per batch row: x' = x 2^S in fp16 with 2^14 <= max |x'| < 2^15 over the
-    // warp's rows: exact for every |x| >= 2^-28 max |x| (fp16 normals);
-    // smaller x round on the fp16 subnormal grid, an error below
-    // 2^-39 max |x'|. Each product q 2^-24 x' (or q 2^-20 x') is then exact in
-    // fp32.
-    int S[BW];
-#pragma unroll
-    for (int bb = 0; bb < BW; ++bb) {
-        const float *xr = rx + (b0 + bb) * rcap;
-        uint16_t *hr = rxh + (b0 + bb) * rcap;
-        float m = 0.f;
-        for (int j = lane; j < n; j += 32)
-            m = fmaxf(m, fabsf(xr[wa + j]));
-        const int e = warp_max_exponent(m);
-        S[bb] = (e == INT32_MIN) ? 0 : 14 - e;
-        const float fa = pow2f(S[bb] - S[bb] / 2), fb = pow2f(S[bb] / 2);
-        for (int j = lane; j < n; j += 32)
-            hr[wa + j] = __half_as_ushort(__float2half_rn((xr[wa + j] * fa) * fb));
-    }
-    __syncwarp();
-    // The staged scale/zero (every thread's oldest cp.async group) have landed
-    // and are visible to every warp before the first fold.
-    cp_async_wait<kStages1>();
-    __syncthreads();
-
-    // accg[bb][o] = this group's sum of q x' 2^-code_shift(o) for code slot o;
-    // acc[bb][o] = folded result of output o in units of 2^-S.
-    float accg[BW][32], acc[BW][OPL];
-#pragma unroll
-    for (int bb = 0; bb < BW; ++bb) {
-#pragma unroll
-        for (int o = 0; o < 32; ++o)
-            accg[bb][o] = 0.f;
-#pragma unroll
-        for (int o = 0; o < OPL; ++o)
-            acc[bb][o] = 0.f;
-    }
-
-    //   acc += s * (2^code_shift accg - z * sum x')
-    auto fold = [&](int G, const float *Xg) {
-        const bool staged = (G >= G0) && (G < G0 + span);
-        uint32_t w[32]; // (s, z) of this lane's 32 outputs
-        if (staged) {
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint4 v = szs[(G - G0) * 256 + part_chunk(lane, c)];
-                w[4 * c] = v.x;
-                w[4 * c + 1] = v.y;
-                w[4 * c + 2] = v.z;
-                w[4 * c + 3] = v.w;
-            }
-        } else {
-            const uint4 *g4 = reinterpret_cast<const uint4 *>(
-                p.sz + (size_t)G * SN + s0 + (lane_ok ? lane * 32 : 0));
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint4 v = __ldg(g4 + c);
-                w[4 * c] = v.x;
-                w[4 * c + 1] = v.y;
-                w[4 * c + 2] = v.z;
-                w[4 * c + 3] = v.w;
-            }
+        // accg[bb][o] = this group's sum of q x' 2^-code_shift(o) for code slot o;
+        // acc[bb][o] = folded result of output o in units of 2^-S.
+        float accg[BW][32], acc[BW][OPL];
+    #pragma unroll
+        for (int bb = 0; bb < BW; ++bb) {
+    #pragma unroll
+            for (int o = 0; o < 32; ++o)
+                accg[bb][o] = 0.f;
+    #pragma unroll
+            for (int o = 0; o < OPL; ++o)
+                acc[bb][o] = 0.f;
         }
-        if (!NM) {
-#pragma unroll
-            for (int o = 0; o < 32; ++o) {
-                const float s = half_lo(w[o]), z = half_hi(w[o]);
-#pragma unroll
-                for (int bb = 0; bb < BW; ++bb) {
-                    const float t = accg[bb][o] * pow2f(code_shift(o));
-                    acc[bb][o] = fmaf(s, fmaf(-z, Xg[bb], t), acc[bb][o]);
-                    accg[bb][o] = 0.f;
+
+        //   acc += s * (2^code_shift accg - z * sum x')
+        auto fold = [&](int G, const float *Xg) {
+            const bool staged = (G >= G0) && (G < G0 + span);
+            uint32_t w[32]; // (s, z) of this lane's 32 outputs
+            if (staged) {
+    #pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 v = szs[(G - G0) * 256 + part_chunk(lane, c)];
+                    w[4 * c] = v.x;
+                    w[4 * c + 1] = v.y;
+                    w[4 * c + 2] = v.z;
+                    w[4 * c + 3] = v.w;
+                }
+            } else {
+                const uint4 *g4 = reinterpret_cast<const uint4 *>(
+                    p.sz + (size_t)G * SN + s0 + (lane_ok ? lane * 32 : 0));
+    #pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 v = __ldg(g4 + c);
+                    w[4 * c] = v.x;
+                    w[4 * c + 1] = v.y;
+                    w[4 * c + 2] = v.z;
+                    w[4 * c + 3] = v.w;
                 }
             }
-        } else {
-            // Keep nibbles of this lane's 16 blocks (8 bytes); block j's slots
-            // 2j, 2j + 1 go to its first and second kept output.
-            const uint2 km = lane_ok ? __ldg(reinterpret_cast<const uint2 *>(
-                                           p.keep + (size_t)G * (p.N / 8) + n0 / 8 + lane * 8))
-                                     : make_uint2(0u, 0u);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                float f[2];
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int o = 2 * j + h;
-                    const float t = accg[0][o] * pow2f(code_shift(o));
-                    f[h] = half_lo(w[o]) * fmaf(-half_hi(w[o]), Xg[0], t);
-                    accg[0][o] = 0.f;
+            if (!NM) {
+    #pragma unroll
+                for (int o = 0; o < 32; ++o) {
+                    const float s = half_lo(w[o]), z = half_hi(w[o]);
+    #pragma unroll
+                    for (int bb = 0; bb < BW; ++bb) {
+                        const float t = accg[bb][o] * pow2f(code_shift(o));
+                        acc[bb][o] = fmaf(s, fmaf(-z, Xg[bb], t), acc[bb][o]);
+                        accg[bb][o] = 0.f;
+                    }
                 }
-                const uint32_t m = ((j < 8 ? km.x : km.y) >> (4 * (j & 7))) & 0xFu;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const bool kept = (m >> i) & 1u;
-                    const bool second = (m & ((1u << i) - 1u)) != 0u; // a kept output below i
-                    acc[0][4 * j + i] += kept ? (second ? f[1] : f[0]) : 0.f;
+            } else {
+                // Keep nibbles of this lane's 16 blocks (8 bytes); block j's slots
+                // 2j, 2j + 1 go to its first and second kept output.
+                const uint2 km = lane_ok ? __ldg(reinterpret_cast<const uint2 *>(
+                                               p.keep + (size_t)G * (p.N / 8) + n0 / 8 + lane * 8))
+                                         : make_uint2(0u, 0u);
+    #pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    float f[2];
+    #pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int o = 2 * j + h;
+                        const float t = accg[0][o] * pow2f(code_shift(o));
+                        f[h] = half_lo(w[o]) * fmaf(-half_hi(w[o]), Xg[0], t);
+                        accg[0][o] = 0.f;
+                    }
+                    const uint32_t m = ((j < 8 ? km.x : km.y) >> (4 * (j & 7))) & 0xFu;
+    #pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const bool kept = (m >> i) & 1u;
+                        const bool second = (m & ((1u << i) - 1u)) != 0u; // a kept output below i
+                        acc[0][4 * j + i] += kept ? (second ? f[1] : f[0]) : 0.f;
+                    }
                 }
             }
-        }
-    };
+        };
 
-    auto xrow = [&](int j, uint16_t *xh) {
-#pragma unroll
-        for (int bb = 0; bb < BW; ++bb)
-            xh[bb] = rxh[(b0 + bb) * rcap + wa + j];
-    };
+        auto xrow = [&](int j, uint16_t *xh) {
+    #pragma unroll
+            for (int bb = 0; bb < BW; ++bb)
+                xh[bb] = rxh[(b0 + bb) * rcap + wa + j];
+        };
 
-    // Runs of rows of one group: the run end comes from one ballot per 32
-    // rows, and sum x' of the run from one warp reduction, so the per-row work
-    // is the ring read, the codes and the refill only.
-    int i = 0;
-    while (i < n) {
-        const int G = row(wa + i) >> lg;
-        int i1 = i;
-        float Xg[BW];
-#pragma unroll
-        for (int bb = 0; bb < BW; ++bb)
-            Xg[bb] = 0.f;
-        for (;;) {
-            const int j = i1 + lane;
-            const bool in = (j < n) && ((row(wa + j) >> lg) == G);
-            const uint32_t bal = __ballot_sync(0xffffffffu, in);
-            const int len = (bal == 0xffffffffu) ? 32 : (__ffs(~bal) - 1);
-            if (lane < len) {
-#pragma unroll
-                for (int bb = 0; bb < BW; ++bb)
-                    Xg[bb] += __half2float(__ushort_as_half(rxh[(b0 + bb) * rcap + wa + j]));
+        // Runs of rows of one group: the run end comes from one ballot per 32
+        // rows, and sum x' of the run from one warp reduction, so the per-row work
+        // is the ring read, the codes and the refill only.
+        int i = 0;
+        while (i < n) {
+            const int G = row(wa + i) >> lg;
+            int i1 = i;
+            float Xg[BW];
+    #pragma unroll
+            for (int bb = 0; bb < BW; ++bb)
+                Xg[bb] = 0.f;
+            for (;;) {
+                const int j = i1 + lane;
+                const bool in = (j < n) && ((row(wa + j) >> lg) == G);
+                const uint32_t bal = __ballot_sync(0xffffffffu, in);
+                const int len = (bal == 0xffffffffu) ? 32 : (__ffs(~bal) - 1);
+                if (lane < len) {
+    #pragma unroll
+                    for (int bb = 0; bb < BW; ++bb)
+                        Xg[bb] += __half2float(__ushort_as_half(rxh[(b0 + bb) * rcap + wa + j]));
+                }
+                i1 += len;
+                if (len < 32)
+                    break;
             }
-            i1 += len;
-            if (len < 32)
-                break;
-        }
-#pragma unroll
-        for (int bb = 0; bb < BW; ++bb)
-#pragma unroll
-            for (int d = 16; d > 0; d >>= 1)
-                Xg[bb] += __shfl_xor_sync(0xffffffffu, Xg[bb], d);
+    #pragma unroll
+            for (int bb = 0; bb < BW; ++bb)
+    #pragma unroll
+                for (int d = 16; d > 0; d >>= 1)
+                    Xg[bb] += __shfl_xor_sync(0xffffffffu, Xg[bb], d);
 
-        for (; i + 1 < i1; i += 2) {
-            cp_async_wait<kStages1 - 2>(); // rows i and i + 1 have landed
-            const int slot = i & (kStages1 - 1), slot1 = (i + 1) & (kStages1 - 1);
-            const uint4 v0 = *reinterpret_cast<const uint4 *>(myring + slot * kRowBytes1);
-            const uint4 v1 = *reinterpret_cast<const uint4 *>(myring + slot1 * kRowBytes1);
-            uint16_t xh0[BW], xh1[BW];
-            xrow(i, xh0);
-            xrow(i + 1, xh1);
-            mac_row<BW>(v0, xh0, accg);
-            mac_row<BW>(v1, xh1, accg);
-            if (i + kStages1 < n)
-                cp_async16(myring + slot * kRowBytes1,
-                           wcol + (size_t)row(wa + i + kStages1) * row_stride);
-            cp_async_commit();
-            if (i + 1 + kStages1 < n)
-                cp_async16(myring + slot1 * kRowBytes1,
-                           wcol + (size_t)row(wa + i + 1 + kStages1) * row_stride);
-            cp_async_commit();
+            for (; i + 1 < i1; i += 2) {
+                cp_async_wait<kStages1 - 2>(); // rows i and i + 1 have landed
+                const int slot = i & (kStages1 - 1), slot1 = (i + 1) & (kStages1 - 1);
+                const uint4 v0 = *reinterpret_cast<const uint4 *>(myring + slot * kRowBytes1);
+                const uint4 v1 = *reinterpret_cast<const uint4 *>(myring + slot1 * kRowBytes1);
+                uint16_t xh0[BW], xh1[BW];
+                xrow(i, xh0);
+                xrow(i + 1, xh1);
+                mac_row<BW>(v0, xh0, accg);
+                mac_row<BW>(v1, xh1, accg);
+                if (i + kStages1 < n)
+                    cp_async16(myring + slot * kRowBytes1,
+                               wcol + (size_t)row(wa + i + kStages1) * row_stride);
+                cp_async_commit();
+                if (i + 1 + kStages1 < n)
+                    cp_async16(myring + slot1 * kRowBytes1,
+                               wcol + (size_t)row(wa + i + 1 + kStages1) * row_stride);
+                cp_async_commit();
+            }
+            if (i < i1) {
+                // The last row of an odd-length run.
+                cp_async_wait<kStages1 - 1>();
+                const int slot = i & (kStages1 - 1);
+                const uint4 v = *reinterpret_cast<const uint4 *>(myring + slot * kRowBytes1);
+                uint16_t xh[BW];
+                xrow(i, xh);
+                mac_row<BW>(v, xh, accg);
+                if (i + kStages1 < n)
+                    cp_async16(myring + slot * kRowBytes1,
+                               wcol + (size_t)row(wa + i + kStages1) * row_stride);
+                cp_async_commit();
+                ++i;
+            }
+            fold(G, Xg);
         }
-        if (i < i1) {
-            // The last row of an odd-length run.
-            cp_async_wait<kStages1 - 1>();
-            const int slot = i & (kStages1 - 1);
-            const uint4 v = *reinterpret_cast<const uint4 *>(myring + slot * kRowBytes1);
-            uint16_t xh[BW];
-            xrow(i, xh);
-            mac_row<BW>(v, xh, accg);
-            if (i + kStages1 < n)
-                cp_async16(myring + slot * kRowBytes1,
-                           wcol + (size_t)row(wa + i + kStages1) * row_stride);
-            cp_async_commit();
-            ++i;
-        }
-        fold(G, Xg);
-    }
 
-    // This warp's partial tiles, in real units (x 2^-S, two exact factors),
-    // into its own region: every cp.async of this warp has landed and been
-    // read, so nothing else touches that region any more.
-    cp_async_wait_all();
-    __syncwarp();
-#pragma unroll
-    for (int bb = 0; bb < BW; ++bb) {
-        float4 *part = reinterpret_cast<float4 *>(region) + bb * (TO / 4);
-        const int E = -S[bb];
-        const float f1 = pow2f(E / 2), f2 = pow2f(E - E / 2);
-        const bool live = lane_ok && n > 0 && bb < nbw;
-#pragma unroll
-        for (int c = 0; c < OPL / 4; ++c)
-            part[NM ? part_chunk16(lane, c) : part_chunk(lane, c)] =
-                live ? make_float4((acc[bb][4 * c] * f1) * f2, (acc[bb][4 * c + 1] * f1) * f2,
-                                   (acc[bb][4 * c + 2] * f1) * f2, (acc[bb][4 * c + 3] * f1) * f2)
-                     : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    __syncthreads();
-    // Each thread owns chunks of 4 outputs of the tile (one, or two for the
-    // 2:4 tile); for every batch row it sums the partial tiles of the warps of
-    // that row's group and adds the sum into the workspace.
-    if (NM) {
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            const int q = tid + r * kThreads1; // chunk of the 2048-output tile
-            const int l = q >> 4, c = q & 15;
+        // This warp's partial tiles, in real units (x 2^-S, two exact factors),
+        // into its own region: every cp.async of this warp has landed and been
+        // read, so nothing else touches that region any more.
+        cp_async_wait_all();
+        __syncwarp();
+    #pragma unroll
+        for (int bb = 0; bb < BW; ++bb) {
+            float4 *part = reinterpret_cast<float4 *>(region) + bb * (TO / 4);
+            const int E = -S[bb];
+            const float f1 = pow2f(E / 2), f2 = pow2f(E - E / 2);
+            const bool live = lane_ok && n > 0 && bb < nbw;
+    #pragma unroll
+            for (int c = 0; c < OPL / 4; ++c)
+                part[NM ? part_chunk16(lane, c) : part_chunk(lane, c)] =
+                    live ? make_float4((acc[bb][4 * c] * f1) * f2, (acc[bb][4 * c + 1] * f1) * f2,
+                                       (acc[bb][4 * c + 2] * f1) * f2, (acc[bb][4 * c + 3] * f1) * f2)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        __syncthreads();
+        // Each thread owns chunks of 4 outputs of the tile (one, or two for the
+        // 2:4 tile); for every batch row it sums the partial tiles of the warps of
+        // that row's group and adds the sum into the workspace.
+        if (NM) {
+    #pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int q = tid + r * kThreads1; // chunk of the 2048-output tile
+                const int l = q >> 4, c = q & 15;
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    #pragma unroll
+                for (int w = 0; w < kWarps1; ++w) {
+                    const float4 u = reinterpret_cast<const float4 *>(
+                        ring + (size_t)w * warp_region_bytes(BW, NM))[part_chunk16(l, c)];
+                    v.x += u.x;
+                    v.y += u.y;
+                    v.z += u.z;
+                    v.w += u.w;
+                }
+                if (n0 + 4 * q < p.N)
+                    red_add_v4(p.ws_acc + n0 + 4 * q, v);
+            }
+        } else     if (BW == 1) {
+            const int l = tid >> 3, c = tid & 7;
             float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
+    #pragma unroll
             for (int w = 0; w < kWarps1; ++w) {
                 const float4 u = reinterpret_cast<const float4 *>(
-                    ring + (size_t)w * warp_region_bytes(BW, NM))[part_chunk16(l, c)];
-                v.x += u.x;
-                v.y += u.y;
-                v.z += u.z;
-                v.w += u.w;
-            }
-            if (n0 + 4 * q < p.N)
-                red_add_v4(p.ws_acc + n0 + 4 * q, v);
-        }
-    } else     if (BW == 1) {
-        const int l = tid >> 3, c = tid & 7;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int w = 0; w < kWarps1; ++w) {
-            const float4 u = reinterpret_cast<const float4 *>(
-                ring + (size_t)w * warp_region_bytes(BW))[part_chunk(l, c)];
-            v.x += u.x;
-            v.y += u.y;
-            v.z += u.z;
-            v.w += u.w;
-        }
-        if (n0 + 4 * tid < p.N)
-            red_add_v4(p.ws_acc + n0 + 4 * tid, v);
-    } else {
-        const int l = tid >> 3, c = tid & 7;
-        for (int b = 0; b < p.B; ++b) {
-            const int w0 = (b / BW) * wpg, bb = b % BW;
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int w = w0; w < w0 + wpg; ++w) {
-                const float4 u = reinterpret_cast<const float4 *>(
-                    ring + (size_t)w * warp_region_bytes(BW))[bb * (kTileN1 / 4) + part_chunk(l, c)];
+                    ring + (size_t)w * warp_region_bytes(BW))[part_chunk(l, c)];
                 v.x += u.x;
                 v.y += u.y;
                 v.z += u.z;
                 v.w += u.w;
             }
             if (n0 + 4 * tid < p.N)
-                red_add_v4(p.ws_acc + (size_t)b * p.N + n0 + 4 * tid, v);
+                red_add_v4(p.ws_acc + n0 + 4 * tid, v);
+        } else {
+            const int l = tid >> 3, c = tid & 7;
+            for (int b = 0; b < p.B; ++b) {
+                const int w0 = (b / BW) * wpg, bb = b % BW;
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int w = w0; w < w0 + wpg; ++w) {
+                    const float4 u = reinterpret_cast<const float4 *>(
+                        ring + (size_t)w * warp_region_bytes(BW))[bb * (kTileN1 / 4) + part_chunk(l, c)];
+                    v.x += u.x;
+                    v.y += u.y;
+                    v.z += u.z;
+                    v.w += u.w;
+                }
+                if (n0 + 4 * tid < p.N)
+                    red_add_v4(p.ws_acc + (size_t)b * p.N + n0 + 4 * tid, v);
+            }
         }
+
     }
 }
 
@@ -676,6 +710,31 @@ cudaError_t launch_gemv_t(KParams kp, int num_sms, cudaStream_t stream)
     if (L.total > kMaxSmem ||
         ((SRC == ROWS_THRESH || SRC == ROWS_GLU) && kp.rows_cap > 4 * kThreads1))
         return cudaErrorInvalidConfiguration;
+    // Index list on a tile count that whole splits per tile cannot spread
+    // over 90% of the SMs (e.g. 50 tiles: 100 of 148 CTAs), or that needs
+    // more than one wave: one equal share of the (tile, list entry) space per
+    // SM instead (segments, see gemv_kernel).
+    if constexpr (SRC == ROWS_LIST && !NM) {
+        const long long ctas = (long long)kp.n_tiles * kp.k_splits;
+        if (kp.n_tiles <= num_sms && (10 * ctas < 9LL * num_sms || ctas > num_sms) &&
+            (long long)kp.n_tiles * p.K < (1ll << 31)) {
+            KParams ks = kp;
+            const int share = ceil_div((long long)kp.n_tiles * p.K, num_sms);
+            ks.rows_cap = std::min(p.K, share) + 8;
+            // scale/zero staged for the groups a share's rows touch (about
+            // twice its rows at 50% sparsity), as many as shared memory holds;
+            // the others are folded from global memory
+            ks.span_cap = std::min(G, ceil_div(2LL * share, 1LL << kp.lg) + 2);
+            Smem1 LS = smem1_layout(ks.span_cap, ks.rows_cap, bp, BW, NM);
+            while (ks.span_cap > 1 && LS.total > kMaxSmem) {
+                --ks.span_cap;
+                LS = smem1_layout(ks.span_cap, ks.rows_cap, bp, BW, NM);
+            }
+            if (LS.total <= kMaxSmem)
+                return launch_gemv_and_finalize(gemv_kernel<SRC, BW, NM, true>, num_sms,
+                                                kThreads1, LS.total, stream, ks);
+        }
+    }
     return launch_gemv_and_finalize(gemv_kernel<SRC, BW, NM>, kp.n_tiles * kp.k_splits,
                                     kThreads1, L.total, stream, kp);
 }

@@ -76,17 +76,23 @@ __device__ __forceinline__ void channel_slice(const KParams &kp, int split, int 
 // ---------------------------------------------------------------------------
 template <int SRC, int NT, bool FILL_X = false>
 __device__ int build_rows(const KParams &kp, int split, int32_t *ridx, float *rx, int *scan,
-                          float *xs = nullptr, bool write_h = false)
+                          float *xs = nullptr, bool write_h = false, int list_lo = -1,
+                          int list_hi = -1)
 {
     const GemvProblem &p = kp.p;
     const int tid = threadIdx.x;
     if (SRC == ROWS_LIST) {
-        const int c = __ldg(p.count);
-        const int a = c < 0 ? 0 : (c > p.K ? p.K : c);
-        if (a != c && tid == 0 && blockIdx.x == 0)
-            set_status(p.status, SGQ_STATUS_BAD_COUNT);
-        const int r0 = (int)((long long)a * split / kp.k_splits);
-        const int r1 = (int)((long long)a * (split + 1) / kp.k_splits);
+        // entries [list_lo, list_hi) when given (the caller has checked the
+        // count), else this split's share of the list
+        int r0 = list_lo, r1 = list_hi;
+        if (list_lo < 0) {
+            const int c = __ldg(p.count);
+            const int a = c < 0 ? 0 : (c > p.K ? p.K : c);
+            if (a != c && tid == 0 && blockIdx.x == 0)
+                set_status(p.status, SGQ_STATUS_BAD_COUNT);
+            r0 = (int)((long long)a * split / kp.k_splits);
+            r1 = (int)((long long)a * (split + 1) / kp.k_splits);
+        }
         for (int j = tid; j < r1 - r0; j += NT) {
             int k = __ldg(p.idx + r0 + j);
             if ((unsigned)k >= (unsigned)p.K) {

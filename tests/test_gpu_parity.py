@@ -271,6 +271,36 @@ def test_gemv_batch_unsorted_list_with_repeats(B, g):
     assert gg.status.item() == 0
 
 
+@pytest.mark.parametrize("B,order", [(1, "sorted"), (3, "sorted"), (1, "unsorted"), (5, "unsorted")])
+def test_gemv_list_equal_shares_over_tiles(B, order):
+    """40 tiles (N = 40928, the last one ragged): whole splits per tile would
+    leave SMs idle, so the CUDA-core kernel gives each SM an equal share of
+    the (tile, list entry) space, some shares spanning two tiles."""
+    N, K, g = 40928, 2048, 64
+    case = wl.gemv_case(N=N, K=K, group=g, B=B, sparsity=0.5, seed=120 + B)
+    gg = GpuGemv(case.W, g, B)
+    x_d = case.x.to(DEV)
+    if order == "sorted":
+        gg.select(x_d, case.t)
+        idx = gg.active()
+        y, y32 = gg.gemv(x_d)
+    else:
+        rng = np.random.default_rng(B)
+        idx = rng.permutation(K)[: K // 3]
+        idx = np.concatenate([idx, idx[:50]]).astype(np.int32)
+        rng.shuffle(idx)
+        idx_d = torch.tensor(idx, dtype=torch.int32, device=DEV)
+        cnt = torch.tensor([idx.size], dtype=torch.int32, device=DEV)
+        y, y32 = gg.gemv(x_d, idx_d, cnt)
+    rows = sample_rows(N, 512, B)
+    q, s, z = oracle_codes(case.W, g, rows)
+    y64, sa, _ = oracle.gemv(q, s, z, g, bits(case.x), idx)
+    torch.cuda.synchronize()
+    check_y(y[:, rows], y32[:, rows], y64, sa, f"equal shares B={B} {order}")
+    assert gg.workspace_is_zero()
+    assert gg.status.item() == 0
+
+
 @pytest.mark.parametrize("sparsity", [0.0, 0.5, 0.9])
 def test_gemv_thresh_matches_oracle(sparsity):
     case = wl.gemv_case(**wl.LLAMA8B_DOWN, sparsity=sparsity, seed=2, act="silu")
