@@ -95,6 +95,12 @@ def test_host_argument_checks(lib):
     assert lib.sgq_gemv(*args(idx=None)) == -1
     assert lib.sgq_gemv(*args(y=odd)) == -4
     assert lib.sgq_gemv(*args(wsb=ws - 1)) == -6
+    # the wait-limit test hook runs only on the tensor-core batch sizes
+    wsb = lib.sgq_gemv_workspace_bytes(4096, 14336, 12)
+    assert lib.sgq_debug_gemv_withhold(*args(B=4)) == -2
+    assert lib.sgq_debug_gemv_withhold(*args(B=17)) == -2
+    assert lib.sgq_debug_gemv_withhold(*args(B=12, idx=None, wsb=wsb)) == -1
+    assert lib.sgq_debug_gemv_withhold(*args(B=12, wsb=wsb - 1)) == -6
     assert lib.sgq_glu(fake, fake, fake, 1, 12, 0, None) == -2               # not % 8
     assert lib.sgq_glu(fake, fake, fake, 1, 16, 5, None) == -7               # activation
     assert lib.sgq_pack(fake, 4096, 14336, 100, fake, fake, None, None) == -3
