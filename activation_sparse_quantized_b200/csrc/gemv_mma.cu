@@ -59,11 +59,14 @@ constexpr int kMWarps = 16;                 // warps that expand rows (one slot 
 constexpr int kIssuer = kMWarps;            // one more warp issues the MMAs
 constexpr int kAllWarps = kMWarps + 1;
 constexpr int kMThreads = kAllWarps * 32;
-constexpr int kKb = 16;                     // rows per K-block (the fp16 MMA's K)
+constexpr int kKStep = 16;                  // the fp16 MMA's K
 constexpr int kMmaN = 16;                   // MMA N: batch columns, padded to 16
 constexpr int kMBlocks = kTileN1 / 128;     // MMA M-blocks per tile
-constexpr int kAStage = kKb * kTileN1 * 2;  // A operand of one K-block: 32 KB
-constexpr int kBStage = kKb * kMmaN * 2;    // B operand of one K-block: 512 B
+// A K-block (one hand-off between the expanding warps and the issuer) holds
+// KB = 16 or 32 rows: its A operand is KB x 1024 outputs (32 or 64 KB), its B
+// operand KB x 16 batch columns; warp w expands slots w and w + 16.
+__host__ __device__ constexpr int a_stage_bytes(int kb) { return kb * kTileN1 * 2; }
+__host__ __device__ constexpr int b_stage_bytes(int kb) { return kb * kMmaN * 2; }
 constexpr int kMaxStages = 4;               // operand stages (2..4, by shared memory)
 constexpr int kMRing = 4;                   // rows in flight per expanding warp
 constexpr int kTmemCols = 512;              // two accumulator sets and the running totals
@@ -111,10 +114,10 @@ __host__ __device__ constexpr int mma_out_of_slot(int m)
 
 // Byte offset of element (batch column c, slot k) in a K-block's B stage:
 // K-major, no swizzle, core matrices of 8 columns x 8 slots (16-byte rows),
-// 128 bytes apart along K and 256 along N.
-__device__ __forceinline__ uint32_t b_elem_off(int c, int k)
+// 128 bytes apart along K and KB / 8 x 128 along N.
+__device__ __forceinline__ uint32_t b_elem_off(int c, int k, int kb)
 {
-    return (uint32_t)((k & 7) * 2 + (c & 7) * 16 + (k >> 3) * 128 + (c >> 3) * 256);
+    return (uint32_t)((k & 7) * 2 + (c & 7) * 16 + (k >> 3) * 128 + (c >> 3) * (kb / 8) * 128);
 }
 
 struct SmemM {
@@ -132,12 +135,12 @@ __host__ __device__ inline int rxh_stride(int rows_cap) { return (((rows_cap + 7
 // warp's per-lane rings; rxh: x' of the CTA's rows, [bp batch rows][stride]
 // fp16; ridx: the CTA's rows; rstart / rkb: first row / first K-block of each
 // run (+1 entry); scan: per-32-row counts.
-__host__ __device__ inline SmemM smemm_layout(int rows_cap, int stages, int bp)
+__host__ __device__ inline SmemM smemm_layout(int rows_cap, int stages, int bp, int kb)
 {
     SmemM s;
     s.a = 0;
-    s.b = s.a + (size_t)stages * kAStage;
-    s.ring = s.b + (size_t)stages * kBStage;
+    s.b = s.a + (size_t)stages * a_stage_bytes(kb);
+    s.ring = s.b + (size_t)stages * b_stage_bytes(kb);
     s.rxh = s.ring + (size_t)kMWarps * kMRing * kRowBytes1;
     s.ridx = align16(s.rxh + (size_t)bp * rxh_stride(rows_cap) * 2);
     s.rstart = align16(s.ridx + (size_t)rows_cap * 4);
@@ -322,7 +325,7 @@ __device__ int segment_rows(const GemvProblem &p, int lo, int hi, int32_t *ridx,
     }
 }
 
-template <int SRC>
+template <int SRC, int KB>
 __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -336,7 +339,9 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nst = kp.stages, bp = kp.bp;
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    const SmemM L = smemm_layout(kp.rows_cap, nst, bp);
+    constexpr int SPW = KB / 16; // slots per expanding warp
+    constexpr int AST = a_stage_bytes(KB), BST = b_stage_bytes(KB);
+    const SmemM L = smemm_layout(kp.rows_cap, nst, bp, KB);
     uint8_t *ring = smem + L.ring;
     uint16_t *rxh = reinterpret_cast<uint16_t *>(smem + L.rxh);
     int32_t *ridx = reinterpret_cast<int32_t *>(smem + L.ridx);
@@ -447,7 +452,7 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
             int carry = 0;
             for (int c = 0; c * 32 < nruns; ++c) {
                 const int r = c * 32 + lane;
-                const int v = (r < nruns) ? (rstart[r + 1] - rstart[r] + kKb - 1) / kKb : 0;
+                const int v = (r < nruns) ? (rstart[r + 1] - rstart[r] + KB - 1) / KB : 0;
                 int incl = v;
     #pragma unroll
                 for (int d = 1; d < 32; d <<= 1) {
@@ -489,17 +494,22 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
                         ok = mbar_wait(bar_free + (rg & 1), (uint32_t)(((rg >> 1) - 1) & 1), ok);
                         tc_fence_after();
                     }
-                    const uint32_t a_st = sA + (uint32_t)(s * kAStage);
+                    const uint32_t a_st = sA + (uint32_t)(s * AST);
                     const uint32_t dcol = tmem + (uint32_t)(128 * (rg & 1));
-                    const uint64_t bdesc = smem_desc(sB + (uint32_t)(s * kBStage), 128, 256, 0);
                     // Every M-block: a lane's outputs are spread over the M-blocks
                     // (lanes past N hold finite codes of column 0 and are dropped
                     // in the epilogue).
     #pragma unroll
-                    for (int mb = 0; mb < kMBlocks; ++mb)
-                        mma_f16(dcol + (uint32_t)(kMmaN * mb),
-                                smem_desc(a_st + (uint32_t)(mb * 2048), 1024, 16 * 1024, 2), bdesc,
-                                !first);
+                    for (int kk = 0; kk < KB / kKStep; ++kk) {
+                        const uint64_t bdesc = smem_desc(
+                            sB + (uint32_t)(s * BST + kk * 256), 128, (KB / 8) * 128, 0);
+    #pragma unroll
+                        for (int mb = 0; mb < kMBlocks; ++mb)
+                            mma_f16(dcol + (uint32_t)(kMmaN * mb),
+                                    smem_desc(a_st + (uint32_t)(kk * 32768 + mb * 2048), 1024,
+                                              16 * 1024, 2),
+                                    bdesc, !first || kk > 0);
+                    }
                     mma_commit(bar_empty + s);
                     if (last && !(p.debug_withhold_ready && run == nruns - 1))
                         mma_commit(bar_ready + (rg & 1));
@@ -590,15 +600,16 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
             const uint8_t *wcol = p.qweight + (lane_ok ? ((size_t)n0 / 2 + lane * 16) : 0);
             uint8_t *myring = ring + (size_t)warp * kMRing * kRowBytes1 + lane * 16;
             int ring_run = 0;
-            auto kb_row = [&](int kb) -> int { // ridx position of this warp's slot, or -1
+            // ridx position of this warp's slot u of K-block kb, or -1
+            auto kb_row = [&](int kb, int u) -> int {
                 kb_run(kb, ring_run);
-                const int j = rstart[ring_run] + kKb * (kb - rkb[ring_run]) + warp;
+                const int j = rstart[ring_run] + KB * (kb - rkb[ring_run]) + warp + 16 * u;
                 return (j < rstart[ring_run + 1]) ? j : -1;
             };
     #pragma unroll
             for (int i = 0; i < kMRing; ++i) {
-                if (i < nkb) {
-                    const int j = kb_row(i);
+                if (i < SPW * nkb) {
+                    const int j = kb_row(i / SPW, i % SPW);
                     if (j >= 0)
                         cp_async16(myring + i * kRowBytes1,
                                    wcol + (size_t)max(ridx[j], 0) * row_bytes);
@@ -607,11 +618,14 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
             }
             // This lane's four A chunks of slot `warp` (stage-relative) and its B
             // element (lanes 0..15: batch column = lane).
-            uint32_t aoff[4];
+            uint32_t aoff[SPW][4], boff[SPW];
     #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                aoff[j] = a_chunk_off(lane, j, warp);
-            const uint32_t boff = b_elem_off(lane & 15, warp);
+            for (int u = 0; u < SPW; ++u) {
+    #pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    aoff[u][j] = a_chunk_off(lane, j, warp + 16 * u);
+                boff[u] = b_elem_off(lane & 15, warp + 16 * u, KB);
+            }
 
             // Zero points of this lane's 32 outputs for one group, as subnormal
             // fp16 pairs matching the AND results: word j, pairs = outputs
@@ -701,8 +715,8 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
                 kb_run(kb, run);
                 const int kg = kb_base + kb;
                 const int s = kg % nst;
-                const int j0 = rstart[run] + kKb * (kb - rkb[run]);
-                const bool valid = warp < rstart[run + 1] - j0;
+                const int j0 = rstart[run] + KB * (kb - rkb[run]);
+                const int nv = rstart[run + 1] - j0; // valid slots (may exceed KB)
                 const bool first = kb == rkb[run];
                 if (first) {
                     unpack_z(); // this run's zero points (loaded a run ahead)
@@ -712,39 +726,47 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
                 // The stage's previous K-block has been multiplied.
                 if (kg >= nst)
                     ok = mbar_wait(bar_empty + s, (uint32_t)((kg / nst - 1) & 1), ok);
-                const uint32_t a_st = sA + (uint32_t)(s * kAStage);
-                cp_async_wait<kMRing - 1>();
-                uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                if (valid)
-                    v = *reinterpret_cast<const uint4 *>(myring + (kb % kMRing) * kRowBytes1);
-                // refill the ring slot with this warp's row kMRing K-blocks ahead
-                if (kb + kMRing < nkb) {
-                    const int j = kb_row(kb + kMRing);
-                    if (j >= 0)
-                        cp_async16(myring + (kb % kMRing) * kRowBytes1,
-                                   wcol + (size_t)max(ridx[j], 0) * row_bytes);
-                }
-                cp_async_commit();
-                const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+                const uint32_t a_st = sA + (uint32_t)(s * AST);
     #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    uint32_t t0 = 0u, t1 = 0u, t2 = 0u, t3 = 0u;
-                    if (valid) {
-                        const uint32_t w = wv[j], w8 = w >> 8;
-                        t0 = hsub2(w & 0x000F000Fu, zc[j][0]);
-                        t1 = hsub2(w & 0x00F000F0u, zc[j][1]);
-                        t2 = hsub2(w8 & 0x000F000Fu, zc[j][2]);
-                        t3 = hsub2(w8 & 0x00F000F0u, zc[j][3]);
+                for (int u = 0; u < SPW; ++u) {
+                    const int i = SPW * kb + u; // this warp's ring position
+                    const int slot = warp + 16 * u;
+                    const bool valid = slot < nv;
+                    cp_async_wait<kMRing - 1>();
+                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                    if (valid)
+                        v = *reinterpret_cast<const uint4 *>(myring + (i % kMRing) * kRowBytes1);
+                    // refill the ring slot with this warp's row kMRing positions ahead
+                    if (i + kMRing < SPW * nkb) {
+                        const int j = kb_row((i + kMRing) / SPW, (i + kMRing) % SPW);
+                        if (j >= 0)
+                            cp_async16(myring + (i % kMRing) * kRowBytes1,
+                                       wcol + (size_t)max(ridx[j], 0) * row_bytes);
                     }
-                    st_shared_v4(a_st + aoff[j], t0, t1, t2, t3);
-                }
-                if (lane < kMmaN) {
-                    // B operand: x' of slot `warp` for batch column `lane`.
-                    const uint16_t xv =
-                        (valid && lane < p.B) ? rxh[(size_t)lane * rs + j0 + warp] : (uint16_t)0;
-                    asm volatile("st.shared.u16 [%0], %1;" ::"r"(sB + (uint32_t)(s * kBStage) + boff),
-                                 "h"(xv)
-                                 : "memory");
+                    cp_async_commit();
+                    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+    #pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        uint32_t t0 = 0u, t1 = 0u, t2 = 0u, t3 = 0u;
+                        if (valid) {
+                            const uint32_t w = wv[j], w8 = w >> 8;
+                            t0 = hsub2(w & 0x000F000Fu, zc[j][0]);
+                            t1 = hsub2(w & 0x00F000F0u, zc[j][1]);
+                            t2 = hsub2(w8 & 0x000F000Fu, zc[j][2]);
+                            t3 = hsub2(w8 & 0x00F000F0u, zc[j][3]);
+                        }
+                        st_shared_v4(a_st + aoff[u][j], t0, t1, t2, t3);
+                    }
+                    if (lane < kMmaN) {
+                        // B operand: x' of this slot for batch column `lane`.
+                        const uint16_t xv = (valid && lane < p.B)
+                                                ? rxh[(size_t)lane * rs + j0 + slot]
+                                                : (uint16_t)0;
+                        asm volatile("st.shared.u16 [%0], %1;" ::"r"(sB + (uint32_t)(s * BST) +
+                                                                     boff[u]),
+                                     "h"(xv)
+                                     : "memory");
+                    }
                 }
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
@@ -840,28 +862,34 @@ cudaError_t launch_mma_t(KParams kp, int num_sms, cudaStream_t stream)
     int grid = num_sms;
     if (kp.n_tiles <= num_sms && 10 * kp.n_tiles * (num_sms / kp.n_tiles) >= 9 * num_sms)
         grid = kp.n_tiles * (num_sms / kp.n_tiles);
-    SmemM L;
-    for (;;) {
-        kp.rows_cap = (int)(8 * ((units + grid - 1) / grid + 1) + 8);
-        kp.rows_cap = std::min(kp.rows_cap, p.K + 8);
-        // the most operand stages that fit, at least two
-        kp.stages = kMaxStages;
-        L = smemm_layout(kp.rows_cap, kp.stages, kp.bp);
-        while (kp.stages > 2 && L.total + 1024 > kMaxSmem) {
-            --kp.stages;
-            L = smemm_layout(kp.rows_cap, kp.stages, kp.bp);
+    // 32-row K-blocks (half the hand-offs) when two stages of them fit with
+    // the share's rows; else 16-row K-blocks, more CTAs only if even those do
+    // not fit.
+    for (const int kb : {32, 16}) {
+        for (int g = grid;; g *= 2) {
+            KParams kq = kp;
+            kq.rows_cap = (int)(8 * ((units + g - 1) / g + 1) + 8);
+            kq.rows_cap = std::min(kq.rows_cap, p.K + 8);
+            kq.stages = kMaxStages;
+            SmemM L = smemm_layout(kq.rows_cap, kq.stages, kq.bp, kb);
+            while (kq.stages > 2 && L.total + 1024 > kMaxSmem) {
+                --kq.stages;
+                L = smemm_layout(kq.rows_cap, kq.stages, kq.bp, kb);
+            }
+            if (L.total + 1024 <= kMaxSmem) {
+                const size_t smem = std::max(L.total + 1024, kOneCtaSmem);
+                cudaError_t err =
+                    (kb == 32) ? launch_pdl(gemv_mma_kernel<SRC, 32>, g, kMThreads, smem, stream, kq)
+                               : launch_pdl(gemv_mma_kernel<SRC, 16>, g, kMThreads, smem, stream, kq);
+                if (err != cudaSuccess || p.accumulate)
+                    return err;
+                return launch_finalize(p, stream);
+            }
+            if (kb == 32 || (long long)g >= units)
+                break; // 32-row blocks only without extra waves
         }
-        if (L.total + 1024 <= kMaxSmem || (long long)grid >= units)
-            break;
-        grid *= 2;
     }
-    if (L.total + 1024 > kMaxSmem)
-        return cudaErrorInvalidConfiguration;
-    const size_t smem = std::max(L.total + 1024, kOneCtaSmem);
-    cudaError_t err = launch_pdl(gemv_mma_kernel<SRC>, grid, kMThreads, smem, stream, kp);
-    if (err != cudaSuccess || p.accumulate)
-        return err;
-    return launch_finalize(p, stream);
+    return cudaErrorInvalidConfiguration;
 }
 
 } // namespace
