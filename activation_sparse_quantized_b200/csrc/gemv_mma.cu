@@ -16,19 +16,20 @@
 //  * Tiles of 1024 outputs (512 bytes of a packed row) and k_splits shares of
 //    the rows per tile, as in the batch-1 kernel, with the same row lists.
 //  * The CTA's rows are cut into runs of one quantization group, and each run
-//    into K-blocks of 16 rows (the MMA's K; a run's last block is padded with
-//    zero rows).
-//  * 16 expanding warps; warp w expands slot w of every K-block. Its lanes
-//    stream their own 16-byte columns of its rows through per-lane cp.async
-//    rings (4 K-blocks ahead) and turn each code, minus the group's zero,
+//    into K-blocks of 32 rows (two MMA K-steps; 16 where two 64 KB operand
+//    stages do not fit shared memory), a run's last block padded with zero
+//    rows.
+//  * 16 expanding warps; warp w expands slots w and w + 16 of every K-block.
+//    Its lanes stream their own 16-byte columns of its rows through per-lane
+//    cp.async rings (4 rows ahead) and turn each code, minus the group's zero,
 //    into the exact fp16 value (q - z) 2^-24 (2^-20 for the high nibble of a
 //    byte): one AND and one packed fp16 subtraction per two codes, the zero
 //    being held in the same subnormal form. A K-block's A operand (1024
-//    outputs x 16 rows, M-major, 128-byte swizzle) and B operand (16 rows x
-//    16 batch columns of x' = x 2^S_b in fp16, K-major) go to one of 2..4
+//    outputs x its rows, M-major, 128-byte swizzle) and B operand (its rows
+//    x 16 batch columns of x' = x 2^S_b in fp16, K-major) go to one of 2..4
 //    stages.
-//  * A 17th warp issues the K-block's 8 MMAs (M = 128 outputs, N = 16,
-//    K = 16) into the run's accumulators (two alternating sets of 8 x 16
+//  * A 17th warp issues the K-block's MMAs (8 per K-step: M = 128 outputs,
+//    N = 16, K = 16) into the run's accumulators (two alternating sets of 8 x 16
 //    columns of tensor memory), then commits them to the stage's "empty"
 //    barrier and, at a run's end, to the set's "ready" barrier.
 //  * A run later the expanding warps read their outputs' sums from tensor
