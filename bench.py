@@ -2,7 +2,7 @@
 """Benchmark of the activation-sparse int4 GEMV on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--path auto|list|thresh] [--sparsity 0.5] [--sweep]
+                    [--path auto|list|thresh|mask] [--sparsity 0.5] [--no-ffn]
 
 Workload: the Llama-3-8B FFN down_proj GEMV (K = 14336 input channels,
 N = 4096 outputs), int4 asymmetric weights in groups of 128 along K with fp16
@@ -15,7 +15,19 @@ active channels and the sparse GEMV over them (select + gemv, or the fused
 threshold-GEMV). Steps cycle through R copies of the packed weights whose total
 size is more than 4x the L2 cache, so every step reads its weights from HBM.
 The K timed steps run as CUDA-graph replays on one stream, timed with CUDA
-events, bracketed by a barrier and a device synchronize.
+events, bracketed by a barrier and a device synchronize. Every graph of the
+timed region is replayed once before the warm-up (its first replay uploads
+it), and a bounded device delay ahead of the start event keeps the host's
+submission of the graphs outside the event window. The kernel-alone and
+call-alone timings (roofline kernel, dense GEMV, select, each entry point,
+the sparsity sweep, the ReGLU FFN, the tiny case) use a fixed 2000 launches
+whatever --steps is.
+
+Further legs on the same protocol: the sparsity sweep 0/30/50/70/90% of the
+same GEMV with a roofline fraction per row, the ReGLU FFN (natural ReLU zeros
+and an 88% stand-in), the tiny case (latency), the Llama-3-8B FFN and decode
+layer, the Qwen3-32B FFN at batch 1..16 and the 2:4 weight-sparse GEMV
+(--no-ffn skips them all).
 
 Metric: HBM GB/s on active bytes (and us per GEMV). Active bytes per GEMV are
 the weight bytes of the active channels (a*N/2), the scale/zero bytes of the
@@ -28,8 +40,10 @@ own steps, and reports the units of all ranks over the slowest rank's time
 (weak scaling).
 
 `--impl reference` times the CPU oracle (the plain fp64 C restatement under
-oracle/) on the machine's host cores on a bounded sample of the same workload; it
-is a deliberately slow reference arm, not a target.
+oracle/, its OpenMP form over every host core) on a bounded sample of the
+same workload; it is a deliberately slow reference arm, not a target. The
+cpu_baseline key of the main line times the oracle twice: on one thread and
+on every core.
 """
 from __future__ import annotations
 
@@ -241,29 +255,47 @@ class Replica:
         self.l2 = l2
         self.x_host = [wl.x_silu_gated(1, K, 1000 + r) for r in range(self.R)]
         self.x = [x.cuda() for x in self.x_host]
-        self.t = [wl.percentile_threshold(x[0], sparsity) for x in self.x_host]
-        # per-copy index lists (for timing the GEMV kernel alone) and byte counts
-        self.idx, self.cnt, self.abytes, self.active = [], [], [], []
-        for r in range(self.R):
-            idx, cnt = sgq.alloc_select(K)
-            sgq.sgq_select(self.x[r], 1, K, [self.t[r]], idx, cnt)
-            a = int(cnt.item())
-            groups = int(np.unique(idx[:a].cpu().numpy() // GROUP).size)
-            self.idx.append(idx)
-            self.cnt.append(cnt)
-            self.active.append(a)
-            self.abytes.append(active_bytes(a, groups))
         self.y = torch.empty(1, N, dtype=torch.bfloat16, device="cuda")
         self.ws = sgq.alloc_workspace(N, K, 1)
         self.sidx, self.scnt = sgq.alloc_select(K)
-        # per-copy bitmasks (for timing the mask GEMV alone) and a scratch mask
-        self.mask = []
-        for r in range(self.R):
-            m = sgq.alloc_mask(K)
-            sgq.sgq_select_mask(self.x[r], 1, K, [self.t[r]], m)
-            self.mask.append(m)
         self.smask = sgq.alloc_mask(K)
         self.yacc = torch.zeros(1, N, dtype=torch.float32, device="cuda")
+        self.idx = [sgq.alloc_select(K) for _ in range(self.R)]
+        self.mask = [sgq.alloc_mask(K) for _ in range(self.R)]
+        self.set_sparsity(sparsity)
+
+    def set_sparsity(self, sparsity: float):
+        """Thresholds for `sparsity` on every copy's x, with the per-copy index
+        lists and bitmasks (for timing the GEMV kernel alone) and the active
+        byte counts."""
+        self.sparsity = sparsity
+        self.t = [wl.percentile_threshold(x[0], sparsity) for x in self.x_host]
+        self.cnt, self.abytes, self.active, self.groups = [], [], [], []
+        for r in range(self.R):
+            idx, cnt = self.idx[r]
+            sgq.sgq_select(self.x[r], 1, K, [self.t[r]], idx, cnt)
+            a = int(cnt.item())
+            groups = int(np.unique(idx[:a].cpu().numpy() // GROUP).size)
+            self.cnt.append(cnt)
+            self.active.append(a)
+            self.groups.append(groups)
+            self.abytes.append(active_bytes(a, groups))
+            sgq.sgq_select_mask(self.x[r], 1, K, [self.t[r]], self.mask[r])
+        torch.cuda.synchronize()
+
+    def kernel_bytes(self, which: str) -> float:
+        """Algorithmic bytes per launch of one timed form, mean over the copies:
+        the fused threshold forms read all of x (2K) and no index list; the
+        accumulating forms write fp32 y (4N)."""
+        a = float(np.mean(self.active))
+        base = float(np.mean(self.abytes))
+        if which in ("thresh", "thresh_acc"):
+            base = base - 6 * a + 2 * K
+        if which == "mask":
+            base = base - 4 * a + K // 8
+        if which in ("thresh_acc", "gemv_acc"):
+            base = base + 2 * N
+        return base
 
     def step(self, r: int, path: str):
         """One pass of the hot path on copy r (kernels launched: 2 or 1)."""
@@ -281,7 +313,7 @@ class Replica:
 
     def kernel_only(self, r: int, which: str):
         if which == "gemv":
-            sgq.sgq_gemv(self.qw[r], self.sz[r], N, K, GROUP, self.x[r], 1, self.idx[r],
+            sgq.sgq_gemv(self.qw[r], self.sz[r], N, K, GROUP, self.x[r], 1, self.idx[r][0],
                          self.cnt[r], self.y, None, self.ws)
         elif which == "dense":
             sgq.sgq_gemv_dense(self.qw[r], self.sz[r], N, K, GROUP, self.x[r], 1, self.y, None,
@@ -300,7 +332,7 @@ class Replica:
             sgq.sgq_gemv_thresh_acc(self.qw[r], self.sz[r], N, K, GROUP, self.x[r], self.t[r],
                                     self.yacc)
         elif which == "gemv_acc":
-            sgq.sgq_gemv_acc(self.qw[r], self.sz[r], N, K, GROUP, self.x[r], 1, self.idx[r],
+            sgq.sgq_gemv_acc(self.qw[r], self.sz[r], N, K, GROUP, self.x[r], 1, self.idx[r][0],
                              self.cnt[r], self.yacc)
 
 
@@ -322,19 +354,38 @@ class GraphRunner:
             self.graphs[key] = g
         return self.graphs[key]
 
-    def prepare(self, n: int):
+    def _parts(self, n: int):
         full, rem = divmod(n, self.period)
-        if full:
-            self._graph(self.period, 0)
-        if rem:
-            self._graph(rem, 0)
+        return [self.period] * full + ([rem] if rem else [])
+
+    def prepare(self, n: int):
+        for length in set(self._parts(n)):
+            self._graph(length, 0)
+
+    def prewarm(self, n: int):
+        """Replays, once and untimed, every graph that run(n) replays (the
+        first replay of a graph uploads it to the device)."""
+        with torch.cuda.stream(self.stream):
+            for length in set(self._parts(n)):
+                self._graph(length, 0).replay()
+        torch.cuda.synchronize()
 
     def run(self, n: int):
-        full, rem = divmod(n, self.period)
-        for _ in range(full):
-            self._graph(self.period, 0).replay()
-        if rem:
-            self._graph(rem, 0).replay()
+        for length in self._parts(n):
+            self._graph(length, 0).replay()
+
+
+# Launches for every kernel-alone or call-alone timing, whatever --steps is.
+FIXED_LAUNCHES = 2000
+
+
+def device_delay(stream, us: float = 300.0):
+    """A bounded spin (torch's own sleep kernel, a fixed number of clock
+    cycles) enqueued before a start event, so that the host's submission of
+    the timed graphs happens while the device is still busy and is not inside
+    the event window."""
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(int(us * 2.0e3))   # cycles at ~2 GHz
 
 
 def whole_job(bytes_local: float, ms_local: float, dist: Dist):
@@ -345,11 +396,14 @@ def whole_job(bytes_local: float, ms_local: float, dist: Dist):
 
 
 def time_calls(fn, n: int, period: int, dist: Dist | None = None, warm: int = 3):
-    """Device time (ms) of exactly n calls of fn(i), via CUDA graphs."""
+    """Device time (ms) of exactly n calls of fn(i), via CUDA graphs: every
+    graph replayed once untimed, warm-up calls, then a bounded device delay
+    ahead of the start event and the n calls."""
     stream = torch.cuda.Stream()
     gr = GraphRunner(fn, period, stream)
     gr.prepare(n)
     gr.prepare(max(warm, 1))
+    gr.prewarm(n)
     with torch.cuda.stream(stream):
         gr.run(max(warm, 1))
     torch.cuda.synchronize()
@@ -358,6 +412,7 @@ def time_calls(fn, n: int, period: int, dist: Dist | None = None, warm: int = 3)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    device_delay(stream)
     with torch.cuda.stream(stream):
         e0.record(stream)
         gr.run(n)
@@ -386,10 +441,14 @@ def run_ours(args, dist: Dist):
     period = R * max(1, 64 // R)
 
     # warm-up (untimed) then exactly K timed steps
+    # (every graph of the timed region is replayed once before the warm-up,
+    # so the timed replays are not the graphs' first; a bounded device delay
+    # ahead of the start event keeps the host's submission out of the window)
     stream = torch.cuda.Stream()
     runner = GraphRunner(lambda i: rep.step(i % R, path), period, stream)
     runner.prepare(args.steps)
     runner.prepare(args.warmup)
+    runner.prewarm(args.steps)
     with torch.cuda.stream(stream):
         runner.run(args.warmup)
     torch.cuda.synchronize()
@@ -397,6 +456,7 @@ def run_ours(args, dist: Dist):
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(dist.local) as clk:
+        device_delay(stream)
         with torch.cuda.stream(stream):
             e0.record(stream)
             runner.run(args.steps)
@@ -412,16 +472,10 @@ def run_ours(args, dist: Dist):
     # split-K sums into an fp32 buffer, so no epilogue kernel follows it);
     # the mask path has no accumulating form and is timed as the whole call
     dom = {"thresh": "thresh_acc", "list": "gemv_acc", "mask": "mask"}[path]
-    nk = max(args.steps, 2 * R)
+    nk = FIXED_LAUNCHES
     kms = time_calls(lambda i: rep.kernel_only(i % R, dom), nk, period)
     k_us = kms * 1e3 / nk
-    k_bytes = sum(rep.abytes[i % R] for i in range(nk)) / nk
-    if dom == "thresh_acc":   # reads all of x, no index list; fp32 y
-        k_bytes = k_bytes - 6 * np.mean(rep.active) + 2 * K + 2 * N
-    elif dom == "gemv_acc":   # fp32 y
-        k_bytes = k_bytes + 2 * N
-    elif dom == "mask":   # K/8 bytes of mask instead of the 4a-byte index list
-        k_bytes = k_bytes - 4 * np.mean(rep.active) + K // 8
+    k_bytes = rep.kernel_bytes(dom)
     peak, peak_kind = measured_peak()
     rpk = read_peak_gbs()
     achieved = k_bytes / (k_us * 1e-6) / 1e9
@@ -442,7 +496,7 @@ def run_ours(args, dist: Dist):
                          if dom != "mask" else "the sgq_gemv_mask call (GEMV + epilogue kernel)"}
 
     # comparison points on the same rotation: dense int4 GEMV, select alone
-    nc = max(min(args.steps, 4000), 2 * period)
+    nc = FIXED_LAUNCHES
     dense_ms = time_calls(lambda i: rep.kernel_only(i % R, "dense"), nc, period)
     sel_ms = time_calls(lambda i: rep.kernel_only(i % R, "select"), nc, period)
     cmp_us = {}
@@ -450,7 +504,11 @@ def run_ours(args, dist: Dist):
         cms = time_calls(lambda i: rep.kernel_only(i % R, name), nc, period)
         cmp_us[name] = round(cms * 1e3 / nc, 3)
 
-    e2e = run_e2e(rep, path, min(args.steps, 2000), args.warmup, dist)
+    e2e = run_e2e(rep, path, 500, args.warmup, dist)
+    sweep = None if args.no_ffn else run_sweep(rep)
+    rep.set_sparsity(args.sparsity)
+    reglu = None if args.no_ffn else run_reglu()
+    tiny = None if args.no_ffn else run_tiny()
     layer = None if args.no_ffn else run_layer()
     batch = None if args.no_ffn else run_batch()
     nm = None if args.no_ffn else run_nm()
@@ -487,6 +545,12 @@ def run_ours(args, dist: Dist):
         line["batch_ffn"] = batch
     if nm is not None:
         line["nm_2of4"] = nm
+    if sweep is not None:
+        line["sparsity_sweep"] = sweep
+    if reglu is not None:
+        line["reglu_ffn"] = reglu
+    if tiny is not None:
+        line["tiny"] = tiny
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     return line
@@ -718,6 +782,164 @@ def run_layer(n_steps: int = 1000):
     }
 
 
+def run_sweep(rep: "Replica", sparsities=wl.SPARSITY_SWEEP):
+    """The same down_proj GEMV over the sparsity sweep: per sparsity, the bf16
+    call (fused threshold GEMV + epilogue kernel) and the GEMV kernel alone
+    (accumulating form), each over FIXED_LAUNCHES launches on the rotation,
+    with the kernel's roofline fraction on its algorithmic bytes."""
+    peak, _ = measured_peak()
+    R = rep.R
+    period = R * max(1, 64 // R)
+    rows = []
+    for sp in sparsities:
+        rep.set_sparsity(sp)
+        n = FIXED_LAUNCHES
+        call_us = time_calls(lambda i: rep.kernel_only(i % R, "thresh"), n, period) * 1e3 / n
+        k_us = time_calls(lambda i: rep.kernel_only(i % R, "thresh_acc"), n, period) * 1e3 / n
+        kb = rep.kernel_bytes("thresh_acc")
+        cb = rep.kernel_bytes("thresh")
+        rows.append({"sparsity": sp, "active_channels": int(np.mean(rep.active)),
+                     "us_per_gemv": round(call_us, 3), "kernel_us": round(k_us, 3),
+                     "algorithmic_bytes": int(kb),
+                     "GBps_call": round(cb / (call_us * 1e-6) / 1e9, 1),
+                     "GBps_kernel": round(kb / (k_us * 1e-6) / 1e9, 1),
+                     "frac_kernel": round(kb / (k_us * 1e-6) / 1e9 / peak, 4),
+                     "frac_kernel_of_8TBps": round(kb / (k_us * 1e-6) / 1e9 / 8000.0, 4)})
+    return {"workload": "Llama-3-8B down_proj (K=14336, N=4096, int4 g128), x = SiLU(g)*u, "
+                        "batch 1, magnitude threshold at each sparsity; fused select",
+            "rows": rows, "launches_per_row": FIXED_LAUNCHES,
+            "rotation": f"{R} copies, {rep.bytes_resident / 1e6:.0f} MB"}
+
+
+class ReGluReplica:
+    """R copies of a ReGLU FFN (hidden 4096, intermediate 11008, int4 g128):
+    stacked [W_g; W_u] and W_d; R x bytes > 4x L2. x ~ N(0, 1) (dense: every
+    channel of the gate/up input is read), h = ReLU(W_g x) * (W_u x) whose
+    zeros the down projection skips (t = 0). Random weights leave about half
+    of h zero; the stand-in h = ReLU(g - beta) * u with 88% zeros stands for a
+    trained ReGLU model's ~90%."""
+
+    def __init__(self, seed: int = 21):
+        cfg = wl.REGLU_FFN
+        self.H, self.I, self.g = cfg["hidden"], cfg["inter"], cfg["group"]
+        H, I, g = self.H, self.I, self.g
+        gu = self._pack(torch.cat([wl.weight(I, H, seed), wl.weight(I, H, seed + 1)], 0))
+        down = self._pack(wl.weight(H, I, seed + 2))
+        per = sum(a.numel() * a.element_size() for t in (gu, down) for a in t)
+        l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+        self.R = max(2, int(math.ceil(4 * l2 / per)) + 1)
+        self.gu = [gu] + [tuple(a.clone() for a in gu) for _ in range(self.R - 1)]
+        self.down = [down] + [tuple(a.clone() for a in down) for _ in range(self.R - 1)]
+        self.bytes_resident = self.R * per
+        self.x = [wl.x_gaussian(1, H, 5000 + r).cuda() for r in range(self.R)]
+        self.h88 = [wl.x_relu_shifted(1, I, 6000 + r).cuda() for r in range(self.R)]
+        self.h = torch.empty(1, I, dtype=torch.bfloat16, device="cuda")
+        self.hs = torch.empty(1, I, dtype=torch.bfloat16, device="cuda")
+        self.y = torch.empty(1, H, dtype=torch.bfloat16, device="cuda")
+        self.ws = sgq.alloc_workspace(2 * I, max(H, I), 1)
+        self.wsf = sgq.alloc_ffn_workspace(H, I)
+        idx, cnt = sgq.alloc_select(I)
+        # gate/up (dense) bytes and down bytes at each h
+        gub = 2 * I * H // 2 + (H // g) * 2 * I * 4 + 2 * H
+        self.nat_down, self.s88_down, self.nat_frac, self.s88_frac = [], [], [], []
+        for r in range(self.R):
+            self.gate_up(r, self.h)
+            for hv, out, fr in ((self.h, self.nat_down, self.nat_frac),
+                                (self.h88[r], self.s88_down, self.s88_frac)):
+                sgq.sgq_select(hv, 1, I, [0.0], idx, cnt)
+                a = int(cnt.item())
+                gr = int(np.unique(idx[:a].cpu().numpy() // g).size)
+                out.append(a * H // 2 + gr * H * 4 + 2 * I + 2 * H)
+                fr.append(1.0 - a / I)
+        self.gu_bytes = gub
+        torch.cuda.synchronize()
+
+    def _pack(self, W):
+        N, K = W.shape
+        qw, sz = sgq.alloc_packed(N, K, self.g)
+        sgq.sgq_pack(W.cuda(), N, K, self.g, qw, sz)
+        return qw, sz
+
+    def gate_up(self, r, h):
+        qw, sz = self.gu[r]
+        sgq.sgq_gemv_glu_dense(qw, sz, self.I, self.H, self.g, self.x[r], 1, sgq.SGQ_ACT_RELU,
+                               h, None, self.ws)
+
+    def ffn_natural(self, r):                    # 3 launches: sgq_ffn
+        qg, sg = self.gu[r]
+        qd, sd = self.down[r]
+        sgq.sgq_ffn(qg, sg, qd, sd, self.H, self.I, self.g, self.x[r], -1.0, sgq.SGQ_ACT_RELU,
+                    0.0, self.y, None, None, self.wsf)
+
+    def ffn_standin(self, r):                    # 4 launches
+        self.gate_up(r, self.hs)
+        qd, sd = self.down[r]
+        sgq.sgq_gemv_thresh(qd, sd, self.H, self.I, self.g, self.h88[r], 0.0, self.y, None,
+                            self.ws)
+
+    def down_only(self, r, h):
+        qd, sd = self.down[r]
+        sgq.sgq_gemv_thresh(qd, sd, self.H, self.I, self.g, h, 0.0, self.y, None, self.ws)
+
+
+def run_reglu():
+    """us per ReGLU FFN (natural ReLU zeros and the 88% stand-in) and per down
+    projection alone, each over FIXED_LAUNCHES calls on the rotation."""
+    f = ReGluReplica()
+    R = f.R
+    period = R * max(1, 32 // R)
+    n = FIXED_LAUNCHES
+    peak, _ = measured_peak()
+    us = {"ffn_natural": time_calls(lambda i: f.ffn_natural(i % R), n, period) * 1e3 / n,
+          "ffn_standin": time_calls(lambda i: f.ffn_standin(i % R), n, period) * 1e3 / n}
+    # the down projection alone over the stand-in h (per copy) and over the
+    # natural h of copy 0 (gate/up output, computed once)
+    f.gate_up(0, f.h)
+    us["down_natural"] = time_calls(lambda i: f.down_only(i % R, f.h), n, period) * 1e3 / n
+    us["down_standin"] = time_calls(lambda i: f.down_only(i % R, f.h88[i % R]), n,
+                                    period) * 1e3 / n
+    nat = f.gu_bytes + float(np.mean(f.nat_down))
+    s88 = f.gu_bytes + float(np.mean(f.s88_down))
+    return {"workload": "ReGLU FFN decode, batch 1: hidden 4096, intermediate 11008, int4 "
+                        "g128; x ~ N(0,1) dense into the stacked gate/up GEMV with the ReLU "
+                        "GLU; down_proj over h's nonzeros (t = 0)",
+            "h_zero_frac_natural": round(float(np.mean(f.nat_frac)), 3),
+            "h_zero_frac_standin": round(float(np.mean(f.s88_frac)), 3),
+            "us_per_ffn_natural": round(us["ffn_natural"], 3), "launches_natural": 3,
+            "us_per_ffn_standin": round(us["ffn_standin"], 3), "launches_standin": 4,
+            "active_bytes_natural": int(nat), "active_bytes_standin": int(s88),
+            "GBps_natural": round(nat / (us["ffn_natural"] * 1e-6) / 1e9, 1),
+            "GBps_standin": round(s88 / (us["ffn_standin"] * 1e-6) / 1e9, 1),
+            "down_us_natural": round(us["down_natural"], 3),
+            "down_us_standin": round(us["down_standin"], 3),
+            "down_frac_standin": round(float(np.mean(f.s88_down)) /
+                                       (us["down_standin"] * 1e-6) / 1e9 / peak, 4),
+            "note": "natural: sgq_ffn (h formed and selected inside the down projection); "
+                    "stand-in: the gate/up GLU GEMV, then the down GEMV over a synthetic h "
+                    "with 88% zeros (h = ReLU(g - beta) * u, not the GLU's output)",
+            "rotation": f"{R} copies, {f.bytes_resident / 1e6:.0f} MB"}
+
+
+def run_tiny():
+    """The tiny GEMV (K=256, N=512, g64, 50%): latency of one fused call (its
+    48 KB of inputs stay in L2; correctness case, not a bandwidth case)."""
+    shp = wl.TINY
+    n_, k_, g_ = shp["N"], shp["K"], shp["group"]
+    case = wl.gemv_case(n_, k_, g_, sparsity=0.5, seed=0)
+    qw, sz = sgq.alloc_packed(n_, k_, g_)
+    sgq.sgq_pack(case.W.cuda(), n_, k_, g_, qw, sz)
+    x = case.x.cuda()
+    y = torch.empty(1, n_, dtype=torch.bfloat16, device="cuda")
+    ws = sgq.alloc_workspace(n_, k_, 1)
+    t = case.t[0]
+    n = FIXED_LAUNCHES
+    us = time_calls(lambda i: sgq.sgq_gemv_thresh(qw, sz, n_, k_, g_, x, t, y, None, ws), n,
+                    64) * 1e3 / n
+    return {"workload": "tiny GEMV K=256, N=512, int4 g64, x ~ N(0,1), 50% sparsity, fused "
+                        "select; inputs resident in L2 (latency only)",
+            "us_per_gemv": round(us, 3), "launches": n}
+
+
 class BatchFfnReplica:
     """R copies of one Qwen3-32B FFN (hidden 5120, intermediate 25600, int4
     g128): stacked [W_g; W_u] and W_d; R x bytes > 4x L2. At batch B, x has B
@@ -862,51 +1084,65 @@ class OracleSample:
         self.a = int(idx.size)
         self.groups = int(np.unique(idx // GROUP).size)
 
-    def run(self, rows: np.ndarray):
-        """select + GEMV for the given outputs; returns the active bytes covered."""
+    def run(self, rows: np.ndarray, threads: int | None = None):
+        """select + GEMV for the given outputs (on `threads` OpenMP threads, or
+        the one-thread form); returns the active bytes covered."""
         idx = self.o.select(self.xb, self.t)
-        self.o.gemv(self.q[rows], self.s[rows], self.z[rows], GROUP, self.xb, idx)
+        self.o.gemv(self.q[rows], self.s[rows], self.z[rows], GROUP, self.xb, idx,
+                    threads=threads)
         n = len(rows)
         return active_bytes(self.a, self.groups, n=n)
 
 
-def cpu_cores_used():
-    return 1   # the oracle is single-threaded C
+def host_cores() -> int:
+    return len(os.sched_getaffinity(0))
 
 
 def cpu_baseline(seconds: float):
+    """The oracle's select + GEMV on the benchmark workload, timed twice on the
+    host: the one-thread form, and the OpenMP form over every core of the
+    affinity mask (each output keeps its summation order: same results). Each
+    runs whole GEMVs for about `seconds` (at most 50)."""
     smp = OracleSample(0.5)
     rows = np.arange(N)
-    done, t0 = 0, time.perf_counter()
-    reps = 0
-    while True:
-        done += smp.run(rows)
-        reps += 1
-        el = time.perf_counter() - t0
-        if el >= seconds or reps >= 50:
-            break
-    return {"value": round(done / el / 1e9, 3), "unit": UNIT, "cores": cpu_cores_used(),
-            "kind": "oracle",
-            "sample": f"{reps} full GEMVs (select + fp64 GEMV, all {N} outputs) in {el:.1f} s, "
-                      f"host has {len(os.sched_getaffinity(0))} cores"}
+    cores = host_cores()
+
+    def timed(threads):
+        done, reps, t0 = 0, 0, time.perf_counter()
+        while True:
+            done += smp.run(rows, threads)
+            reps += 1
+            el = time.perf_counter() - t0
+            if el >= seconds or reps >= 50:
+                return done / el / 1e9, reps, el
+
+    v1, r1, e1 = timed(None)
+    vm, rm, em = timed(cores)
+    return {"value": round(vm, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{rm} full GEMVs (select + fp64 GEMV, all {N} outputs) in {em:.1f} s "
+                      f"on {cores} OpenMP threads (outputs shared out, sums unchanged)",
+            "single_thread": {"value": round(v1, 4), "unit": UNIT, "cores": 1,
+                              "sample": f"{r1} full GEMVs in {e1:.1f} s on one thread"}}
 
 
 def run_reference(args, dist: Dist):
-    """The reference arm: the CPU oracle as it stands, on a bounded sample of
-    the workload per step (a slice of the outputs), K steps after W warm-up."""
+    """The reference arm: the CPU oracle as it stands (its OpenMP form on every
+    core of the affinity mask), on a bounded sample of the workload per step
+    (a slice of the outputs), K steps after W warm-up."""
     smp = OracleSample(args.sparsity)
-    budget = max(60.0, 0.0) / max(args.steps + args.warmup, 1)
+    cores = host_cores()
+    budget = 60.0 / max(args.steps + args.warmup, 1)
     t0 = time.perf_counter()
-    smp.run(np.arange(8))
-    per_row = (time.perf_counter() - t0) / 8
+    smp.run(np.arange(8 * cores), cores)
+    per_row = (time.perf_counter() - t0) / (8 * cores)
     nrows = int(max(1, min(N, budget / max(per_row, 1e-9))))
     rng = np.random.default_rng(0)
     for _ in range(args.warmup):
-        smp.run(np.sort(rng.choice(N, nrows, replace=False)))
+        smp.run(np.sort(rng.choice(N, nrows, replace=False)), cores)
     done = 0
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        done += smp.run(np.sort(rng.choice(N, nrows, replace=False)))
+        done += smp.run(np.sort(rng.choice(N, nrows, replace=False)), cores)
     el = time.perf_counter() - t0
     value = done / el / 1e9
     return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT,
@@ -915,8 +1151,9 @@ def run_reference(args, dist: Dist):
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": WORKLOAD, "K": K, "N": N, "group": GROUP, "batch": 1,
                        "sparsity": args.sparsity,
-                       "path": "CPU oracle: select + fp64 GEMV (plain C, one thread)"},
-            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cpu_cores_used(),
+                       "path": f"CPU oracle: select + fp64 GEMV (plain C, OpenMP over the "
+                               f"outputs, {cores} threads)"},
+            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores,
                              "kind": "oracle",
                              "sample": f"each step: {nrows} of {N} outputs of the GEMV"},
             "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,

@@ -329,10 +329,13 @@ int sgq_ffn(const void *qweight_gu, const void *sz_gu, const void *qweight_d, co
  * The split-K scratch is a fixed array of SGQ_NOALLOC_MAX_N floats compiled
  * into the library (held on every GPU that loads it until the process exits).
  * N > SGQ_NOALLOC_MAX_N returns SGQ_ERR_TOO_LARGE. The first call on a device
- * looks up the array's device address and clears it (synchronously), so make
- * that first call before any stream capture. Every call leaves the array at
- * zero again; calls that overlap on the GPU share the array and race. Nothing
- * is allocated or freed. Other arguments as sgq_gemv_thresh.
+ * (that device current) looks up the array's device address once
+ * (cudaGetSymbolAddress, thread-safe) and caches it, so make that first call
+ * before any stream capture; the cached address is not valid across a
+ * cudaDeviceReset. Every call clears the N floats it uses with
+ * cudaMemsetAsync on `stream` before the GEMV, so it never depends on what an
+ * earlier call left there; calls that overlap on the GPU share the array and
+ * race. Nothing is allocated or freed. Other arguments as sgq_gemv_thresh.
  */
 #define SGQ_NOALLOC_MAX_N 65536
 int sgq_gemv_thresh_noalloc(const void *qweight, const void *sz, int N, int K, int group,

@@ -29,7 +29,8 @@ _SRC = os.path.join(_HERE, "sgq_oracle.c")
 _HDR = os.path.join(_HERE, "sgq_oracle.h")
 LIB_PATH = os.path.join(_HERE, "libsgq_oracle.so")
 
-CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
+CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
+          "-fopenmp"]
 
 _lib = None
 _lock = threading.Lock()
@@ -93,13 +94,14 @@ def _declare(lib):
     lib.oracle_select.argtypes = [P, i, i, P, P, P]
     lib.oracle_gemv.argtypes = [P, P, P, i, i, i, P, i, P, i, P, P, P]
     lib.oracle_gemv_dense.argtypes = [P, P, P, i, i, i, P, i, P, P, P]
+    lib.oracle_gemv_threads.argtypes = [P, P, P, i, i, i, P, i, P, i, P, P, P, i]
     lib.oracle_glu.argtypes = [P, P, ctypes.c_int64, i, P, P]
     lib.oracle_act_mul.argtypes = [P, P, ctypes.c_int64, i, P, P]
     lib.oracle_select_mask.argtypes = [P, i, i, P, P, P]
     lib.oracle_nm_keep.argtypes = [P, i, i, i, P, P]
     lib.oracle_pack_layout_nm.argtypes = [P, P, P, P, P, i, i, i, P, P, P]
     for f in ("oracle_quantize", "oracle_pack_layout", "oracle_select",
-              "oracle_gemv", "oracle_gemv_dense", "oracle_glu", "oracle_act_mul", "oracle_select_mask", "oracle_nm_keep",
+              "oracle_gemv", "oracle_gemv_threads", "oracle_gemv_dense", "oracle_glu", "oracle_act_mul", "oracle_select_mask", "oracle_nm_keep",
               "oracle_pack_layout_nm"):
         getattr(lib, f).restype = ctypes.c_int
     return lib
@@ -193,8 +195,10 @@ def select(x_bits, t, lib=None):
     return idx[: int(cnt[0])].copy()
 
 
-def gemv(q, s, z, g, x_bits, idx, lib=None):
-    """Returns (y f64 [B,N], sumabs f64 [B,N], y_bf16 u16 [B,N])."""
+def gemv(q, s, z, g, x_bits, idx, lib=None, threads=None):
+    """Returns (y f64 [B,N], sumabs f64 [B,N], y_bf16 u16 [B,N]). With
+    ``threads`` the outputs are shared over that many OpenMP threads (same
+    results bit for bit)."""
     lib = lib or load()
     q = _c(q, np.uint8)
     s = _c(s, np.uint16)
@@ -206,9 +210,12 @@ def gemv(q, s, z, g, x_bits, idx, lib=None):
     y = np.empty((B, N), np.float64)
     sa = np.empty((B, N), np.float64)
     yb = np.empty((B, N), np.uint16)
-    _check(lib.oracle_gemv(q.ctypes.data, s.ctypes.data, z.ctypes.data, N, K, g,
-                           x.ctypes.data, B, idx.ctypes.data, int(idx.size),
-                           y.ctypes.data, sa.ctypes.data, yb.ctypes.data), "oracle_gemv")
+    args = (q.ctypes.data, s.ctypes.data, z.ctypes.data, N, K, g, x.ctypes.data, B,
+            idx.ctypes.data, int(idx.size), y.ctypes.data, sa.ctypes.data, yb.ctypes.data)
+    if threads is None:
+        _check(lib.oracle_gemv(*args), "oracle_gemv")
+    else:
+        _check(lib.oracle_gemv_threads(*args, int(threads)), "oracle_gemv_threads")
     return y, sa, yb
 
 

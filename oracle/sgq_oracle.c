@@ -347,39 +347,75 @@ int oracle_select_mask(const uint16_t *x, int B, int K, const float *t,
 /* to the active channels). Every row of a batch uses the same active set.   */
 /* ------------------------------------------------------------------------- */
 
+/* Output n of batch row b over the listed channels, in list order. */
+static void gemv_output(const uint8_t *q, const uint16_t *s, const uint16_t *z,
+                        int N, int K, int g, const uint16_t *x, int b, int n,
+                        const int32_t *idx, int count,
+                        double *y, double *sumabs, uint16_t *y_bf16)
+{
+    int G = K / g;
+    double acc = 0.0, acc_abs = 0.0;
+    for (int i = 0; i < count; ++i) {
+        int k = idx[i];
+        int grp = k / g;
+        double sv = oracle_half_to_double(s[(size_t)n * G + grp]);
+        double zv = oracle_half_to_double(z[(size_t)n * G + grp]);
+        double w = sv * ((double)q[(size_t)n * K + k] - zv);
+        double p = w * oracle_bf16_to_double(x[(size_t)b * K + k]);
+        acc += p;
+        acc_abs += fabs(p);
+    }
+    size_t o = (size_t)b * N + n;
+    if (y)
+        y[o] = acc;
+    if (sumabs)
+        sumabs[o] = acc_abs;
+    if (y_bf16)
+        y_bf16[o] = oracle_double_to_bf16(acc);
+}
+
+static int gemv_args_ok(int N, int K, int g, int B, const int32_t *idx, int count)
+{
+    if (N <= 0 || K <= 0 || g <= 0 || K % g != 0 || B <= 0 || count < 0 || count > K)
+        return -2;
+    for (int i = 0; i < count; ++i)
+        if (idx[i] < 0 || idx[i] >= K)
+            return -3;
+    return 0;
+}
+
 int oracle_gemv(const uint8_t *q, const uint16_t *s, const uint16_t *z,
                 int N, int K, int g, const uint16_t *x, int B,
                 const int32_t *idx, int count,
                 double *y, double *sumabs, uint16_t *y_bf16)
 {
-    if (N <= 0 || K <= 0 || g <= 0 || K % g != 0 || B <= 0 || count < 0 || count > K)
+    int rc = gemv_args_ok(N, K, g, B, idx, count);
+    if (rc)
+        return rc;
+    for (int b = 0; b < B; ++b)
+        for (int n = 0; n < N; ++n)
+            gemv_output(q, s, z, N, K, g, x, b, n, idx, count, y, sumabs, y_bf16);
+    return 0;
+}
+
+/* The same GEMV with the outputs shared out over `threads` OpenMP threads.
+ * Each output is still one sum in list order by one thread, so the results
+ * are bit-identical to oracle_gemv; only the wall time changes. */
+int oracle_gemv_threads(const uint8_t *q, const uint16_t *s, const uint16_t *z,
+                        int N, int K, int g, const uint16_t *x, int B,
+                        const int32_t *idx, int count,
+                        double *y, double *sumabs, uint16_t *y_bf16, int threads)
+{
+    int rc = gemv_args_ok(N, K, g, B, idx, count);
+    if (rc)
+        return rc;
+    if (threads < 1)
         return -2;
-    int G = K / g;
-    for (int i = 0; i < count; ++i)
-        if (idx[i] < 0 || idx[i] >= K)
-            return -3;
-    for (int b = 0; b < B; ++b) {
-        for (int n = 0; n < N; ++n) {
-            double acc = 0.0, acc_abs = 0.0;
-            for (int i = 0; i < count; ++i) {
-                int k = idx[i];
-                int grp = k / g;
-                double sv = oracle_half_to_double(s[(size_t)n * G + grp]);
-                double zv = oracle_half_to_double(z[(size_t)n * G + grp]);
-                double w = sv * ((double)q[(size_t)n * K + k] - zv);
-                double p = w * oracle_bf16_to_double(x[(size_t)b * K + k]);
-                acc += p;
-                acc_abs += fabs(p);
-            }
-            size_t o = (size_t)b * N + n;
-            if (y)
-                y[o] = acc;
-            if (sumabs)
-                sumabs[o] = acc_abs;
-            if (y_bf16)
-                y_bf16[o] = oracle_double_to_bf16(acc);
-        }
-    }
+    long long total = (long long)B * N;
+#pragma omp parallel for num_threads(threads) schedule(static)
+    for (long long o = 0; o < total; ++o)
+        gemv_output(q, s, z, N, K, g, x, (int)(o / N), (int)(o % N), idx, count, y, sumabs,
+                    y_bf16);
     return 0;
 }
 

@@ -77,6 +77,13 @@ int oracle_gemv(const uint8_t *q, const uint16_t *s, const uint16_t *z,
                 const int32_t *idx, int count,
                 double *y, double *sumabs, uint16_t *y_bf16);
 
+/* oracle_gemv with the B * N outputs shared out over `threads` OpenMP
+ * threads; every output keeps its sum order, so the results are identical. */
+int oracle_gemv_threads(const uint8_t *q, const uint16_t *s, const uint16_t *z,
+                        int N, int K, int g, const uint16_t *x, int B,
+                        const int32_t *idx, int count,
+                        double *y, double *sumabs, uint16_t *y_bf16, int threads);
+
 /* Same with every k of 0..K-1 (the dense quantized GEMV). */
 int oracle_gemv_dense(const uint8_t *q, const uint16_t *s, const uint16_t *z,
                       int N, int K, int g, const uint16_t *x, int B,

@@ -315,6 +315,25 @@ def pin_gemv_sparse_vs_masked_matmul(lib):
     assert np.all(np.abs(y[0] - ref) <= 1e-13 * sa[0] + 1e-300)
 
 
+def pin_gemv_threads(lib):
+    """The OpenMP form against numpy matmul of the masked activations, and bit
+    for bit against the one-thread form (each output keeps its sum order)."""
+    rng = np.random.default_rng(21)
+    N, K, g, B = 67, 384, 64, 3
+    q, s, z, x = _small_problem(rng, N, K, g, B)
+    xd = torch_bf16(x)
+    t = [float(np.median(np.abs(xd[b]))) for b in range(B)]
+    idx = oracle.select(x, t, lib)
+    mask = np.zeros(K)
+    mask[idx] = 1.0
+    ref = (xd * mask) @ dequant(q, s, z, g).T
+    y1, sa1, yb1 = oracle.gemv(q, s, z, g, x, idx, lib)
+    for threads in (1, 2, 5):
+        y, sa, yb = oracle.gemv(q, s, z, g, x, idx, lib, threads=threads)
+        assert np.all(np.abs(y - ref) <= 1e-13 * sa + 1e-300)
+        assert np.array_equal(y, y1) and np.array_equal(sa, sa1) and np.array_equal(yb, yb1)
+
+
 def pin_gemv_all_masked(lib):
     rng = np.random.default_rng(10)
     q, s, z, x = _small_problem(rng, 16, 128, 32, 2)

@@ -27,8 +27,8 @@ MUTANTS = {
                    "double c = clamp15(floor(w / sv) + zv);"),
     "scale_over_16": ("(hi - lo) / 15.0", "(hi - lo) / 16.0"),
     "range_without_zero": ("double lo = 0.0, hi = 0.0;", "double lo = INFINITY, hi = -INFINITY;"),
-    "drop_last_active": ("for (int i = 0; i < count; ++i) {\n                int k = idx[i];",
-                         "for (int i = 0; i < count - 1; ++i) {\n                int k = idx[i];"),
+    "drop_last_active": ("for (int i = 0; i < count; ++i) {\n        int k = idx[i];",
+                         "for (int i = 0; i < count - 1; ++i) {\n        int k = idx[i];"),
     "nibble_order": ("(uint8_t)(lo | (hi << 4))", "(uint8_t)(hi | (lo << 4))"),
     "ties_away_from_zero": ("return nearbyint(a / quantum) * quantum;",
                             "return round(a / quantum) * quantum;"),
@@ -52,6 +52,9 @@ MUTANTS = {
                       "qweight[(size_t)k * (N / 4) + j] = (uint8_t)(c1 | (c0 << 4));"),
     "act_mul_drops_up": ("double hv = oracle_act(gate[i], act) * up[i];",
                          "double hv = oracle_act(gate[i], act);"),
+    "threads_skip_last_output": ("for (long long o = 0; o < total; ++o)",
+                                 "for (long long o = 0; o < total - 1; ++o)"),
+    "threads_batch_forgotten": ("long long total = (long long)B * N;", "long long total = N;"),
     "act_mul_swapped": ("double hv = oracle_act(gate[i], act) * up[i];",
                         "double hv = oracle_act(up[i], act) * gate[i];"),
 }
