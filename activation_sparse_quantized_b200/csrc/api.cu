@@ -83,7 +83,7 @@ int run_gemv(sgq::GemvProblem &p, size_t ws_bytes, void *workspace, void *stream
     if (!aligned16(p.qweight) || !aligned16(p.sz) || !aligned16(p.x) || !aligned16(p.y) ||
         !aligned16(workspace) || (p.y_f32 && !aligned16(p.y_f32)))
         return SGQ_ERR_ALIGN;
-    if (p.source == sgq::ROWS_THRESH && (p.B != 1 || p.K % 8 != 0))
+    if (p.source == sgq::ROWS_THRESH && (p.K % 8 != 0 || (p.keep && p.B != 1)))
         return SGQ_ERR_SHAPE;
     if (ws_bytes < sgq::gemv_workspace_bytes(p.N, p.B))
         return SGQ_ERR_WORKSPACE;
@@ -344,6 +344,32 @@ int sgq_gemv_thresh(const void *qweight, const void *sz, int N, int K, int group
     return run_gemv(p, ws_bytes, workspace, stream);
 }
 
+int sgq_gemv_thresh_batch(const void *qweight, const void *sz, int N, int K, int group,
+                          const void *x, int B, const float *t_host, void *y, float *y_f32,
+                          void *workspace, size_t ws_bytes, int32_t *status, void *stream)
+{
+    if (B < 1 || B > SGQ_MAX_BATCH)
+        return SGQ_ERR_BATCH;
+    if (!t_host)
+        return SGQ_ERR_NULL;
+    sgq::GemvProblem p{};
+    p.qweight = static_cast<const uint8_t *>(qweight);
+    p.sz = static_cast<const uint32_t *>(sz);
+    p.x = static_cast<const uint16_t *>(x);
+    p.y = static_cast<uint16_t *>(y);
+    p.y_f32 = y_f32;
+    p.status = status;
+    p.N = N;
+    p.K = K;
+    p.group = group;
+    p.B = B;
+    p.t = t_host[0];
+    for (int b = 0; b < B; ++b)
+        p.tb[b] = t_host[b];
+    p.source = sgq::ROWS_THRESH;
+    return run_gemv(p, ws_bytes, workspace, stream);
+}
+
 // Accumulating forms: y_acc [B][N] fp32 (caller-owned) += the GEMV; the GEMV
 // kernel's split-K reductions land in y_acc itself, so there is no workspace
 // and no epilogue kernel.
@@ -535,6 +561,32 @@ int sgq_gemv_glu_thresh(const void *qweight, const void *sz, int I, int K, int g
     p.group = group;
     p.B = 1;
     p.t = t;
+    p.source = sgq::ROWS_THRESH;
+    return run_gemv_glu(p, I, act, ws_bytes, workspace, stream);
+}
+
+int sgq_gemv_glu_thresh_batch(const void *qweight, const void *sz, int I, int K, int group,
+                              const void *x, int B, const float *t_host, int act, void *h,
+                              float *h_f32, void *workspace, size_t ws_bytes, int32_t *status,
+                              void *stream)
+{
+    if (B < 1 || B > SGQ_MAX_BATCH)
+        return SGQ_ERR_BATCH;
+    if (!t_host)
+        return SGQ_ERR_NULL;
+    sgq::GemvProblem p{};
+    p.qweight = static_cast<const uint8_t *>(qweight);
+    p.sz = static_cast<const uint32_t *>(sz);
+    p.x = static_cast<const uint16_t *>(x);
+    p.y = static_cast<uint16_t *>(h);
+    p.y_f32 = h_f32;
+    p.status = status;
+    p.K = K;
+    p.group = group;
+    p.B = B;
+    p.t = t_host[0];
+    for (int b = 0; b < B; ++b)
+        p.tb[b] = t_host[b];
     p.source = sgq::ROWS_THRESH;
     return run_gemv_glu(p, I, act, ws_bytes, workspace, stream);
 }

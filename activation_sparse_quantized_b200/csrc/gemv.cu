@@ -270,10 +270,11 @@ __device__ __forceinline__ int part_chunk16(int l, int c)
 // NM: the 2:4 layout (batch 1): the codes of a row are the kept outputs'
 // slots, 1024 slots = 2048 outputs per tile, 64 outputs per lane; the fold
 // adds each slot's sum to its output through the group's keep nibbles.
-// SEG (index list only): instead of (tile, split) from the block index, the
-// CTA takes an equal share of the (tile, list entry) space, which may end one
-// tile and start the next; each part (segment) runs the whole body in turn,
-// adding into the workspace.
+// SEG (index list, or the batch-row threshold): instead of (tile, split) from
+// the block index, the CTA takes an equal share of the (tile, list entry)
+// space, or of the (tile, 8-channel unit) space, which may end one tile and
+// start the next; each part (segment) runs the whole body in turn, adding into
+// the workspace.
 template <int SRC, int BW, bool NM = false, bool SEG = false>
 __global__ void __launch_bounds__(kThreads1, 1) gemv_kernel(const KParams kp)
 {
@@ -297,11 +298,15 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_kernel(const KParams kp)
     int su = 0, su1 = 1, per_tile = 1;
     if constexpr (SEG) {
         grid_launch_dependents();
-        grid_dependency_wait(); // x, idx, count may come from the previous kernel
-        const int c = __ldg(p.count);
-        per_tile = c < 0 ? 0 : (c > p.K ? p.K : c);
-        if (per_tile != c && tid == 0 && blockIdx.x == 0)
-            set_status(p.status, SGQ_STATUS_BAD_COUNT);
+        if constexpr (SRC == ROWS_LIST) {
+            grid_dependency_wait(); // x, idx, count may come from the previous kernel
+            const int c = __ldg(p.count);
+            per_tile = c < 0 ? 0 : (c > p.K ? p.K : c);
+            if (per_tile != c && tid == 0 && blockIdx.x == 0)
+                set_status(p.status, SGQ_STATUS_BAD_COUNT);
+        } else {
+            per_tile = p.K / 8; // channel units
+        }
         const long long W = (long long)kp.n_tiles * per_tile;
         su = (int)(W * blockIdx.x / gridDim.x);
         su1 = (int)(W * (blockIdx.x + 1) / gridDim.x);
@@ -347,7 +352,10 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_kernel(const KParams kp)
         };
         if (SRC != ROWS_LIST) {
             int c0, c1;
-            if (SRC == ROWS_THRESH || SRC == ROWS_MASK || SRC == ROWS_GLU) {
+            if (SEG) {
+                c0 = 8 * seg_lo; // the segment's channel units (threshold source)
+                c1 = 8 * seg_hi;
+            } else if (SRC == ROWS_THRESH || SRC == ROWS_MASK || SRC == ROWS_GLU) {
                 channel_slice(kp, split, c0, c1);
             } else {
                 c0 = (int)((long long)p.K * split / kp.k_splits);
@@ -356,11 +364,23 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_kernel(const KParams kp)
             if (c1 > c0) {
                 G0 = c0 >> lg;
                 span = min(((c1 - 1) >> lg) - G0 + 1, kp.span_cap);
+                // The slice of the input this CTA reads right after the wait
+                // (x of each batch row, the gate/up sums, or the mask words),
+                // requested into L2 now: a hint only, the loads after the wait
+                // still see whatever the previous kernel wrote.
+                if (warp == 0) {
+                    if (SRC == ROWS_THRESH && lane < p.B)
+                        prefetch_l2_bulk(p.x + (size_t)lane * p.K + c0, 2u * (uint32_t)(c1 - c0));
+                    if (SRC == ROWS_GLU && lane < 2)
+                        prefetch_l2_bulk(p.gu + (size_t)lane * p.K + c0, 4u * (uint32_t)(c1 - c0));
+                    if (SRC == ROWS_MASK)
+                        prefetch_l2_lines(p.mask + (c0 >> 5), p.mask + ((c1 - 1) >> 5) + 1);
+                }
             }
             stage_sz();
         }
 
-        if constexpr (!SEG)
+        if constexpr (!SEG || SRC != ROWS_LIST)
             grid_dependency_wait(); // x, idx, count, mask may come from the previous kernel
 
         // Rows (build_rows ends with a barrier). Invalid list entries stay -1: they
@@ -401,7 +421,7 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv_kernel(const KParams kp)
         // x of this warp's rows and batch rows (after the weights are in flight),
         // unless build_rows already read it (threshold; bitmask at batch 1).
         // Padded batch rows and invalid list entries get x = 0.
-        if (!(SRC == ROWS_THRESH || SRC == ROWS_GLU || (SRC == ROWS_MASK && BW == 1))) {
+        if (!((SRC == ROWS_THRESH && BW == 1) || SRC == ROWS_GLU || (SRC == ROWS_MASK && BW == 1))) {
             for (int e = lane; e < n * BW; e += 32) {
                 const int j = e / BW, bb = e - j * BW;
                 const int k = ridx[wa + j];
@@ -701,30 +721,36 @@ cudaError_t launch_gemv_t(KParams kp, int num_sms, cudaStream_t stream)
         kp.span_cap = std::min(G, ceil_div(p.K, (long long)kp.k_splits << kp.lg) + 2);
         L = smem1_layout(kp.span_cap, kp.rows_cap, bp, BW, NM);
         // the threshold path handles at most 4 runs of 32 channels per warp
-        const bool fused_select = (SRC == ROWS_THRESH || SRC == ROWS_GLU);
+        // (the batch-1 threshold / GLU prologue keeps up to 4 runs of 32
+        // channels per warp in registers; the batch-row union has no limit)
+        const bool fused_select = (SRC == ROWS_THRESH || SRC == ROWS_GLU) && BW == 1;
         const bool runs_ok = !fused_select || (kp.rows_cap <= 4 * kThreads1);
         if ((L.total <= kMaxSmem && runs_ok) || kp.k_splits >= p.K / 8)
             break;
         kp.k_splits *= 2;
     }
     if (L.total > kMaxSmem ||
-        ((SRC == ROWS_THRESH || SRC == ROWS_GLU) && kp.rows_cap > 4 * kThreads1))
+        ((SRC == ROWS_THRESH || SRC == ROWS_GLU) && BW == 1 && kp.rows_cap > 4 * kThreads1))
         return cudaErrorInvalidConfiguration;
     // Index list on a tile count that whole splits per tile cannot spread
     // over 90% of the SMs (e.g. 50 tiles: 100 of 148 CTAs), or that needs
     // more than one wave: one equal share of the (tile, list entry) space per
     // SM instead (segments, see gemv_kernel).
-    if constexpr (SRC == ROWS_LIST && !NM) {
+    if constexpr ((SRC == ROWS_LIST || (SRC == ROWS_THRESH && BW == 2)) && !NM) {
         const long long ctas = (long long)kp.n_tiles * kp.k_splits;
         if (kp.n_tiles <= num_sms && (10 * ctas < 9LL * num_sms || ctas > num_sms) &&
             (long long)kp.n_tiles * p.K < (1ll << 31)) {
             KParams ks = kp;
+            // a share: at most this many list entries, or channels of one
+            // tile's slice (threshold source)
             const int share = ceil_div((long long)kp.n_tiles * p.K, num_sms);
             ks.rows_cap = std::min(p.K, share) + 8;
             // scale/zero staged for the groups a share's rows touch (about
-            // twice its rows at 50% sparsity), as many as shared memory holds;
-            // the others are folded from global memory
-            ks.span_cap = std::min(G, ceil_div(2LL * share, 1LL << kp.lg) + 2);
+            // twice its rows at 50% sparsity, or its channels' groups), as
+            // many as shared memory holds; the others are folded from global
+            // memory
+            ks.span_cap = std::min(G, ceil_div((SRC == ROWS_LIST ? 2LL : 1LL) * share,
+                                               1LL << kp.lg) + 2);
             Smem1 LS = smem1_layout(ks.span_cap, ks.rows_cap, bp, BW, NM);
             while (ks.span_cap > 1 && LS.total > kMaxSmem) {
                 --ks.span_cap;
@@ -776,8 +802,9 @@ cudaError_t launch_gemv(const GemvProblem &p, int num_sms, cudaStream_t stream)
     // B > 8 over the plain layout: the tensor-core kernel. Up to 8 rows the
     // CUDA-core kernel (two batch rows per warp, one FMA per code and row)
     // measured as fast; above, its warps each carry every row of the CTA.
-    if (p.B > 8 && !p.keep &&
-        (p.source == ROWS_LIST || p.source == ROWS_DENSE || p.source == ROWS_MASK))
+    if (p.B > 6 && !p.keep &&
+        (p.source == ROWS_LIST || p.source == ROWS_DENSE || p.source == ROWS_MASK ||
+         p.source == ROWS_THRESH))
         return launch_gemv_mma(p, num_sms, stream);
     switch (p.source) {
     case ROWS_LIST: return launch_src<ROWS_LIST>(kp, num_sms, stream);
@@ -785,10 +812,12 @@ cudaError_t launch_gemv(const GemvProblem &p, int num_sms, cudaStream_t stream)
     case ROWS_MASK: return launch_src<ROWS_MASK>(kp, num_sms, stream);
     case ROWS_GLU: return launch_gemv_t<ROWS_GLU, 1>(kp, num_sms, stream); // batch 1
     default:
-        // the API admits the threshold path at B = 1 only
+        // the API admits the 2:4 threshold path at B = 1 only
         if (p.keep)
             return launch_gemv_t<ROWS_THRESH, 1, true>(kp, num_sms, stream);
-        return launch_gemv_t<ROWS_THRESH, 1>(kp, num_sms, stream);
+        if (p.B == 1)
+            return launch_gemv_t<ROWS_THRESH, 1>(kp, num_sms, stream);
+        return launch_gemv_t<ROWS_THRESH, 2>(kp, num_sms, stream);
     }
 }
 

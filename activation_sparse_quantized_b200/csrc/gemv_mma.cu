@@ -3,7 +3,8 @@
 //   y[b][n] = sum_{k in U} s[g(k)][n] * (q[k][n] - z[g(k)][n]) * x[b][k]
 //
 // U is the one active set of the batch (the union of the rows' active
-// channels, or the caller's index list or bitmask). Method: "Enabling Dynamic
+// channels, found by the CTAs themselves from x and the rows' thresholds, or
+// the caller's index list or bitmask). Method: "Enabling Dynamic
 // Sparsity in Quantized LLM Inference", Abstract: a GEMV over the quantized
 // layout that reads only the weight runs of the active channels.
 //
@@ -69,7 +70,7 @@ constexpr int kMBlocks = kTileN1 / 128;     // MMA M-blocks per tile
 __host__ __device__ constexpr int a_stage_bytes(int kb) { return kb * kTileN1 * 2; }
 __host__ __device__ constexpr int b_stage_bytes(int kb) { return kb * kMmaN * 2; }
 constexpr int kMaxStages = 4;               // operand stages (2..4, by shared memory)
-constexpr int kMRing = 4;                   // rows in flight per expanding warp
+constexpr int kPfRows = 4;                  // rows of packed codes in flight per expanding lane
 constexpr int kTmemCols = 512;              // two accumulator sets and the running totals
 constexpr int kTotCol = 256;                // first column of the totals
 constexpr unsigned long long kWaitNs = 200000000ull; // a barrier wait gives up after 0.2 s
@@ -122,31 +123,31 @@ __device__ __forceinline__ uint32_t b_elem_off(int c, int k, int kb)
 }
 
 struct SmemM {
-    size_t a, b, ring, rxh, ridx, rstart, rkb, scan, total;
+    size_t a, b, rxh, ridx, rstart, rkb, kbj, kbn, scan, total;
 };
 
 __host__ __device__ inline size_t align16(size_t v) { return (v + 15) / 16 * 16; }
 
 // Row stride of the staged x' (batch-major): an odd multiple of 8 rows, so
-// that a lane's 8 rows are one 16-byte access and the 16 batch columns of one
-// row fall into distinct bank pairs.
+// that the 16 batch columns of one row fall into distinct bank pairs.
 __host__ __device__ inline int rxh_stride(int rows_cap) { return (((rows_cap + 7) / 8) | 1) * 8; }
 
-// a: `stages` A stages (1024-aligned); b: B stages; ring: each expanding
-// warp's per-lane rings; rxh: x' of the CTA's rows, [bp batch rows][stride]
-// fp16; ridx: the CTA's rows; rstart / rkb: first row / first K-block of each
-// run (+1 entry); scan: per-32-row counts.
+// a: `stages` A stages (1024-aligned); b: B stages; rxh: x' of the CTA's
+// rows, [bp batch rows][stride] fp16; ridx: the CTA's rows; rstart / rkb:
+// first row / first K-block of each run (+1 entry); kbj / kbn: first row and
+// number of valid rows of each K-block; scan: per-32-row counts.
 __host__ __device__ inline SmemM smemm_layout(int rows_cap, int stages, int bp, int kb)
 {
     SmemM s;
     s.a = 0;
     s.b = s.a + (size_t)stages * a_stage_bytes(kb);
-    s.ring = s.b + (size_t)stages * b_stage_bytes(kb);
-    s.rxh = s.ring + (size_t)kMWarps * kMRing * kRowBytes1;
+    s.rxh = s.b + (size_t)stages * b_stage_bytes(kb);
     s.ridx = align16(s.rxh + (size_t)bp * rxh_stride(rows_cap) * 2);
     s.rstart = align16(s.ridx + (size_t)rows_cap * 4);
     s.rkb = align16(s.rstart + (size_t)(rows_cap + 1) * 4);
-    s.scan = align16(s.rkb + (size_t)(rows_cap + 1) * 4);
+    s.kbj = align16(s.rkb + (size_t)(rows_cap + 1) * 4);
+    s.kbn = align16(s.kbj + (size_t)(rows_cap + 1) * 4);
+    s.scan = align16(s.kbn + (size_t)(rows_cap + 1) * 4);
     s.total = align16(s.scan + (size_t)((rows_cap + 31) / 32 + 4) * 4);
     return s;
 }
@@ -270,9 +271,10 @@ __device__ __forceinline__ uint32_t zero_of(uint32_t w)
 // Rows of one segment into ridx (ascending positions of the caller's list, or
 // of the active channels), returns their number. Index list: entries
 // [lo, hi) of idx (outside [0, K) -> -1, flagged); dense: channels
-// [8 lo, 8 hi); bitmask: the active channels of [8 lo, 8 hi), by ballots over
-// runs of 32 channels and a prefix over the runs' counts. All threads; ends
-// with a barrier.
+// [8 lo, 8 hi); bitmask or threshold: the active channels of [8 lo, 8 hi)
+// (mask bit, or |x[b][c]| > t_b for some batch row b), by ballots over runs of
+// 32 channels and a prefix over the runs' counts. All threads; ends with a
+// barrier.
 template <int SRC>
 __device__ int segment_rows(const GemvProblem &p, int lo, int hi, int32_t *ridx, int *scan)
 {
@@ -295,11 +297,22 @@ __device__ int segment_rows(const GemvProblem &p, int lo, int hi, int32_t *ridx,
         __syncthreads();
         return n;
     } else {
+        // bitmask: bit c of the mask; threshold: |x[b][c]| > t_b for some
+        // batch row b (the union of the rows' active sets)
         const int c0 = 8 * lo, c1 = 8 * hi;
         const int runs = (c1 - c0 + 31) / 32;
         auto run_bits = [&](int q) -> uint32_t {
             const int c = c0 + q * 32 + lane;
-            const bool act = (c < c1) && ((__ldg(p.mask + (c >> 5)) >> (c & 31)) & 1u);
+            bool act = false;
+            if (c < c1) {
+                if (SRC == ROWS_MASK) {
+                    act = (__ldg(p.mask + (c >> 5)) >> (c & 31)) & 1u;
+                } else {
+                    for (int b = 0; b < p.B; ++b)
+                        act = act || (fabsf(bf16_bits_to_float(__ldg(p.x + (size_t)b * p.K + c))) >
+                                      p.tb[b]);
+                }
+            }
             return __ballot_sync(0xffffffffu, act);
         };
         for (int q = warp; q < runs; q += kAllWarps) {
@@ -343,11 +356,12 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
     constexpr int SPW = KB / 16; // slots per expanding warp
     constexpr int AST = a_stage_bytes(KB), BST = b_stage_bytes(KB);
     const SmemM L = smemm_layout(kp.rows_cap, nst, bp, KB);
-    uint8_t *ring = smem + L.ring;
     uint16_t *rxh = reinterpret_cast<uint16_t *>(smem + L.rxh);
     int32_t *ridx = reinterpret_cast<int32_t *>(smem + L.ridx);
     int *rstart = reinterpret_cast<int *>(smem + L.rstart);
     int *rkb = reinterpret_cast<int *>(smem + L.rkb);
+    int *kbj = reinterpret_cast<int *>(smem + L.kbj);
+    int *kbn = reinterpret_cast<int *>(smem + L.kbn);
     int *scan = reinterpret_cast<int *>(smem + L.scan);
     const uint32_t sA = smem_u32(smem + L.a), sB = smem_u32(smem + L.b);
 
@@ -472,6 +486,22 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
         }
         __syncthreads();
         const int nkb = s_nkb;
+        // First row and valid rows of every K-block (its run by a binary search
+        // over the runs' first K-blocks), so that neither side walks the runs.
+        for (int t = tid; t < nkb; t += kMThreads) {
+            int lo = 0, hi = nruns - 1; // the run r with rkb[r] <= t < rkb[r + 1]
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (rkb[mid] <= t)
+                    lo = mid;
+                else
+                    hi = mid - 1;
+            }
+            const int j0 = rstart[lo] + KB * (t - rkb[lo]);
+            kbj[t] = j0;
+            kbn[t] = rstart[lo + 1] - j0; // may exceed KB
+        }
+        __syncthreads();
 
         // K-block kb: its run (a pointer advanced monotonically), the ridx
         // position of its slot 0 and its valid slots.
@@ -519,60 +549,37 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
             __syncwarp();
         } else {
             // ---- the expanding warps ---------------------------------------------
-            // Warp w expands slot w of every K-block: its row stream is one row
-            // per K-block, through a per-lane ring kMRing K-blocks ahead (with its
-            // own run pointer).
+            // Warp w expands slots w (and w + 16) of every K-block. Its lanes read
+            // their 16-byte columns of those rows straight into registers,
+            // kPfRows rows ahead, so that no shared memory carries packed codes.
             constexpr int kEx = kMWarps * 32; // threads of the expanding warps
+            constexpr int PF = kPfRows / SPW; // K-blocks prefetched ahead
             // x' = x 2^S_b in fp16 per batch row b, 2^14 <= max |x'| < 2^15 over
             // the CTA's rows (as in the batch-1 kernel), staged batch-major in
-            // rxh. Warp w owns batch row b = w: each lane gathers chunks of 8 rows
-            // (one 16-byte load when the 8 rows are 8 consecutive aligned
-            // channels), four chunks in flight, before any weight row is
-            // requested; the warp reduces max |x|, then converts its row in place.
+            // rxh. Warp w owns batch row b = w: lane l gathers rows l, l + 32,
+            // ... (one bf16 each, 16 loads in flight; consecutive channels make
+            // each warp load one coalesced 64-byte request), then the warp
+            // reduces max |x| and converts its row in place.
             const int rs = rxh_stride(kp.rows_cap);
             if (warp < p.B) {
                 const int b = warp;
                 uint16_t *xr = rxh + (size_t)b * rs;
                 const uint16_t *xb = p.x + (size_t)b * p.K;
-                const int nch = (nr + 7) / 8;
                 float m = 0.f;
-                for (int c0 = lane; c0 < nch; c0 += 4 * 32) {
-                    uint4 v[4];
+                for (int j0 = 0; j0 < nr; j0 += 32 * 16) {
+                    uint16_t v[16];
     #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int c = c0 + 32 * u;
-                        v[u] = make_uint4(0u, 0u, 0u, 0u);
-                        if (c < nch) {
-                            const int j0 = 8 * c;
-                            const int k0 = ridx[j0];
-                            bool vec = (j0 + 8 <= nr) && k0 >= 0 && (k0 & 7) == 0;
-    #pragma unroll
-                            for (int i = 1; i < 8; ++i)
-                                vec = vec && (ridx[min(j0 + i, nr - 1)] == k0 + i);
-                            if (vec) {
-                                v[u] = __ldg(reinterpret_cast<const uint4 *>(xb + k0));
-                            } else {
-                                uint32_t h[8];
-    #pragma unroll
-                                for (int i = 0; i < 8; ++i) {
-                                    const int k = (j0 + i < nr) ? ridx[j0 + i] : -1;
-                                    h[i] = (k >= 0) ? (uint32_t)__ldg(xb + k) : 0u;
-                                }
-                                v[u] = make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16),
-                                                  h[4] | (h[5] << 16), h[6] | (h[7] << 16));
-                            }
-                        }
+                    for (int u = 0; u < 16; ++u) {
+                        const int j = j0 + 32 * u + lane;
+                        const int k = (j < nr) ? ridx[j] : -1;
+                        v[u] = (k >= 0) ? __ldg(xb + k) : (uint16_t)0;
                     }
     #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int c = c0 + 32 * u;
-                        if (c < nch) {
-                            *reinterpret_cast<uint4 *>(xr + 8 * c) = v[u];
-                            const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-    #pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                m = fmaxf(m, fabsf(bf16_bits_to_float(
-                                                 (uint16_t)(w[i >> 1] >> (16 * (i & 1))))));
+                    for (int u = 0; u < 16; ++u) {
+                        const int j = j0 + 32 * u + lane;
+                        if (j < nr) {
+                            xr[j] = v[u];
+                            m = fmaxf(m, fabsf(bf16_bits_to_float(v[u])));
                         }
                     }
                 }
@@ -582,41 +589,36 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
                     s_S[b] = S;
                 const float fa = pow2f(S - S / 2), fb = pow2f(S / 2);
                 __syncwarp();
-                for (int c = lane; c < nch; c += 32) {
-                    uint4 v = *reinterpret_cast<const uint4 *>(xr + 8 * c);
-                    uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const uint32_t lo = __half_as_ushort(__float2half_rn(
-                            (bf16_bits_to_float((uint16_t)(w[i] & 0xffffu)) * fa) * fb));
-                        const uint32_t hi = __half_as_ushort(__float2half_rn(
-                            (bf16_bits_to_float((uint16_t)(w[i] >> 16)) * fa) * fb));
-                        w[i] = lo | (hi << 16);
-                    }
-                    *reinterpret_cast<uint4 *>(xr + 8 * c) = make_uint4(w[0], w[1], w[2], w[3]);
-                }
+                for (int j = lane; j < nr; j += 32)
+                    xr[j] = __half_as_ushort(__float2half_rn((bf16_bits_to_float(xr[j]) * fa) * fb));
             }
 
             const size_t row_bytes = (size_t)(p.N / 2);
             const uint8_t *wcol = p.qweight + (lane_ok ? ((size_t)n0 / 2 + lane * 16) : 0);
-            uint8_t *myring = ring + (size_t)warp * kMRing * kRowBytes1 + lane * 16;
-            int ring_run = 0;
-            // ridx position of this warp's slot u of K-block kb, or -1
-            auto kb_row = [&](int kb, int u) -> int {
-                kb_run(kb, ring_run);
-                const int j = rstart[ring_run] + KB * (kb - rkb[ring_run]) + warp + 16 * u;
-                return (j < rstart[ring_run + 1]) ? j : -1;
-            };
+            // This warp's rows of K-block kb into dst (zero for slots past the
+            // K-block's valid rows; lanes past N read column 0).
+            auto fetch = [&](int kb, uint4 *dst) {
+                if (kb < nkb) {
+                    const int j0 = kbj[kb], nv = kbn[kb];
     #pragma unroll
-            for (int i = 0; i < kMRing; ++i) {
-                if (i < SPW * nkb) {
-                    const int j = kb_row(i / SPW, i % SPW);
-                    if (j >= 0)
-                        cp_async16(myring + i * kRowBytes1,
-                                   wcol + (size_t)max(ridx[j], 0) * row_bytes);
+                    for (int u = 0; u < SPW; ++u) {
+                        const int slot = warp + 16 * u;
+                        dst[u] = make_uint4(0u, 0u, 0u, 0u);
+                        if (slot < nv) {
+                            const uint8_t *src =
+                                wcol + (size_t)max(ridx[j0 + slot], 0) * row_bytes;
+                            asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                         : "=r"(dst[u].x), "=r"(dst[u].y), "=r"(dst[u].z),
+                                           "=r"(dst[u].w)
+                                         : "l"(src));
+                        }
+                    }
                 }
-                cp_async_commit();
-            }
+            };
+            uint4 pf[PF][SPW];
+    #pragma unroll
+            for (int q = 0; q < PF; ++q)
+                fetch(q, pf[q]);
             // This lane's four A chunks of slot `warp` (stage-relative) and its B
             // element (lanes 0..15: batch column = lane).
             uint32_t aoff[SPW][4], boff[SPW];
@@ -631,21 +633,22 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
             // Zero points of this lane's 32 outputs for one group, as subnormal
             // fp16 pairs matching the AND results: word j, pairs = outputs
             // (8j, 8j+4), (8j+1, 8j+5) << 4, (8j+2, 8j+6), (8j+3, 8j+7) << 4.
-            uint4 zraw[8];
+            // The next run's scale/zero slice of the tile (4 KB) is prefetched
+            // into L1 a run ahead by warp 0, one 128-byte line per lane; every
+            // warp reads its lanes' words from there at the run's start.
             auto load_sz = [&](int G) {
+                if (warp == 0)
+                    asm volatile("prefetch.global.L1 [%0];" ::"l"(
+                        p.sz + (size_t)G * p.N + n0 + (lane_ok ? lane * 32 : 0)));
+            };
+            uint32_t zc[4][4];
+            auto unpack_z = [&](int G) {
                 const uint4 *src = reinterpret_cast<const uint4 *>(p.sz + (size_t)G * p.N + n0 +
                                                                    (lane_ok ? lane * 32 : 0));
     #pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    zraw[c] = __ldg(src + c);
-            };
-            uint32_t zc[4][4];
-            auto unpack_z = [&]() {
-    #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    const uint32_t w[8] = {zraw[2 * j].x,     zraw[2 * j].y,     zraw[2 * j].z,
-                                           zraw[2 * j].w,     zraw[2 * j + 1].x, zraw[2 * j + 1].y,
-                                           zraw[2 * j + 1].z, zraw[2 * j + 1].w};
+                    const uint4 a = __ldg(src + 2 * j), c = __ldg(src + 2 * j + 1);
+                    const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
                     uint32_t z[8];
     #pragma unroll
                     for (int o = 0; o < 8; ++o)
@@ -711,18 +714,28 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
             // every batch row's x' (written by its warp above) is in place
             asm volatile("bar.sync 1, %0;" ::"n"(kEx) : "memory");
 
+            // K-block kb from the registers in v: expand into stage kb % nst,
+            // the B operand beside it, hand the stage to the issuer; then the
+            // previous run's fold, one K-block into the next run (its MMAs have
+            // had that long to finish).
             int run = 0;
-            for (int kb = 0; kb < nkb; ++kb) {
+            auto step = [&](int kb, const uint4 *v) {
                 kb_run(kb, run);
                 const int kg = kb_base + kb;
                 const int s = kg % nst;
-                const int j0 = rstart[run] + KB * (kb - rkb[run]);
-                const int nv = rstart[run + 1] - j0; // valid slots (may exceed KB)
+                const int j0 = kbj[kb];
+                const int nv = kbn[kb]; // valid slots (may exceed KB)
                 const bool first = kb == rkb[run];
                 if (first) {
-                    unpack_z(); // this run's zero points (loaded a run ahead)
+                    unpack_z(grp(rstart[run])); // this run's zero points (in L1 since a run ago)
                     if (run + 1 < nruns)
                         load_sz(grp(rstart[run + 1]));
+                    if (run > 0) {
+    #pragma unroll
+                        for (int i = 0; i < 2; ++i)
+                            sfold[i] = snew[i];
+                        load_s(grp(rstart[run]), snew); // this run's scales, for its fold
+                    }
                 }
                 // The stage's previous K-block has been multiplied.
                 if (kg >= nst)
@@ -730,22 +743,9 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
                 const uint32_t a_st = sA + (uint32_t)(s * AST);
     #pragma unroll
                 for (int u = 0; u < SPW; ++u) {
-                    const int i = SPW * kb + u; // this warp's ring position
                     const int slot = warp + 16 * u;
                     const bool valid = slot < nv;
-                    cp_async_wait<kMRing - 1>();
-                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                    if (valid)
-                        v = *reinterpret_cast<const uint4 *>(myring + (i % kMRing) * kRowBytes1);
-                    // refill the ring slot with this warp's row kMRing positions ahead
-                    if (i + kMRing < SPW * nkb) {
-                        const int j = kb_row((i + kMRing) / SPW, (i + kMRing) % SPW);
-                        if (j >= 0)
-                            cp_async16(myring + (i % kMRing) * kRowBytes1,
-                                       wcol + (size_t)max(ridx[j], 0) * row_bytes);
-                    }
-                    cp_async_commit();
-                    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+                    const uint32_t wv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
     #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         uint32_t t0 = 0u, t1 = 0u, t2 = 0u, t3 = 0u;
@@ -773,15 +773,19 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
                 __syncwarp();
                 if (lane == 0)
                     mbar_arrive(bar_full + s);
-
-                // The previous run ended with the previous K-block: fold it now,
-                // while this K-block is being multiplied.
-                if (first && run > 0) {
-    #pragma unroll
-                    for (int i = 0; i < 2; ++i)
-                        sfold[i] = snew[i];
-                    load_s(grp(rstart[run]), snew); // this run's scales, for its fold
+                const int fold_kb = rkb[run] + min(1, rkb[run + 1] - rkb[run] - 1);
+                if (run > 0 && kb == fold_kb)
                     fold(run - 1);
+            };
+
+            for (int kb0 = 0; kb0 < nkb; kb0 += PF) {
+    #pragma unroll
+                for (int q = 0; q < PF; ++q) {
+                    const int kb = kb0 + q;
+                    if (kb < nkb) {
+                        step(kb, pf[q]);
+                        fetch(kb + PF, pf[q]);
+                    }
                 }
             }
             if (nruns > 0) {
@@ -790,8 +794,6 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
                     sfold[i] = snew[i];
                 fold(nruns - 1);
             }
-            cp_async_wait_all();
-
             // Split-K partials from the totals, back in real units (x 2^-S_b,
             // two exact factors).
             if (nkb > 0) {
@@ -904,6 +906,7 @@ cudaError_t launch_gemv_mma(const GemvProblem &p, int num_sms, cudaStream_t stre
     case ROWS_LIST: return launch_mma_t<ROWS_LIST>(kp, num_sms, stream);
     case ROWS_DENSE: return launch_mma_t<ROWS_DENSE>(kp, num_sms, stream);
     case ROWS_MASK: return launch_mma_t<ROWS_MASK>(kp, num_sms, stream);
+    case ROWS_THRESH: return launch_mma_t<ROWS_THRESH>(kp, num_sms, stream);
     default: return cudaErrorInvalidValue;
     }
 }

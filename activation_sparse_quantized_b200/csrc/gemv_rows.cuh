@@ -158,6 +158,53 @@ __device__ int build_rows(const KParams &kp, int split, int32_t *ridx, float *rx
         }
         __syncthreads();
         return total;
+    } else if (SRC == ROWS_THRESH && !FILL_X) {
+        // Batch rows (B > 1): channel c of this CTA's slice is active when
+        // |x[b][c]| > t_b for some row b (the union of the rows' active sets).
+        // Runs of 32 channels, one per lane, a ballot per run and the count of
+        // each run in scan[]; a second pass recomputes the ballots (the x lines
+        // stay in L1) and writes each active channel at its ascending position.
+        // Channels [8 list_lo, 8 list_hi) when given (a segment), else this
+        // split's slice.
+        int c0, c1;
+        if (list_lo >= 0) {
+            c0 = 8 * list_lo;
+            c1 = 8 * list_hi;
+        } else {
+            channel_slice(kp, split, c0, c1);
+        }
+        const int lane = tid & 31, warp = tid >> 5;
+        const int runs = (c1 - c0 + 31) / 32;
+        auto run_bits = [&](int q) -> uint32_t {
+            const int c = c0 + q * 32 + lane;
+            bool act = false;
+            if (c < c1)
+                for (int b = 0; b < p.B; ++b)
+                    act = act || (fabsf(bf16_bits_to_float(__ldg(p.x + (size_t)b * p.K + c))) >
+                                  p.tb[b]);
+            return __ballot_sync(0xffffffffu, act);
+        };
+        for (int q = warp; q < runs; q += NT / 32) {
+            const uint32_t m = run_bits(q);
+            if (lane == 0)
+                scan[q] = __popc(m);
+        }
+        __syncthreads();
+        int total = 0;
+        for (int c = 0; c * 32 < runs; ++c) {
+            int ct;
+            const int excl = chunk_prefix(scan, runs, c, total, &ct);
+            for (int q = c * 32 + ((warp - c * 32) % (NT / 32) + NT / 32) % (NT / 32);
+                 q < runs && q < c * 32 + 32; q += NT / 32) {
+                const int base = __shfl_sync(0xffffffffu, excl, q - c * 32);
+                const uint32_t m = run_bits(q);
+                if ((m >> lane) & 1u)
+                    ridx[base + __popc(m & ((1u << lane) - 1u))] = c0 + q * 32 + lane;
+            }
+            total += ct;
+        }
+        __syncthreads();
+        return total;
     } else {
         // Threshold this CTA's channel slice: each warp takes runs of 32
         // channels, one per lane; a ballot gives each run's active channels,

@@ -47,6 +47,26 @@ __device__ __forceinline__ void cp_async_wait_all()
     asm volatile("cp.async.wait_all;\n" ::: "memory");
 }
 
+// ---- L2 prefetch hints ----
+
+// [p, p + bytes) into L2 with one bulk prefetch (p 16-byte aligned, bytes a
+// multiple of 16).
+__device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes)
+{
+    if (bytes)
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// The 128-byte lines of [p, end) into L2, one line per lane of the calling
+// warp (at most 32 lines).
+__device__ __forceinline__ void prefetch_l2_lines(const void *p, const void *end)
+{
+    const uintptr_t a = (uintptr_t)p & ~(uintptr_t)127, e = (uintptr_t)end;
+    const uintptr_t line = a + 128u * (threadIdx.x & 31);
+    if (line < e)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(line) : "memory");
+}
+
 // ---- Programmatic dependent launch ----
 
 __device__ __forceinline__ void grid_dependency_wait()

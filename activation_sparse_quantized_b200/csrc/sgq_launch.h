@@ -17,7 +17,7 @@ struct Thresholds {
 enum RowSource : int {
     ROWS_LIST = 0,   // device list idx[0..*count)
     ROWS_DENSE = 1,  // every channel
-    ROWS_THRESH = 2, // |x[k]| > t, found by each CTA for its own channel slice
+    ROWS_THRESH = 2, // |x[b][k]| > t_b for some row b, found by each CTA for its own channel slice
     ROWS_MASK = 3,   // bit k of a device bitmask, decoded by each CTA for its own slice
     ROWS_GLU = 4,    // x = bf16(act(gate) * up) from the fp32 sums of a gate/up GEMV, |x| > t
 };
@@ -43,6 +43,7 @@ struct GemvProblem {
     int32_t *status;
     int N, K, group, B;
     float t;
+    float tb[SGQ_MAX_BATCH]; // ROWS_THRESH at B > 1: threshold of each batch row
     int source;
     int epilogue; // Epilogue; y (and y_f32) are [B][N/2] for the GLU epilogues
     bool accumulate; // add into ws_acc (the caller's fp32 [B][N]) and launch no epilogue kernel

@@ -35,6 +35,7 @@ EXPORTS = (
     "sgq_gemv_glu_dense", "sgq_select_mask", "sgq_gemv_mask", "sgq_packed_sizes_nm",
     "sgq_pack_nm", "sgq_gemv_nm", "sgq_gemv_nm_thresh", "sgq_gemv_acc", "sgq_gemv_thresh_acc",
     "sgq_ffn_workspace_bytes", "sgq_ffn", "sgq_read_status", "sgq_debug_gemv_withhold",
+    "sgq_gemv_thresh_batch", "sgq_gemv_glu_thresh_batch",
 )
 
 
@@ -80,6 +81,8 @@ def _declare(lib):
         "sgq_gemv": ([P, P, I, I, I, P, I, P, P, P, P, P, Z, P, P], I),
         "sgq_debug_gemv_withhold": ([P, P, I, I, I, P, I, P, P, P, P, P, Z, P, P], I),
         "sgq_gemv_thresh": ([P, P, I, I, I, P, F, P, P, P, Z, P, P], I),
+        "sgq_gemv_thresh_batch": ([P, P, I, I, I, P, I, P, P, P, P, Z, P, P], I),
+        "sgq_gemv_glu_thresh_batch": ([P, P, I, I, I, P, I, P, I, P, P, P, Z, P, P], I),
         "sgq_gemv_dense": ([P, P, I, I, I, P, I, P, P, P, Z, P, P], I),
         "sgq_gemv_thresh_noalloc": ([P, P, I, I, I, P, F, P, P, P, P], I),
         "sgq_glu": ([P, P, P, I, I, I, P], I),
@@ -244,6 +247,15 @@ def sgq_gemv_thresh(qweight, sz, N, K, group, x, t, y, y_f32, workspace, status=
         _stream(stream)))
 
 
+def sgq_gemv_thresh_batch(qweight, sz, N, K, group, x, B, t_host, y, y_f32, workspace,
+                          status=None, stream=None):
+    t = (ctypes.c_float * B)(*[float(v) for v in t_host])
+    _check("sgq_gemv_thresh_batch", load().sgq_gemv_thresh_batch(
+        _ptr(qweight), _ptr(sz), N, K, group, _ptr(x), B, t, _ptr(y), _ptr(y_f32),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status),
+        _stream(stream)))
+
+
 def sgq_gemv_thresh_noalloc(qweight, sz, N, K, group, x, t, y, y_f32, status=None, stream=None):
     """sgq_gemv_thresh with the library's fixed scratch instead of a workspace
     (for callers that cannot allocate); N <= SGQ_NOALLOC_MAX_N."""
@@ -272,6 +284,15 @@ def sgq_gemv_glu_thresh(qweight, sz, I, K, group, x, t, act, h, h_f32, workspace
                         stream=None):
     _check("sgq_gemv_glu_thresh", load().sgq_gemv_glu_thresh(
         _ptr(qweight), _ptr(sz), I, K, group, _ptr(x), float(t), act, _ptr(h), _ptr(h_f32),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status),
+        _stream(stream)))
+
+
+def sgq_gemv_glu_thresh_batch(qweight, sz, I, K, group, x, B, t_host, act, h, h_f32, workspace,
+                              status=None, stream=None):
+    t = (ctypes.c_float * B)(*[float(v) for v in t_host])
+    _check("sgq_gemv_glu_thresh_batch", load().sgq_gemv_glu_thresh_batch(
+        _ptr(qweight), _ptr(sz), I, K, group, _ptr(x), B, t, act, _ptr(h), _ptr(h_f32),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status),
         _stream(stream)))
 

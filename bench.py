@@ -995,6 +995,16 @@ class BatchFfnReplica:
         sgq.sgq_gemv_glu(qw, sz, I, H, g, self.x[r], B, self.idx_x, self.cnt_x,
                          sgq.SGQ_ACT_SILU, self.h, None, self.ws)
 
+    def ffn_fused(self, r):                      # 4 launches
+        """The rows' union found inside each GEMV (sgq_gemv_glu_thresh_batch,
+        sgq_gemv_thresh_batch): two GEMVs and their epilogue kernels."""
+        B, H, I, g = self.B, self.H, self.I, self.g
+        qw, sz = self.gu[r]
+        sgq.sgq_gemv_glu_thresh_batch(qw, sz, I, H, g, self.x[r], B, self.t[r],
+                                      sgq.SGQ_ACT_SILU, self.h, None, self.ws)
+        qd, sd = self.down[r]
+        sgq.sgq_gemv_thresh_batch(qd, sd, H, I, g, self.h, B, self.th[r], self.y, None, self.ws)
+
     def ffn(self, r):                            # 6 launches
         B, H, I, g = self.B, self.H, self.I, self.g
         self.front(r)
@@ -1011,16 +1021,21 @@ def run_batch(batches=(1, 2, 4, 8, 16), n_steps: int = 64):
     for B in batches:
         f.setup(B)
         n = max(n_steps, 2 * R)
-        us = time_calls(lambda i: f.ffn(i % R), n, R) * 1e3 / n
+        us6 = time_calls(lambda i: f.ffn(i % R), n, R) * 1e3 / n
+        us = time_calls(lambda i: f.ffn_fused(i % R), n, R) * 1e3 / n
         ux, uh = float(np.mean(f.union_x)), float(np.mean(f.union_h))
         wbytes = ux * f.H * f.I + uh * f.I * f.H / 2    # codes of the union rows (gate+up, down)
-        out.append({"batch": B, "us_per_ffn": round(us, 2), "union_active_in": round(ux, 3),
+        out.append({"batch": B, "us_per_ffn": round(us, 2), "launches": 4,
+                    "us_per_ffn_select_kernels": round(us6, 2), "launches_select_kernels": 6,
+                    "union_active_in": round(ux, 3),
                     "union_active_h": round(uh, 3),
                     "weight_code_GBps": round(wbytes / (us * 1e-6) / 1e9, 1),
                     "tokens_per_s_equiv_ffn_only_64_layers": round(B * 1e6 / (64 * us), 1)})
     return {"workload": "Qwen3-32B FFN decode (hidden 5120, intermediate 25600, int4 g128, "
-                        "SiLU): per-row 50% thresholds, union active sets, fused gate/up GLU; "
-                        "6 launches per FFN (two selects, two GEMV calls)",
+                        "SiLU): per-row 50% thresholds, union active sets found inside each GEMV "
+                        "(sgq_gemv_glu_thresh_batch, sgq_gemv_thresh_batch: 4 launches); "
+                        "us_per_ffn_select_kernels: the same with sgq_select before each GEMV "
+                        "(6 launches)",
             "rows": out, "rotation": f"{R} copies, {f.bytes_resident / 1e6:.0f} MB"}
 
 

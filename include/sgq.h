@@ -173,6 +173,25 @@ int sgq_gemv_thresh(const void *qweight, const void *sz, int N, int K, int group
                     void *workspace, size_t ws_bytes, int32_t *status, void *stream);
 
 /*
+ * The same at batch B (1..16) with one threshold per batch row: the result of
+ * sgq_select(x, B, t_host) (the union of the rows' active channels, "Enabling
+ * Dynamic Sparsity in Quantized LLM Inference", Abstract: runtime gathering of
+ * the active indices) followed by sgq_gemv over that list, in one GEMV launch
+ * (plus the epilogue kernel): each CTA thresholds all B rows of its own slice
+ * of channels, so no index list is written or read.
+ *
+ *   x        bf16 [B][K], K a multiple of 8.
+ *   t_host   host array of B floats; channel k is active when |x[b][k]| > t[b]
+ *            for some b (strict; NaN never; t < 0 selects every channel).
+ *   y, y_f32, workspace, status, stream  as sgq_gemv (workspace for B rows).
+ * Returns as sgq_gemv; SGQ_ERR_BATCH for B outside 1..16, SGQ_ERR_NULL for a
+ * NULL t_host.
+ */
+int sgq_gemv_thresh_batch(const void *qweight, const void *sz, int N, int K, int group,
+                          const void *x, int B, const float *t_host, void *y, float *y_f32,
+                          void *workspace, size_t ws_bytes, int32_t *status, void *stream);
+
+/*
  * Accumulating forms: y_acc += W_deq[:, S] x[S] into a caller-owned fp32
  * buffer y_acc [B][N] (16-byte aligned), e.g. the fp32 residual stream of a
  * decode step (the pages fuse no such epilogue; it is a deployment form of
@@ -288,6 +307,12 @@ int sgq_gemv_glu(const void *qweight, const void *sz, int I, int K, int group,
 int sgq_gemv_glu_thresh(const void *qweight, const void *sz, int I, int K, int group,
                         const void *x, float t, int act, void *h, float *h_f32,
                         void *workspace, size_t ws_bytes, int32_t *status, void *stream);
+/* The fused-select form at batch B with one threshold per row (rows as
+ * sgq_gemv_thresh_batch: the union of the rows' active channels). */
+int sgq_gemv_glu_thresh_batch(const void *qweight, const void *sz, int I, int K, int group,
+                              const void *x, int B, const float *t_host, int act, void *h,
+                              float *h_f32, void *workspace, size_t ws_bytes,
+                              int32_t *status, void *stream);
 int sgq_gemv_glu_dense(const void *qweight, const void *sz, int I, int K, int group,
                        const void *x, int B, int act, void *h, float *h_f32,
                        void *workspace, size_t ws_bytes, int32_t *status, void *stream);
