@@ -6,12 +6,22 @@
 // exactly the nonzero channels, the ReLU zeros of "SVD Contextual Sparsity
 // Predictors", Abstract). The list is written in ascending order.
 //
-// One CTA of 1024 threads walks the channels in tiles of 16 per thread:
-// 16-byte loads of each batch row, a per-thread 16-bit mask, a warp shuffle
-// scan and a cross-warp scan in shared memory; each thread puts its indices at
-// its exclusive offset in a shared-memory copy of the tile, which the CTA then
-// writes out with coalesced stores. The activation vector is small (2*B*K
-// bytes), so one CTA keeps the whole list ordered without any inter-CTA wait.
+// Batch 1: tiles of 2048 channels, one CTA of 256 threads
+// per tile, one 16-byte load (8 channels) per thread. A CTA finds where its
+// indices start by counting the active channels of every earlier tile itself
+// (at most 2 K bytes of x, from L2), so the list comes out in ascending order
+// with no wait between CTAs and no scratch memory; the last CTA writes the
+// count.
+//
+// Otherwise one CTA of 1024 threads walks the channels in tiles of 16 per
+// thread: 16-byte loads of each batch row, a per-thread 16-bit mask, a warp
+// shuffle scan and a cross-warp scan in shared memory; each thread puts its
+// indices at its exclusive offset in a shared-memory copy of the tile, which
+// the CTA then writes out with coalesced stores.
+//
+// Both are launched with programmatic dependent launch: they wait for the
+// previous kernel only before reading x, and let the next one (the GEMV)
+// launch early.
 #include "sgq_device.cuh"
 #include "sgq_launch.h"
 
@@ -33,6 +43,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const uint16_t *__r
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
+    grid_launch_dependents();
+    grid_dependency_wait(); // x may come from the previous kernel
     int offset = 0;
     // tiles of 16 channels per thread: two 16-byte loads per batch row, both
     // in flight before either is used (K <= 16384 is a single tile)
@@ -103,6 +115,76 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const uint16_t *__r
         *count = offset;
 }
 
+constexpr int kTileThreads = 256;           // batch-1 tiled select: threads per CTA
+constexpr int kTileCh = 8 * kTileThreads;   // channels per tile
+
+// Active bits of 8 channels (one 16-byte load of bf16 x) against t.
+__device__ __forceinline__ uint32_t mask8(const uint4 v, float t)
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t m = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        m |= (fabsf(__uint_as_float(w[e] << 16)) > t ? 1u : 0u) << (2 * e);
+        m |= (fabsf(__uint_as_float(w[e] & 0xffff0000u)) > t ? 1u : 0u) << (2 * e + 1);
+    }
+    return m;
+}
+
+// Batch 1: CTA c owns channels [c kTileCh, (c + 1) kTileCh).
+__global__ void __launch_bounds__(kTileThreads) select_tiled_kernel(const uint16_t *__restrict__ x,
+                                                                    int K, float t,
+                                                                    int32_t *__restrict__ idx,
+                                                                    int32_t *__restrict__ count)
+{
+    __shared__ int warp_sum[kTileThreads / 32], warp_excl[kTileThreads / 32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int lo = blockIdx.x * kTileCh;
+    grid_launch_dependents();
+    grid_dependency_wait(); // x may come from the previous kernel
+    // this thread's 8 channels (issued first), then the earlier tiles' chunks
+    const int c8 = lo / 8 + tid;
+    const uint4 own = (8 * c8 < K) ? __ldg(reinterpret_cast<const uint4 *>(x) + c8)
+                                   : make_uint4(0u, 0u, 0u, 0u);
+    int before = 0;
+    for (int ch = tid; ch < lo / 8; ch += kTileThreads)
+        before += __popc(mask8(__ldg(reinterpret_cast<const uint4 *>(x) + ch), t));
+    const uint32_t m = (8 * c8 < K) ? mask8(own, t) : 0u;
+    const int cnt = __popc(m);
+    // warp sums of `before` and inclusive warp scans of `cnt`
+    int incl = cnt;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d)
+            incl += v;
+    }
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1)
+        before += __shfl_xor_sync(0xffffffffu, before, d);
+    if (lane == 31)
+        warp_excl[warp] = incl;
+    if (lane == 0)
+        warp_sum[warp] = before;
+    __syncthreads();
+    int base = 0, wex = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kTileThreads / 32; ++w) {
+        base += warp_sum[w];
+        wex += (w < warp) ? warp_excl[w] : 0;
+        total += warp_excl[w];
+    }
+    int pos = base + wex + incl - cnt;
+    uint32_t mm = m;
+    while (mm) {
+        const int j = __ffs(mm) - 1;
+        idx[pos++] = lo + 8 * tid + j;
+        mm &= mm - 1;
+    }
+    if (blockIdx.x == gridDim.x - 1 && tid == 0)
+        *count = base + total;
+}
+
 // Bitmask form of the same active set, one bit per channel (the bitmask
 // indexing of "SparseDecoding: Decoding-Aware Pruning for Accurate and
 // Efficient LLM Inference", Abstract, and the shared-memory bitmap decoding of
@@ -120,6 +202,8 @@ __global__ void __launch_bounds__(kSelThreads) select_mask_kernel(const uint16_t
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
+    grid_launch_dependents();
+    grid_dependency_wait(); // x may come from the previous kernel
     int total = 0;
     for (int base = 0; base < K; base += 16 * kSelThreads) {
         const int c0 = base + tid * 16;
@@ -169,23 +253,42 @@ __global__ void __launch_bounds__(kSelThreads) select_mask_kernel(const uint16_t
 
 } // namespace
 
+// One launch with programmatic dependent launch allowed.
+template <typename Kern, typename... Args>
+cudaError_t launch_pdl_sel(Kern kern, int grid, int block, size_t smem, cudaStream_t stream,
+                           Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 cudaError_t launch_select(const uint16_t *x, int B, int K, const Thresholds &th, int32_t *idx,
                           int32_t *count, cudaStream_t stream)
 {
+    if (B == 1 && K % 8 == 0)
+        return launch_pdl_sel(select_tiled_kernel, (K + kTileCh - 1) / kTileCh, kTileThreads, 0,
+                              stream, x, K, th.t[0], idx, count);
     const size_t smem = sizeof(int) * 16 * kSelThreads; // 64 KB: one tile of indices
     cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess)
         return e;
-    select_kernel<<<1, kSelThreads, smem, stream>>>(x, B, K, th, idx, count);
-    return cudaGetLastError();
+    return launch_pdl_sel(select_kernel, 1, kSelThreads, smem, stream, x, B, K, th, idx, count);
 }
 
 cudaError_t launch_select_mask(const uint16_t *x, int B, int K, const Thresholds &th,
                                uint32_t *mask, int32_t *count, cudaStream_t stream)
 {
-    select_mask_kernel<<<1, kSelThreads, 0, stream>>>(x, B, K, th, mask, count);
-    return cudaGetLastError();
+    return launch_pdl_sel(select_mask_kernel, 1, kSelThreads, 0, stream, x, B, K, th, mask, count);
 }
 
 } // namespace sgq

@@ -91,7 +91,7 @@ def test_pack_flags_nonfinite():
 # sgq_select: bit-exact against the oracle
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("K", [8, 256, 8192, 8200, 14336, 25600])
+@pytest.mark.parametrize("K", [8, 256, 2048, 2056, 8192, 8200, 14336, 25600, 65536])
 @pytest.mark.parametrize("sparsity", [0.0, 0.3, 0.5, 0.7, 0.9, 1.0])
 def test_select_bit_exact(K, sparsity):
     x = wl.x_silu_gated(1, K, 11)
