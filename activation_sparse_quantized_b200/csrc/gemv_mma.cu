@@ -1,4 +1,4 @@
-// gemv_mma.cu -- the activation-sparse GEMV for batch 9..16, on the tensor cores.
+// gemv_mma.cu -- the activation-sparse GEMV for batch 7..16, on the tensor cores.
 //
 //   y[b][n] = sum_{k in U} s[g(k)][n] * (q[k][n] - z[g(k)][n]) * x[b][k]
 //
@@ -44,7 +44,10 @@
 // out sets SGQ_STATUS_TIMEOUT, the thread waits on nothing further and the
 // kernel runs to its end (y is then not valid). Before the tensor memory is
 // freed, the issuing thread waits (bounded too) for a commit that covers every
-// MMA of the CTA. The kernel takes more than half of an SM's shared memory, so
+// MMA of the CTA; if that wait runs out as well, the memory is freed with MMAs
+// possibly in flight (keeping it would leave the next allocation on the SM
+// waiting for ever), so a timed-out call leaves that SM's tensor memory
+// undefined until the stream drains. The kernel takes more than half of an SM's shared memory, so
 // at most one of its CTAs is resident per SM and the allocation of all 512
 // tensor-memory columns never waits.
 #include "gemv_rows.cuh"

@@ -64,6 +64,9 @@ extern "C" {
 #define SGQ_STATUS_BAD_INDEX    2  /* sgq_gemv: an index outside [0, K) was skipped             */
 #define SGQ_STATUS_BAD_COUNT    4  /* sgq_gemv: *count outside [0, K]; clamped                  */
 #define SGQ_STATUS_TIMEOUT      8  /* a bounded wait inside a GEMV kernel ran out: y is not valid */
+/* After SGQ_STATUS_TIMEOUT the tensor-core kernel may have freed its tensor
+ * memory with MMAs still in flight: treat it as fatal for the results of that
+ * context until the stream has drained. */
 
 /* Activations for sgq_glu. */
 #define SGQ_ACT_SILU 0
@@ -390,9 +393,10 @@ int sgq_layout_version(void);
  * sgq_gemv with B = 9..16 (the tensor-core kernel) in which the MMA issuer
  * withholds the commit that releases the last group run's accumulators. The
  * CTAs' waits on it give up after 0.2 s, SGQ_STATUS_TIMEOUT is set in *status
- * (status must be non-NULL to see it), y is not valid, and the kernel still
- * frees its tensor memory only after its MMAs have completed; the context
- * stays usable. Arguments as sgq_gemv; B outside 9..16 returns SGQ_ERR_SHAPE.
+ * (status must be non-NULL to see it) and y is not valid; the commit that
+ * covers every MMA is not withheld, so the kernel still frees its tensor
+ * memory after its MMAs have completed and the context stays usable.
+ * Arguments as sgq_gemv; B outside 9..16 returns SGQ_ERR_SHAPE.
  */
 int sgq_debug_gemv_withhold(const void *qweight, const void *sz, int N, int K, int group,
                             const void *x, int B, const int32_t *idx, const int32_t *count,
