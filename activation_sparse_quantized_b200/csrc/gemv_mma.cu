@@ -77,6 +77,9 @@ constexpr int kPfRows = 4;                  // rows of packed codes in flight pe
 constexpr int kTmemCols = 512;              // two accumulator sets and the running totals
 constexpr int kTotCol = 256;                // first column of the totals
 constexpr unsigned long long kWaitNs = 200000000ull; // a barrier wait gives up after 0.2 s
+// A thread in a barrier wait sleeps until the phase completes or this many
+// ns pass (then checks the wall-time limit), instead of spinning on it.
+constexpr unsigned kSuspendNs = 20000;
 constexpr size_t kOneCtaSmem = 116 * 1024;  // more than half of the SM's shared memory
 
 static_assert(kTotCol + kMBlocks * kMmaN <= kTmemCols, "accumulators and totals");
@@ -185,10 +188,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, bool o
     for (;;) {
         uint32_t done;
         asm volatile("{\n\t.reg .pred p;\n\t"
-                     "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                     "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
                      "selp.u32 %0, 1, 0, p;\n\t}"
                      : "=r"(done)
-                     : "r"(smem_u32(bar)), "r"(parity)
+                     : "r"(smem_u32(bar)), "r"(parity), "n"(kSuspendNs)
                      : "memory");
         if (done)
             return true;

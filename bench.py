@@ -1025,11 +1025,19 @@ def run_batch(batches=(1, 2, 4, 8, 16), n_steps: int = 64):
         us = time_calls(lambda i: f.ffn_fused(i % R), n, R) * 1e3 / n
         ux, uh = float(np.mean(f.union_x)), float(np.mean(f.union_h))
         wbytes = ux * f.H * f.I + uh * f.I * f.H / 2    # codes of the union rows (gate+up, down)
+        # algorithmic bytes of the FFN: codes and (scale, zero) of every group
+        # the union rows touch (all of them at these densities), x, h and y
+        G_in, G_h = f.H // f.g, f.I // f.g
+        abytes = (wbytes + G_in * 2 * f.I * 4 + G_h * f.H * 4
+                  + 2 * B * f.H + 2 * B * f.I * 2 + 2 * B * f.H)
+        peak, _ = measured_peak()
         out.append({"batch": B, "us_per_ffn": round(us, 2), "launches": 4,
                     "us_per_ffn_select_kernels": round(us6, 2), "launches_select_kernels": 6,
                     "union_active_in": round(ux, 3),
                     "union_active_h": round(uh, 3),
                     "weight_code_GBps": round(wbytes / (us * 1e-6) / 1e9, 1),
+                    "algorithmic_bytes": int(abytes),
+                    "frac_of_measured_peak": round(abytes / (us * 1e-6) / 1e9 / peak, 4),
                     "tokens_per_s_equiv_ffn_only_64_layers": round(B * 1e6 / (64 * us), 1)})
     return {"workload": "Qwen3-32B FFN decode (hidden 5120, intermediate 25600, int4 g128, "
                         "SiLU): per-row 50% thresholds, union active sets found inside each GEMV "

@@ -126,6 +126,28 @@ def test_thresh_batch_qwen_down_sampled(B):
     assert gg.workspace_is_zero()
 
 
+@pytest.mark.parametrize("B", [2, 5, 8, 16])
+def test_glu_thresh_batch_qwen_gate_up_sampled(B):
+    """The Qwen3-32B stacked gate/up shape (K = 5120, I = 25600: 50 output
+    tiles, equal per-SM shares that span tile boundaries) through the fused
+    GLU form at batch B, checked on sampled outputs of h."""
+    I, K, g = 25600, 5120, 128
+    Wg, Wu = wl.weight(I, K, 80), wl.weight(I, K, 81)
+    x = wl.x_silu_gated(B, K, 82 + B)
+    t = [wl.percentile_threshold(x[b], 0.5) for b in range(B)]
+    gl = GpuGlu(Wg, Wu, g, B)
+    h, h32 = gl.outputs(B)
+    sgq.sgq_gemv_glu_thresh_batch(gl.qw, gl.sz, I, K, g, x.to(DEV), B, t, sgq.SGQ_ACT_SILU, h,
+                                  h32, gl.ws, gl.status)
+    torch.cuda.synchronize()
+    rows = sample_rows(I, 40, seed=B)
+    _, h64, a64, u64, sag, sau = fused_expect(Wg, Wu, g, x, t, sgq.SGQ_ACT_SILU, rows=rows)
+    check_h(h, h32, h64, a64, u64, sag, sau, sgq.SGQ_ACT_SILU, rows=rows,
+            what=f"qwen gate/up B={B}")
+    assert bool((gl.ws == 0).all().item())
+    assert sgq.sgq_read_status(gl.status) == 0
+
+
 @pytest.mark.parametrize("B", [2, 5, 16])
 @pytest.mark.parametrize("act", [sgq.SGQ_ACT_SILU, sgq.SGQ_ACT_RELU])
 def test_glu_thresh_batch(B, act):
