@@ -315,7 +315,7 @@ __device__ int segment_rows(const GemvProblem &p, int lo, int hi, int32_t *ridx,
                     act = (__ldg(p.mask + (c >> 5)) >> (c & 31)) & 1u;
                 } else {
                     for (int b = 0; b < p.B; ++b)
-                        act = act || (fabsf(bf16_bits_to_float(__ldg(p.x + (size_t)b * p.K + c))) >
+                        act |= (fabsf(bf16_bits_to_float(__ldg(p.x + (size_t)b * p.K + c))) >
                                       p.tb[b]);
                 }
             }
@@ -399,6 +399,18 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
     const int lg = kp.lg;
     bool ok = true;
 
+    // With a fixed row source (dense, bitmask, threshold) the channels of this
+    // CTA's first segment are known now: their x (every batch row) is
+    // requested into L2 before the wait, a hint only (the loads after the
+    // wait see whatever the previous kernel wrote).
+    if (SRC != ROWS_LIST && warp == 0 && lane < p.B) {
+        const long long W0 = (long long)kp.n_tiles * (p.K / 8);
+        const int v0 = (int)(W0 * blockIdx.x / gridDim.x), v1 = (int)(W0 * (blockIdx.x + 1) / gridDim.x);
+        const int pt = p.K / 8, t0 = v0 / pt;
+        const int lo = v0 - t0 * pt, hi = min(pt, v1 - t0 * pt);
+        if (hi > lo)
+            prefetch_l2_bulk(p.x + (size_t)lane * p.K + 8 * lo, 16u * (uint32_t)(hi - lo));
+    }
     grid_dependency_wait(); // x, idx, count, mask may come from the previous kernel
 
     // This CTA's equal share [u0, u1) of the (tile, row) work: units of one
@@ -520,12 +532,17 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
             // ---- the MMA issuer --------------------------------------------------
             if (lane == 0) {
                 int run = 0;
+                int ist = kb_base % nst, iph = (kb_base / nst) & 1; // stage, phase of K-block 0
                 for (int kb = 0; kb < nkb; ++kb) {
                     kb_run(kb, run);
                     const bool first = kb == rkb[run], last = kb == rkb[run + 1] - 1;
-                    const int kg = kb_base + kb, rg = run_base + run;
-                    const int s = kg % nst;
-                    ok = mbar_wait(bar_full + s, (uint32_t)((kg / nst) & 1), ok);
+                    const int rg = run_base + run;
+                    const int s = ist;
+                    ok = mbar_wait(bar_full + s, (uint32_t)iph, ok);
+                    if (++ist == nst) {
+                        ist = 0;
+                        iph ^= 1;
+                    }
                     tc_fence_after();
                     if (first && rg >= 2) {
                         ok = mbar_wait(bar_free + (rg & 1), (uint32_t)(((rg >> 1) - 1) & 1), ok);
@@ -725,10 +742,11 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
             // previous run's fold, one K-block into the next run (its MMAs have
             // had that long to finish).
             int run = 0;
+            int est = kb_base % nst, eph = (kb_base / nst) & 1; // stage, phase of K-block 0
             auto step = [&](int kb, const uint4 *v) {
                 kb_run(kb, run);
                 const int kg = kb_base + kb;
-                const int s = kg % nst;
+                const int s = est;
                 const int j0 = kbj[kb];
                 const int nv = kbn[kb]; // valid slots (may exceed KB)
                 const bool first = kb == rkb[run];
@@ -745,7 +763,7 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
                 }
                 // The stage's previous K-block has been multiplied.
                 if (kg >= nst)
-                    ok = mbar_wait(bar_empty + s, (uint32_t)((kg / nst - 1) & 1), ok);
+                    ok = mbar_wait(bar_empty + s, (uint32_t)(eph ^ 1), ok);
                 const uint32_t a_st = sA + (uint32_t)(s * AST);
     #pragma unroll
                 for (int u = 0; u < SPW; ++u) {
@@ -754,14 +772,12 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
                     const uint32_t wv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
     #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        uint32_t t0 = 0u, t1 = 0u, t2 = 0u, t3 = 0u;
-                        if (valid) {
-                            const uint32_t w = wv[j], w8 = w >> 8;
-                            t0 = hsub2(w & 0x000F000Fu, zc[j][0]);
-                            t1 = hsub2(w & 0x00F000F0u, zc[j][1]);
-                            t2 = hsub2(w8 & 0x000F000Fu, zc[j][2]);
-                            t3 = hsub2(w8 & 0x00F000F0u, zc[j][3]);
-                        }
+                        // invalid slots hold zero codes and meet a zero B operand
+                        const uint32_t w = wv[j], w8 = w >> 8;
+                        const uint32_t t0 = hsub2(w & 0x000F000Fu, zc[j][0]);
+                        const uint32_t t1 = hsub2(w & 0x00F000F0u, zc[j][1]);
+                        const uint32_t t2 = hsub2(w8 & 0x000F000Fu, zc[j][2]);
+                        const uint32_t t3 = hsub2(w8 & 0x00F000F0u, zc[j][3]);
                         st_shared_v4(a_st + aoff[u][j], t0, t1, t2, t3);
                     }
                     if (lane < kMmaN) {
@@ -782,6 +798,10 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
                 const int fold_kb = rkb[run] + min(1, rkb[run + 1] - rkb[run] - 1);
                 if (run > 0 && kb == fold_kb)
                     fold(run - 1);
+                if (++est == nst) {
+                    est = 0;
+                    eph ^= 1;
+                }
             };
 
             for (int kb0 = 0; kb0 < nkb; kb0 += PF) {

@@ -180,7 +180,7 @@ __device__ int build_rows(const KParams &kp, int split, int32_t *ridx, float *rx
             bool act = false;
             if (c < c1)
                 for (int b = 0; b < p.B; ++b)
-                    act = act || (fabsf(bf16_bits_to_float(__ldg(p.x + (size_t)b * p.K + c))) >
+                    act |= (fabsf(bf16_bits_to_float(__ldg(p.x + (size_t)b * p.K + c))) >
                                   p.tb[b]);
             return __ballot_sync(0xffffffffu, act);
         };
