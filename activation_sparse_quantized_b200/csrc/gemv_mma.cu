@@ -140,8 +140,10 @@ __host__ __device__ inline int rxh_stride(int rows_cap) { return (((rows_cap + 7
 
 // a: `stages` A stages (1024-aligned); b: B stages; rxh: x' of the CTA's
 // rows, [bp batch rows][stride] fp16; ridx: the CTA's rows; rstart / rkb:
-// first row / first K-block of each run (+1 entry); kbj / kbn: first row and
-// number of valid rows of each K-block; scan: per-32-row counts.
+// first row / first K-block of each run (+1 entry); kbj: first row of each
+// K-block; kbn: each K-block's valid rows (bits 0-7), its run (bits 8-28),
+// whether it opens its run (bit 30) and whether the previous run folds
+// after it (bit 29); scan: per-32-row counts.
 __host__ __device__ inline SmemM smemm_layout(int rows_cap, int stages, int bp, int kb)
 {
     SmemM s;
@@ -504,8 +506,12 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
         }
         __syncthreads();
         const int nkb = s_nkb;
-        // First row and valid rows of every K-block (its run by a binary search
-        // over the runs' first K-blocks), so that neither side walks the runs.
+        // First row, valid rows, run and flags of every K-block (its run by a
+        // binary search over the runs' first K-blocks), so that the expansion
+        // warps read one word per K-block instead of walking the runs. The
+        // previous run folds one K-block into a run (on its only K-block when
+        // it has one). rows_cap, bounded by shared memory, keeps the run index
+        // far inside its 21 bits.
         for (int t = tid; t < nkb; t += kMThreads) {
             int lo = 0, hi = nruns - 1; // the run r with rkb[r] <= t < rkb[r + 1]
             while (lo < hi) {
@@ -517,12 +523,13 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
             }
             const int j0 = rstart[lo] + KB * (t - rkb[lo]);
             kbj[t] = j0;
-            kbn[t] = rstart[lo + 1] - j0; // may exceed KB
+            const int fkb = rkb[lo] + min(1, rkb[lo + 1] - rkb[lo] - 1);
+            kbn[t] = min(rstart[lo + 1] - j0, KB) | (lo << 8) | ((t == rkb[lo]) << 30) |
+                     ((t == fkb) << 29);
         }
         __syncthreads();
 
-        // K-block kb: its run (a pointer advanced monotonically), the ridx
-        // position of its slot 0 and its valid slots.
+        // The issuer's run of K-block kb (a pointer advanced monotonically).
         auto kb_run = [&](int kb, int &run) {
             while (kb >= rkb[run + 1])
                 ++run;
@@ -622,7 +629,7 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
             // K-block's valid rows; lanes past N read column 0).
             auto fetch = [&](int kb, uint4 *dst) {
                 if (kb < nkb) {
-                    const int j0 = kbj[kb], nv = kbn[kb];
+                    const int j0 = kbj[kb], nv = kbn[kb] & 0xFF;
     #pragma unroll
                     for (int u = 0; u < SPW; ++u) {
                         const int slot = warp + 16 * u;
@@ -744,12 +751,13 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
             int run = 0;
             int est = kb_base % nst, eph = (kb_base / nst) & 1; // stage, phase of K-block 0
             auto step = [&](int kb, const uint4 *v) {
-                kb_run(kb, run);
+                const int fl = kbn[kb];
+                const int j0 = kbj[kb];
+                const int nv = fl & 0xFF; // valid slots of the K-block (at most KB)
+                run = (fl >> 8) & 0x1FFFFF;
                 const int kg = kb_base + kb;
                 const int s = est;
-                const int j0 = kbj[kb];
-                const int nv = kbn[kb]; // valid slots (may exceed KB)
-                const bool first = kb == rkb[run];
+                const bool first = (fl >> 30) & 1;
                 if (first) {
                     unpack_z(grp(rstart[run])); // this run's zero points (in L1 since a run ago)
                     if (run + 1 < nruns)
@@ -795,8 +803,7 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
                 __syncwarp();
                 if (lane == 0)
                     mbar_arrive(bar_full + s);
-                const int fold_kb = rkb[run] + min(1, rkb[run + 1] - rkb[run] - 1);
-                if (run > 0 && kb == fold_kb)
+                if (run > 0 && ((fl >> 29) & 1))
                     fold(run - 1);
                 if (++est == nst) {
                     est = 0;
