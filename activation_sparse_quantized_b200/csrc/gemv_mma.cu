@@ -14,29 +14,31 @@
 // CTA; there each code is expanded once into an exact fp16 operand and the
 // products go to the tensor cores (tcgen05.mma kind::f16, fp32 accumulators
 // in tensor memory):
-//  * Tiles of 1024 outputs (512 bytes of a packed row) and k_splits shares of
-//    the rows per tile, as in the batch-1 kernel, with the same row lists.
+//  * Every CTA takes an equal share of the (tile, row) space, tiles of 1024
+//    outputs (512 bytes of a packed row); a share that ends one tile and
+//    starts the next is processed as two segments.
 //  * The CTA's rows are cut into runs of one quantization group, and each run
 //    into K-blocks of 32 rows (two MMA K-steps; 16 where two 64 KB operand
 //    stages do not fit shared memory), a run's last block padded with zero
 //    rows.
 //  * 16 expanding warps; warp w expands slots w and w + 16 of every K-block.
-//    Its lanes stream their own 16-byte columns of its rows through per-lane
-//    cp.async rings (4 rows ahead) and turn each code, minus the group's zero,
-//    into the exact fp16 value (q - z) 2^-24 (2^-20 for the high nibble of a
-//    byte): one AND and one packed fp16 subtraction per two codes, the zero
-//    being held in the same subnormal form. A K-block's A operand (1024
-//    outputs x its rows, M-major, 128-byte swizzle) and B operand (its rows
-//    x 16 batch columns of x' = x 2^S_b in fp16, K-major) go to one of 2..4
-//    stages.
-//  * A 17th warp issues the K-block's MMAs (8 per K-step: M = 128 outputs,
-//    N = 16, K = 16) into the run's accumulators (two alternating sets of 8 x 16
-//    columns of tensor memory), then commits them to the stage's "empty"
-//    barrier and, at a run's end, to the set's "ready" barrier.
-//  * A run later the expanding warps read their outputs' sums from tensor
-//    memory and fold them with the group's scale into running totals, also
-//    in tensor memory: total += s 2^c D. The products are those of the
-//    batch-1 kernel (exact fp16 x fp16), summed in fp32.
+//    Its lanes read their own 16-byte columns of its rows into registers (4
+//    rows ahead) and store each code as the exact fp16 value q 2^-24 (2^-20
+//    for the high nibble of a byte): one AND per two codes, no zero point. A
+//    K-block's A operand (1024 outputs x its rows, M-major, 128-byte swizzle)
+//    and B operand (its rows x 16 batch columns of x' = x 2^S_b in fp16,
+//    K-major) go to one of 2..4 stages.
+//  * A 17th warp issues the K-block's MMAs (9 per K-step: M = 128 outputs,
+//    N = 16, K = 16, the ninth with an all-ones A operand, so that its
+//    accumulator holds the sum of x' over the run) into the run's accumulator
+//    set (one of two, 9 x 16 columns of tensor memory each), then commits them
+//    to the stage's "empty" barrier and, at a run's end, to the set's "ready"
+//    barrier.
+//  * One K-block into the next run the expanding warps read their outputs'
+//    sums D and the row sums X from tensor memory and fold them with the
+//    group's scale and zero into running totals, also in tensor memory:
+//    total += s (2^c D - z X), i.e. the sum of s (q - z) x'. The products
+//    are exact (fp16 x fp16), summed in fp32.
 //  * Split-K partials go into the fp32 workspace with float reductions; the
 //    shared epilogue kernel turns the workspace into bf16 y.
 //
@@ -75,13 +77,19 @@ __host__ __device__ constexpr int b_stage_bytes(int kb) { return kb * kMmaN * 2;
 constexpr int kMaxStages = 4;               // operand stages (2..4, by shared memory)
 constexpr int kPfRows = 4;                  // rows of packed codes in flight per expanding lane
 constexpr int kTmemCols = 512;              // two accumulator sets and the running totals
-constexpr int kTotCol = 256;                // first column of the totals
+// An accumulator set: the tile's 8 M-blocks and the row-sum block (below),
+// 16 columns each, 160 columns apart; the totals after both sets.
+constexpr int kSetCols = 160;
+constexpr int kSumCol = kMBlocks * kMmaN;    // the row-sum block inside a set
+constexpr int kTotCol = 2 * kSetCols;        // first column of the totals
+constexpr int kOnesBytes = 4096;             // the all-ones A operand of the row-sum block
 constexpr unsigned long long kWaitNs = 200000000ull; // a barrier wait gives up after 0.2 s
 // A thread in a barrier wait sleeps until the phase completes or this many
 // ns pass (then checks the wall-time limit), instead of spinning on it.
 constexpr unsigned kSuspendNs = 20000;
 constexpr size_t kOneCtaSmem = 116 * 1024;  // more than half of the SM's shared memory
 
+static_assert(kSumCol + kMmaN <= kSetCols, "an accumulator set");
 static_assert(kTotCol + kMBlocks * kMmaN <= kTmemCols, "accumulators and totals");
 
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 D, fp16 A and B,
@@ -129,7 +137,7 @@ __device__ __forceinline__ uint32_t b_elem_off(int c, int k, int kb)
 }
 
 struct SmemM {
-    size_t a, b, rxh, ridx, rstart, rkb, kbj, kbn, scan, total;
+    size_t a, ones, b, rxh, ridx, rstart, rkb, kbj, kbn, scan, total;
 };
 
 __host__ __device__ inline size_t align16(size_t v) { return (v + 15) / 16 * 16; }
@@ -138,7 +146,8 @@ __host__ __device__ inline size_t align16(size_t v) { return (v + 15) / 16 * 16;
 // that the 16 batch columns of one row fall into distinct bank pairs.
 __host__ __device__ inline int rxh_stride(int rows_cap) { return (((rows_cap + 7) / 8) | 1) * 8; }
 
-// a: `stages` A stages (1024-aligned); b: B stages; rxh: x' of the CTA's
+// a: `stages` A stages (1024-aligned); ones: the row-sum block's A operand
+// (fp16 1.0, 1024-aligned); b: B stages; rxh: x' of the CTA's
 // rows, [bp batch rows][stride] fp16; ridx: the CTA's rows; rstart / rkb:
 // first row / first K-block of each run (+1 entry); kbj: first row of each
 // K-block; kbn: each K-block's valid rows (bits 0-7), its run (bits 8-28),
@@ -148,7 +157,8 @@ __host__ __device__ inline SmemM smemm_layout(int rows_cap, int stages, int bp, 
 {
     SmemM s;
     s.a = 0;
-    s.b = s.a + (size_t)stages * a_stage_bytes(kb);
+    s.ones = s.a + (size_t)stages * a_stage_bytes(kb);
+    s.b = s.ones + kOnesBytes;
     s.rxh = s.b + (size_t)stages * b_stage_bytes(kb);
     s.ridx = align16(s.rxh + (size_t)bp * rxh_stride(rows_cap) * 2);
     s.rstart = align16(s.ridx + (size_t)rows_cap * 4);
@@ -255,13 +265,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t addr, const float *v)
                  : "memory");
 }
 
-__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b)
-{
-    uint32_t d;
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d)
 {
@@ -270,11 +273,6 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                  : "memory");
 }
 
-// Integer zero point (0..15) of an (s, z) fp16 pair.
-__device__ __forceinline__ uint32_t zero_of(uint32_t w)
-{
-    return (uint32_t)__float2int_rn(__half2float(__ushort_as_half((uint16_t)(w >> 16))));
-}
 
 // Rows of one segment into ridx (ascending positions of the caller's list, or
 // of the active channels), returns their number. Index list: entries
@@ -372,6 +370,16 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
     int *kbn = reinterpret_cast<int *>(smem + L.kbn);
     int *scan = reinterpret_cast<int *>(smem + L.scan);
     const uint32_t sA = smem_u32(smem + L.a), sB = smem_u32(smem + L.b);
+    const uint32_t sOnes = smem_u32(smem + L.ones);
+
+    // The row-sum block's A operand: every element fp16 1.0, so that its
+    // accumulator holds, in every row, the sum of x' over the run's rows for
+    // each batch column (whatever the operand's layout, all elements being
+    // equal). Written once, made visible to the tensor core's reads.
+    for (int i = tid; i < kOnesBytes / 16; i += kMThreads)
+        reinterpret_cast<uint4 *>(smem + L.ones)[i] =
+            make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -556,10 +564,10 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
                         tc_fence_after();
                     }
                     const uint32_t a_st = sA + (uint32_t)(s * AST);
-                    const uint32_t dcol = tmem + (uint32_t)(128 * (rg & 1));
+                    const uint32_t dcol = tmem + (uint32_t)(kSetCols * (rg & 1));
                     // Every M-block: a lane's outputs are spread over the M-blocks
                     // (lanes past N hold finite codes of column 0 and are dropped
-                    // in the epilogue).
+                    // in the epilogue); then the row sums of x'.
     #pragma unroll
                     for (int kk = 0; kk < KB / kKStep; ++kk) {
                         const uint64_t bdesc = smem_desc(
@@ -570,6 +578,8 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
                                     smem_desc(a_st + (uint32_t)(kk * 32768 + mb * 2048), 1024,
                                               16 * 1024, 2),
                                     bdesc, !first || kk > 0);
+                        mma_f16(dcol + (uint32_t)kSumCol, smem_desc(sOnes, 1024, 2048, 2), bdesc,
+                                !first || kk > 0);
                     }
                     mma_commit(bar_empty + s);
                     if (last && !(p.debug_withhold_ready && run == nruns - 1))
@@ -660,35 +670,6 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
                 boff[u] = b_elem_off(lane & 15, warp + 16 * u, KB);
             }
 
-            // Zero points of this lane's 32 outputs for one group, as subnormal
-            // fp16 pairs matching the AND results: word j, pairs = outputs
-            // (8j, 8j+4), (8j+1, 8j+5) << 4, (8j+2, 8j+6), (8j+3, 8j+7) << 4.
-            // The next run's scale/zero slice of the tile (4 KB) is prefetched
-            // into L1 a run ahead by warp 0, one 128-byte line per lane; every
-            // warp reads its lanes' words from there at the run's start.
-            auto load_sz = [&](int G) {
-                if (warp == 0)
-                    asm volatile("prefetch.global.L1 [%0];" ::"l"(
-                        p.sz + (size_t)G * p.N + n0 + (lane_ok ? lane * 32 : 0)));
-            };
-            uint32_t zc[4][4];
-            auto unpack_z = [&](int G) {
-                const uint4 *src = reinterpret_cast<const uint4 *>(p.sz + (size_t)G * p.N + n0 +
-                                                                   (lane_ok ? lane * 32 : 0));
-    #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint4 a = __ldg(src + 2 * j), c = __ldg(src + 2 * j + 1);
-                    const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
-                    uint32_t z[8];
-    #pragma unroll
-                    for (int o = 0; o < 8; ++o)
-                        z[o] = lane_ok ? zero_of(w[o]) : 0u;
-                    zc[j][0] = z[0] | (z[4] << 16);
-                    zc[j][1] = (z[1] | (z[5] << 16)) << 4;
-                    zc[j][2] = z[2] | (z[6] << 16);
-                    zc[j][3] = (z[3] | (z[7] << 16)) << 4;
-                }
-            };
             // Fold outputs of this thread: its tensor-memory lane (quadrant
             // warp % 4) in M-blocks 2 (warp / 4) and 2 (warp / 4) + 1.
             const int mbA = 2 * (warp >> 2);
@@ -705,33 +686,41 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
                 for (int i = 0; i < 2; ++i)
                     sv[i] = (fout[i] < nvalid_out) ? __ldg(p.sz + (size_t)G * p.N + n0 + fout[i]) : 0u;
             };
-            if (nruns > 0) {
-                load_sz(grp(rstart[0]));
+            if (nruns > 0)
                 load_s(grp(rstart[0]), snew);
-            }
 
-            // totals += s 2^c D for run r's accumulators (set r & 1); the totals
-            // stay in tensor memory (columns kTotCol..), written by run 0.
+            // totals += s (2^c D - z X) for run r's accumulators (set r & 1):
+            // D sums the raw codes q 2^-c times x' over the run's rows, X (the
+            // row-sum block) sums x', so that s (q - z) x' is summed with no
+            // zero point in the operand (z: an integer-valued fp16, s z exact
+            // in fp32). The totals stay in tensor memory (columns kTotCol..),
+            // written by run 0.
             auto fold = [&](int r) { // r: run of this segment
                 const int rg = run_base + r;
                 ok = mbar_wait(bar_ready + (rg & 1), (uint32_t)((rg >> 1) & 1), ok);
                 tc_fence_after();
+                const uint32_t set = tmem + tlane + (uint32_t)(kSetCols * (rg & 1));
     #pragma unroll
                 for (int i = 0; i < 2; ++i) {
                     float d[kMmaN], t[kMmaN];
-                    tmem_ld16(tmem + tlane + 128 * (rg & 1) + kMmaN * (mbA + i), d);
-                    const float f = __half2float(__ushort_as_half((uint16_t)(sfold[i] & 0xffffu))) *
-                                    ((fout[i] & 1) ? 1048576.f : 16777216.f);
+                    const float sc = __half2float(__ushort_as_half((uint16_t)(sfold[i] & 0xffffu)));
+                    const float f = sc * ((fout[i] & 1) ? 1048576.f : 16777216.f);
+                    const float nsz = -sc * __half2float(__ushort_as_half((uint16_t)(sfold[i] >> 16)));
+                    tmem_ld16(set + kSumCol, d); // X
                     if (r == 0) {
     #pragma unroll
                         for (int c = 0; c < kMmaN; ++c)
-                            t[c] = f * d[c];
+                            t[c] = nsz * d[c];
                     } else {
                         tmem_ld16(tmem + tlane + kTotCol + kMmaN * (mbA + i), t);
     #pragma unroll
                         for (int c = 0; c < kMmaN; ++c)
-                            t[c] = fmaf(f, d[c], t[c]);
+                            t[c] = fmaf(nsz, d[c], t[c]);
                     }
+                    tmem_ld16(set + kMmaN * (mbA + i), d); // D
+    #pragma unroll
+                    for (int c = 0; c < kMmaN; ++c)
+                        t[c] = fmaf(f, d[c], t[c]);
                     tmem_st16(tmem + tlane + kTotCol + kMmaN * (mbA + i), t);
                 }
                 asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
@@ -757,17 +746,11 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
                 run = (fl >> 8) & 0x1FFFFF;
                 const int kg = kb_base + kb;
                 const int s = est;
-                const bool first = (fl >> 30) & 1;
-                if (first) {
-                    unpack_z(grp(rstart[run])); // this run's zero points (in L1 since a run ago)
-                    if (run + 1 < nruns)
-                        load_sz(grp(rstart[run + 1]));
-                    if (run > 0) {
+                if (((fl >> 30) & 1) && run > 0) { // a run's first K-block
     #pragma unroll
-                        for (int i = 0; i < 2; ++i)
-                            sfold[i] = snew[i];
-                        load_s(grp(rstart[run]), snew); // this run's scales, for its fold
-                    }
+                    for (int i = 0; i < 2; ++i)
+                        sfold[i] = snew[i];
+                    load_s(grp(rstart[run]), snew); // this run's (s, z), for its fold
                 }
                 // The stage's previous K-block has been multiplied.
                 if (kg >= nst)
@@ -780,13 +763,12 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
                     const uint32_t wv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
     #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        // invalid slots hold zero codes and meet a zero B operand
+                        // The raw codes as exact fp16 subnormals: q 2^-24 (low
+                        // nibbles) and q 2^-20 (high); invalid slots hold zero
+                        // codes and meet a zero B operand.
                         const uint32_t w = wv[j], w8 = w >> 8;
-                        const uint32_t t0 = hsub2(w & 0x000F000Fu, zc[j][0]);
-                        const uint32_t t1 = hsub2(w & 0x00F000F0u, zc[j][1]);
-                        const uint32_t t2 = hsub2(w8 & 0x000F000Fu, zc[j][2]);
-                        const uint32_t t3 = hsub2(w8 & 0x00F000F0u, zc[j][3]);
-                        st_shared_v4(a_st + aoff[u][j], t0, t1, t2, t3);
+                        st_shared_v4(a_st + aoff[u][j], w & 0x000F000Fu, w & 0x00F000F0u,
+                                     w8 & 0x000F000Fu, w8 & 0x00F000F0u);
                     }
                     if (lane < kMmaN) {
                         // B operand: x' of this slot for batch column `lane`.
