@@ -28,7 +28,7 @@
 //    subnormals; a mixed-precision FMA (fp16 x fp16 + fp32) multiplies each by
 //    x held in fp16 under a per-warp power-of-two scale, so every product is
 //    exact. Scale and zero are applied once per (group, output) in a fold.
-//  * B = 2..6: each warp carries two batch rows, which share the extracted codes;
+//  * B = 2..4: each warp carries two batch rows, which share the extracted codes;
 //    the warps form ceil(B / 2) (rounded to a power of two) batch groups that
 //    read the same rows, the later reads hitting L2, so HBM still sees each
 //    active row once.
@@ -799,10 +799,11 @@ cudaError_t launch_gemv(const GemvProblem &p, int num_sms, cudaStream_t stream)
     KParams kp{};
     kp.p = p;
     kp.lg = __builtin_ctz((unsigned)p.group);
-    // B > 6 over the plain layout: the tensor-core kernel. Up to 6 rows the
+    // B > 4 over the plain layout: the tensor-core kernel. Up to 4 rows the
     // CUDA-core kernel (two batch rows per warp, one FMA per code and row)
-    // measured faster; above, its cost keeps growing with the rows.
-    if (p.B > 6 && !p.keep &&
+    // measured faster; from 5 its cost steps up (a third batch group of
+    // warps) and keeps growing with the rows.
+    if (p.B > 4 && !p.keep &&
         (p.source == ROWS_LIST || p.source == ROWS_DENSE || p.source == ROWS_MASK ||
          p.source == ROWS_THRESH))
         return launch_gemv_mma(p, num_sms, stream);

@@ -1,4 +1,4 @@
-// gemv_mma.cu -- the activation-sparse GEMV for batch 7..16, on the tensor cores.
+// gemv_mma.cu -- the activation-sparse GEMV for batch 5..16, on the tensor cores.
 //
 //   y[b][n] = sum_{k in U} s[g(k)][n] * (q[k][n] - z[g(k)][n]) * x[b][k]
 //

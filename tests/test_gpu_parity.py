@@ -199,14 +199,14 @@ def test_gemv_qwen_down_batch(B):
     run_list_case(case, rows=sample_rows(h, 256, B), what=f"qwen down B={B}")
 
 
-@pytest.mark.parametrize("B", [1, 4, 7, 16])
+@pytest.mark.parametrize("B", [1, 4, 5, 16])
 def test_gemv_qwen_up_batch(B):
     h, I = wl.QWEN32B_FFN["hidden"], wl.QWEN32B_FFN["inter"]
     case = wl.gemv_case(N=I, K=h, group=128, B=B, sparsity=0.5, seed=40 + B)
     run_list_case(case, rows=sample_rows(I, 256, B), what=f"qwen up B={B}")
 
 
-@pytest.mark.parametrize("B", [2, 3, 5, 6, 7, 8, 9, 16])
+@pytest.mark.parametrize("B", [2, 3, 4, 5, 6, 7, 8, 9, 16])
 def test_gemv_batch_ragged(B):
     case = wl.gemv_case(N=3168, K=4160, group=64, B=B, sparsity=0.6, seed=50 + B)
     run_list_case(case, what=f"ragged B={B}")
@@ -320,12 +320,12 @@ def test_gemv_thresh_ragged(N, K, g):
     check_y(y, y32, y64, sa, "thresh ragged")
 
 
-@pytest.mark.parametrize("B", [1, 3, 6, 7, 8, 12])
+@pytest.mark.parametrize("B", [1, 3, 4, 5, 6, 8, 12])
 def test_gemv_exact_integer_case_bitwise(B):
     """Power-of-two scales and small-integer x: every partial sum on both sides
     is exact, so fp32 y equals the oracle's fp64 y and bf16 y matches bitwise
-    (B = 3, 6: the CUDA-core batch kernel; B = 7, 8, 12: the tensor-core
-    kernel, whose products and fp32 sums are exact here too)."""
+    (B = 3, 4: the CUDA-core batch kernel; B = 5, 6, 8, 12: the tensor-core
+    kernel, whose products, row sums and fp32 sums are exact here too)."""
     rng = np.random.default_rng(80 + B)
     N, K, g = 2048, 1024, 64
     G = K // g
@@ -344,7 +344,7 @@ def test_gemv_exact_integer_case_bitwise(B):
     assert np.array_equal(bits(y), yb)
 
 
-@pytest.mark.parametrize("B", [1, 7, 12])
+@pytest.mark.parametrize("B", [1, 5, 12])
 def test_gemv_power_of_two_scaling(B):
     case = wl.gemv_case(N=2048, K=4096, group=128, B=B, sparsity=0.5, seed=81, act="silu")
     g = GpuGemv(case.W, 128, B)
