@@ -218,12 +218,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, bool o
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                        bool accumulate)
+// One MMA; the descriptors come as their 32-bit halves, so that the issuer
+// offsets a K-block's descriptors with one 32-bit add each (the start-address
+// field never carries into the next field inside shared memory).
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint32_t alo, uint32_t ahi, uint32_t blo,
+                                        uint32_t bhi, uint32_t accumulate)
 {
-    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-                 "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"((uint32_t)accumulate)
+    asm volatile("{\n\t.reg .pred p;\n\t.reg .b64 a, b;\n\tsetp.ne.b32 p, %5, 0;\n\t"
+                 "mov.b64 a, {%1, %2};\n\tmov.b64 b, {%3, %4};\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %6, p;\n\t}" ::"r"(d_tmem),
+                 "r"(alo), "r"(ahi), "r"(blo), "r"(bhi), "r"(accumulate), "r"(kIdesc)
                  : "memory");
 }
 
@@ -548,6 +552,7 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
             if (lane == 0) {
                 int run = 0;
                 int ist = kb_base % nst, iph = (kb_base / nst) & 1; // stage, phase of K-block 0
+                const uint64_t od = smem_desc(sOnes, 1024, 2048, 2);
                 for (int kb = 0; kb < nkb; ++kb) {
                     kb_run(kb, run);
                     const bool first = kb == rkb[run], last = kb == rkb[run + 1] - 1;
@@ -563,23 +568,25 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
                         ok = mbar_wait(bar_free + (rg & 1), (uint32_t)(((rg >> 1) - 1) & 1), ok);
                         tc_fence_after();
                     }
-                    const uint32_t a_st = sA + (uint32_t)(s * AST);
                     const uint32_t dcol = tmem + (uint32_t)(kSetCols * (rg & 1));
+                    const uint64_t ad = smem_desc(sA + (uint32_t)(s * AST), 1024, 16 * 1024, 2);
+                    const uint64_t bd = smem_desc(sB + (uint32_t)(s * BST), 128, (KB / 8) * 128, 0);
+                    const uint32_t alo = (uint32_t)ad, ahi = (uint32_t)(ad >> 32);
+                    const uint32_t blo = (uint32_t)bd, bhi = (uint32_t)(bd >> 32);
                     // Every M-block: a lane's outputs are spread over the M-blocks
                     // (lanes past N hold finite codes of column 0 and are dropped
                     // in the epilogue); then the row sums of x'.
     #pragma unroll
                     for (int kk = 0; kk < KB / kKStep; ++kk) {
-                        const uint64_t bdesc = smem_desc(
-                            sB + (uint32_t)(s * BST + kk * 256), 128, (KB / 8) * 128, 0);
+                        const uint32_t acc = (kk > 0 || !first) ? 1u : 0u;
+                        const uint32_t bk = blo + (uint32_t)((kk * 256) >> 4);
     #pragma unroll
                         for (int mb = 0; mb < kMBlocks; ++mb)
                             mma_f16(dcol + (uint32_t)(kMmaN * mb),
-                                    smem_desc(a_st + (uint32_t)(kk * 32768 + mb * 2048), 1024,
-                                              16 * 1024, 2),
-                                    bdesc, !first || kk > 0);
-                        mma_f16(dcol + (uint32_t)kSumCol, smem_desc(sOnes, 1024, 2048, 2), bdesc,
-                                !first || kk > 0);
+                                    alo + (uint32_t)((kk * 32768 + mb * 2048) >> 4), ahi, bk, bhi,
+                                    acc);
+                        mma_f16(dcol + (uint32_t)kSumCol, (uint32_t)od, (uint32_t)(od >> 32), bk,
+                                bhi, acc);
                     }
                     mma_commit(bar_empty + s);
                     if (last && !(p.debug_withhold_ready && run == nruns - 1))
