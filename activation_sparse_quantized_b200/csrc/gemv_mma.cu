@@ -286,7 +286,8 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 // 32 channels and a prefix over the runs' counts. All threads; ends with a
 // barrier.
 template <int SRC>
-__device__ int segment_rows(const GemvProblem &p, int lo, int hi, int32_t *ridx, int *scan)
+__device__ int segment_rows(const GemvProblem &p, int lo, int hi, int32_t *ridx, int *scan,
+                            uint16_t *rxh, int rs)
 {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (SRC == ROWS_LIST) {
@@ -338,9 +339,33 @@ __device__ int segment_rows(const GemvProblem &p, int lo, int hi, int32_t *ridx,
             for (int q = c * 32 + ((warp - c * 32) % kAllWarps + kAllWarps) % kAllWarps;
                  q < runs && q < c * 32 + 32; q += kAllWarps) {
                 const int base = __shfl_sync(0xffffffffu, excl, q - c * 32);
-                const uint32_t m = run_bits(q);
-                if ((m >> lane) & 1u)
-                    ridx[base + __popc(m & ((1u << lane) - 1u))] = c0 + q * 32 + lane;
+                if (SRC == ROWS_THRESH) {
+                    // The same test, keeping the rows' x: an active channel's x
+                    // goes to rxh (batch-major) at its position, so that the
+                    // x' staging needs no second gather.
+                    const int ch = c0 + q * 32 + lane;
+                    uint16_t v[kMmaN];
+                    bool act = false;
+    #pragma unroll
+                    for (int b = 0; b < kMmaN; ++b) {
+                        v[b] = (b < p.B && ch < c1) ? __ldg(p.x + (size_t)b * p.K + ch) : (uint16_t)0;
+                        act |= (b < p.B && ch < c1) &&
+                               (fabsf(bf16_bits_to_float(v[b])) > p.tb[b]);
+                    }
+                    const uint32_t m = __ballot_sync(0xffffffffu, act);
+                    if (act) {
+                        const int j = base + __popc(m & ((1u << lane) - 1u));
+                        ridx[j] = ch;
+    #pragma unroll
+                        for (int b = 0; b < kMmaN; ++b)
+                            if (b < p.B)
+                                rxh[(size_t)b * rs + j] = v[b];
+                    }
+                } else {
+                    const uint32_t m = run_bits(q);
+                    if ((m >> lane) & 1u)
+                        ridx[base + __popc(m & ((1u << lane) - 1u))] = c0 + q * 32 + lane;
+                }
             }
             total += ct;
         }
@@ -457,7 +482,7 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
         __syncthreads(); // the previous segment's readers of the row arrays are done
 
         // The segment's rows (invalid list entries are -1: read as row 0, x = 0).
-        const int nr = segment_rows<SRC>(p, lo, hi, ridx, scan);
+        const int nr = segment_rows<SRC>(p, lo, hi, ridx, scan, rxh, rxh_stride(kp.rows_cap));
         auto grp = [&](int j) { return max(ridx[j], 0) >> lg; };
 
         // Runs of one group: starts by ballots over chunks of 32 rows, positions
@@ -604,25 +629,39 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
             // x' = x 2^S_b in fp16 per batch row b, 2^14 <= max |x'| < 2^15 over
             // the CTA's rows (as in the batch-1 kernel), staged batch-major in
             // rxh. Warp w owns batch row b = w: lane l gathers rows l, l + 32,
-            // ... (one bf16 each, 16 loads in flight; consecutive channels make
+            // ... (one bf16 each, 32 loads in flight; consecutive channels make
             // each warp load one coalesced 64-byte request), then the warp
-            // reduces max |x| and converts its row in place.
+            // reduces max |x| and converts its row in place, 8 rows per lane
+            // loaded before any is stored.
             const int rs = rxh_stride(kp.rows_cap);
             if (warp < p.B) {
                 const int b = warp;
                 uint16_t *xr = rxh + (size_t)b * rs;
                 const uint16_t *xb = p.x + (size_t)b * p.K;
                 float m = 0.f;
-                for (int j0 = 0; j0 < nr; j0 += 32 * 16) {
-                    uint16_t v[16];
+                if (SRC == ROWS_THRESH) { // the row selection staged x already
+                    for (int j0 = 0; j0 < nr; j0 += 32 * 8) {
+                        uint16_t v[8];
     #pragma unroll
-                    for (int u = 0; u < 16; ++u) {
+                        for (int u = 0; u < 8; ++u) {
+                            const int j = j0 + 32 * u + lane;
+                            v[u] = (j < nr) ? xr[j] : (uint16_t)0;
+                        }
+    #pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            m = fmaxf(m, fabsf(bf16_bits_to_float(v[u])));
+                    }
+                }
+                for (int j0 = 0; SRC != ROWS_THRESH && j0 < nr; j0 += 32 * 32) {
+                    uint16_t v[32];
+    #pragma unroll
+                    for (int u = 0; u < 32; ++u) {
                         const int j = j0 + 32 * u + lane;
                         const int k = (j < nr) ? ridx[j] : -1;
                         v[u] = (k >= 0) ? __ldg(xb + k) : (uint16_t)0;
                     }
     #pragma unroll
-                    for (int u = 0; u < 16; ++u) {
+                    for (int u = 0; u < 32; ++u) {
                         const int j = j0 + 32 * u + lane;
                         if (j < nr) {
                             xr[j] = v[u];
@@ -636,8 +675,20 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
                     s_S[b] = S;
                 const float fa = pow2f(S - S / 2), fb = pow2f(S / 2);
                 __syncwarp();
-                for (int j = lane; j < nr; j += 32)
-                    xr[j] = __half_as_ushort(__float2half_rn((bf16_bits_to_float(xr[j]) * fa) * fb));
+                for (int j0 = 0; j0 < nr; j0 += 32 * 8) {
+                    uint16_t v[8];
+    #pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int j = j0 + 32 * u + lane;
+                        v[u] = (j < nr) ? xr[j] : (uint16_t)0;
+                    }
+    #pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int j = j0 + 32 * u + lane;
+                        if (j < nr)
+                            xr[j] = __half_as_ushort(__float2half_rn((bf16_bits_to_float(v[u]) * fa) * fb));
+                    }
+                }
             }
 
             const size_t row_bytes = (size_t)(p.N / 2);
