@@ -87,7 +87,7 @@ def test_gemv_mask_ragged(N, K, g):
     run_mask_case(case, what=f"mask ragged {N}x{K}")
 
 
-@pytest.mark.parametrize("B", [2, 4, 16])
+@pytest.mark.parametrize("B", [2, 4, 5, 6, 16])
 def test_gemv_mask_qwen_down_batch(B):
     cfg = wl.QWEN32B_FFN
     case = wl.gemv_case(N=cfg["hidden"], K=cfg["inter"], group=cfg["group"], B=B,

@@ -237,7 +237,7 @@ def test_gemv_dense_matches_oracle_and_full_list():
     assert g.workspace_is_zero()
 
 
-@pytest.mark.parametrize("B", [2, 8, 12])
+@pytest.mark.parametrize("B", [2, 4, 5, 8, 12])
 def test_gemv_dense_batch(B):
     case = wl.gemv_case(N=1024, K=4096, group=128, B=B, sparsity=0.0, seed=70)
     g = GpuGemv(case.W, 128, B)
@@ -247,7 +247,7 @@ def test_gemv_dense_batch(B):
     check_y(y, y32, y64, sa, f"dense B={B}")
 
 
-@pytest.mark.parametrize("B,g", [(9, 32), (12, 128), (16, 64)])
+@pytest.mark.parametrize("B,g", [(5, 64), (9, 32), (12, 128), (16, 64)])
 def test_gemv_batch_unsorted_list_with_repeats(B, g):
     """A caller's index list in no order, with repeated channels, at batch
     sizes of the tensor-core kernel: the list is cut into runs of one group
@@ -372,7 +372,7 @@ def test_gemv_all_masked_gives_positive_zero():
     assert g.workspace_is_zero()
 
 
-@pytest.mark.parametrize("B", [12, 16])
+@pytest.mark.parametrize("B", [5, 12, 16])
 def test_gemv_batch_all_masked_gives_positive_zero(B):
     """The tensor-core kernel with no active channel: no run, no MMA; y = +0
     and the workspace stays zero."""
@@ -388,7 +388,8 @@ def test_gemv_batch_all_masked_gives_positive_zero(B):
     assert g.status.item() == 0
 
 
-@pytest.mark.parametrize("N,K,g,B", [(96, 32, 32, 10), (992, 64, 32, 16), (1056, 128, 64, 9)])
+@pytest.mark.parametrize("N,K,g,B", [(96, 32, 32, 10), (992, 64, 32, 16), (1056, 128, 64, 9),
+                                     (96, 64, 32, 5), (1056, 128, 64, 6)])
 def test_gemv_batch_tiny_shapes(N, K, g, B):
     """The tensor-core kernel on one group, one partial tile, or a tile of
     1024 plus 32 outputs, dense and at 50% sparsity."""
