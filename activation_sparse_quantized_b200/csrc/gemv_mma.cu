@@ -137,7 +137,7 @@ __device__ __forceinline__ uint32_t b_elem_off(int c, int k, int kb)
 }
 
 struct SmemM {
-    size_t a, ones, b, rxh, ridx, rstart, rkb, kbj, kbn, scan, total;
+    size_t a, ones, b, rxh, ridx, rstart, rkb, kbt, scan, total;
 };
 
 __host__ __device__ inline size_t align16(size_t v) { return (v + 15) / 16 * 16; }
@@ -149,8 +149,8 @@ __host__ __device__ inline int rxh_stride(int rows_cap) { return (((rows_cap + 7
 // a: `stages` A stages (1024-aligned); ones: the row-sum block's A operand
 // (fp16 1.0, 1024-aligned); b: B stages; rxh: x' of the CTA's
 // rows, [bp batch rows][stride] fp16; ridx: the CTA's rows; rstart / rkb:
-// first row / first K-block of each run (+1 entry); kbj: first row of each
-// K-block; kbn: each K-block's valid rows (bits 0-7), its run (bits 8-28),
+// first row / first K-block of each run (+1 entry); kbt: per K-block, its
+// first row and a word of its valid rows (bits 0-7), its run (bits 8-28),
 // whether it opens its run (bit 30) and whether the previous run folds
 // after it (bit 29); scan: per-32-row counts.
 __host__ __device__ inline SmemM smemm_layout(int rows_cap, int stages, int bp, int kb)
@@ -163,9 +163,8 @@ __host__ __device__ inline SmemM smemm_layout(int rows_cap, int stages, int bp, 
     s.ridx = align16(s.rxh + (size_t)bp * rxh_stride(rows_cap) * 2);
     s.rstart = align16(s.ridx + (size_t)rows_cap * 4);
     s.rkb = align16(s.rstart + (size_t)(rows_cap + 1) * 4);
-    s.kbj = align16(s.rkb + (size_t)(rows_cap + 1) * 4);
-    s.kbn = align16(s.kbj + (size_t)(rows_cap + 1) * 4);
-    s.scan = align16(s.kbn + (size_t)(rows_cap + 1) * 4);
+    s.kbt = align16(s.rkb + (size_t)(rows_cap + 1) * 4);
+    s.scan = align16(s.kbt + (size_t)(rows_cap + 1) * 8);
     s.total = align16(s.scan + (size_t)((rows_cap + 31) / 32 + 4) * 4);
     return s;
 }
@@ -395,8 +394,7 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
     int32_t *ridx = reinterpret_cast<int32_t *>(smem + L.ridx);
     int *rstart = reinterpret_cast<int *>(smem + L.rstart);
     int *rkb = reinterpret_cast<int *>(smem + L.rkb);
-    int *kbj = reinterpret_cast<int *>(smem + L.kbj);
-    int *kbn = reinterpret_cast<int *>(smem + L.kbn);
+    int2 *kbt = reinterpret_cast<int2 *>(smem + L.kbt);
     int *scan = reinterpret_cast<int *>(smem + L.scan);
     const uint32_t sA = smem_u32(smem + L.a), sB = smem_u32(smem + L.b);
     const uint32_t sOnes = smem_u32(smem + L.ones);
@@ -408,6 +406,9 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
     for (int i = tid; i < kOnesBytes / 16; i += kMThreads)
         reinterpret_cast<uint4 *>(smem + L.ones)[i] =
             make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);
+    // The B stages start at zero: batch columns past B are never written.
+    for (int i = tid; i < nst * BST / 16; i += kMThreads)
+        reinterpret_cast<uint4 *>(smem + L.b)[i] = make_uint4(0u, 0u, 0u, 0u);
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 
     if (warp == 0) {
@@ -559,10 +560,9 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
                     hi = mid - 1;
             }
             const int j0 = rstart[lo] + KB * (t - rkb[lo]);
-            kbj[t] = j0;
             const int fkb = rkb[lo] + min(1, rkb[lo + 1] - rkb[lo] - 1);
-            kbn[t] = min(rstart[lo + 1] - j0, KB) | (lo << 8) | ((t == rkb[lo]) << 30) |
-                     ((t == fkb) << 29);
+            kbt[t] = make_int2(j0, min(rstart[lo + 1] - j0, KB) | (lo << 8) |
+                                       ((t == rkb[lo]) << 30) | ((t == fkb) << 29));
         }
         __syncthreads();
 
@@ -697,7 +697,8 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
             // K-block's valid rows; lanes past N read column 0).
             auto fetch = [&](int kb, uint4 *dst) {
                 if (kb < nkb) {
-                    const int j0 = kbj[kb], nv = kbn[kb] & 0xFF;
+                    const int2 e = kbt[kb];
+                    const int j0 = e.x, nv = e.y & 0xFF;
     #pragma unroll
                     for (int u = 0; u < SPW; ++u) {
                         const int slot = warp + 16 * u;
@@ -717,16 +718,16 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
     #pragma unroll
             for (int q = 0; q < PF; ++q)
                 fetch(q, pf[q]);
-            // This lane's four A chunks of slot `warp` (stage-relative) and its B
-            // element (lanes 0..15: batch column = lane).
-            uint32_t aoff[SPW][4], boff[SPW];
+            // This lane's four A chunks of slot `warp` (stage-relative), and
+            // its B element: warp b < B writes batch column b, lane l slot l.
+            uint32_t aoff[SPW][4];
     #pragma unroll
             for (int u = 0; u < SPW; ++u) {
     #pragma unroll
                 for (int j = 0; j < 4; ++j)
                     aoff[u][j] = a_chunk_off(lane, j, warp + 16 * u);
-                boff[u] = b_elem_off(lane & 15, warp + 16 * u, KB);
             }
+            const uint32_t boffc = b_elem_off(warp & (kMmaN - 1), lane & (KB - 1), KB);
 
             // Fold outputs of this thread: its tensor-memory lane (quadrant
             // warp % 4) in M-blocks 2 (warp / 4) and 2 (warp / 4) + 1.
@@ -798,8 +799,8 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
             int run = 0;
             int est = kb_base % nst, eph = (kb_base / nst) & 1; // stage, phase of K-block 0
             auto step = [&](int kb, const uint4 *v) {
-                const int fl = kbn[kb];
-                const int j0 = kbj[kb];
+                const int2 e = kbt[kb];
+                const int fl = e.y, j0 = e.x;
                 const int nv = fl & 0xFF; // valid slots of the K-block (at most KB)
                 run = (fl >> 8) & 0x1FFFFF;
                 const int kg = kb_base + kb;
@@ -816,8 +817,6 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
                 const uint32_t a_st = sA + (uint32_t)(s * AST);
     #pragma unroll
                 for (int u = 0; u < SPW; ++u) {
-                    const int slot = warp + 16 * u;
-                    const bool valid = slot < nv;
                     const uint32_t wv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
     #pragma unroll
                     for (int j = 0; j < 4; ++j) {
@@ -828,16 +827,14 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
                         st_shared_v4(a_st + aoff[u][j], w & 0x000F000Fu, w & 0x00F000F0u,
                                      w8 & 0x000F000Fu, w8 & 0x00F000F0u);
                     }
-                    if (lane < kMmaN) {
-                        // B operand: x' of this slot for batch column `lane`.
-                        const uint16_t xv = (valid && lane < p.B)
-                                                ? rxh[(size_t)lane * rs + j0 + slot]
-                                                : (uint16_t)0;
-                        asm volatile("st.shared.u16 [%0], %1;" ::"r"(sB + (uint32_t)(s * BST) +
-                                                                     boff[u]),
-                                     "h"(xv)
-                                     : "memory");
-                    }
+                }
+                if (warp < p.B && lane < KB) {
+                    // B operand: x' of batch column `warp` for slot `lane` (zero
+                    // past the K-block's valid rows), one coalesced read.
+                    const uint16_t xv = (lane < nv) ? rxh[(size_t)warp * rs + j0 + lane] : (uint16_t)0;
+                    asm volatile("st.shared.u16 [%0], %1;" ::"r"(sB + (uint32_t)(s * BST) + boffc),
+                                 "h"(xv)
+                                 : "memory");
                 }
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
