@@ -57,6 +57,7 @@
 #include "sgq_launch.h"
 
 #include <algorithm>
+#include <type_traits>
 
 namespace sgq {
 
@@ -273,6 +274,16 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
                  "r"(d)
+                 : "memory");
+}
+
+// The same at a compile-time offset from addr.
+template <int OFF>
+__device__ __forceinline__ void st_shared_v4_at(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                                uint32_t d)
+{
+    asm volatile("st.shared.v4.b32 [%0+%5], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b),
+                 "r"(c), "r"(d), "n"(OFF)
                  : "memory");
 }
 
@@ -718,15 +729,11 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
     #pragma unroll
             for (int q = 0; q < PF; ++q)
                 fetch(q, pf[q]);
-            // This lane's four A chunks of slot `warp` (stage-relative), and
-            // its B element: warp b < B writes batch column b, lane l slot l.
-            uint32_t aoff[SPW][4];
-    #pragma unroll
-            for (int u = 0; u < SPW; ++u) {
-    #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    aoff[u][j] = a_chunk_off(lane, j, warp + 16 * u);
-            }
+            // This lane's A chunks (stage-relative): word j of slot warp + 16 u
+            // sits 4096 j + 32768 u bytes after that of word 0 of slot `warp`
+            // (atoms g + 4 j, and two 8-row atom groups per 16 slots). Its B
+            // element: warp b < B writes batch column b, lane l slot l.
+            const uint32_t aoff = a_chunk_off(lane, 0, warp);
             const uint32_t boffc = b_elem_off(warp & (kMmaN - 1), lane & (KB - 1), KB);
 
             // Fold outputs of this thread: its tensor-memory lane (quadrant
@@ -818,15 +825,19 @@ __global__ void __launch_bounds__(kMThreads, 1) gemv_mma_kernel(const KParams kp
     #pragma unroll
                 for (int u = 0; u < SPW; ++u) {
                     const uint32_t wv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-    #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        // The raw codes as exact fp16 subnormals: q 2^-24 (low
-                        // nibbles) and q 2^-20 (high); invalid slots hold zero
-                        // codes and meet a zero B operand.
-                        const uint32_t w = wv[j], w8 = w >> 8;
-                        st_shared_v4(a_st + aoff[u][j], w & 0x000F000Fu, w & 0x00F000F0u,
-                                     w8 & 0x000F000Fu, w8 & 0x00F000F0u);
-                    }
+                    // The raw codes as exact fp16 subnormals: q 2^-24 (low
+                    // nibbles) and q 2^-20 (high); invalid slots hold zero
+                    // codes and meet a zero B operand.
+                    const uint32_t ab = a_st + aoff + 32768u * u;
+                    auto put = [&](const uint32_t w, auto off) {
+                        const uint32_t w8 = w >> 8;
+                        st_shared_v4_at<decltype(off)::value>(ab, w & 0x000F000Fu, w & 0x00F000F0u,
+                                                              w8 & 0x000F000Fu, w8 & 0x00F000F0u);
+                    };
+                    put(wv[0], std::integral_constant<int, 0>{});
+                    put(wv[1], std::integral_constant<int, 4096>{});
+                    put(wv[2], std::integral_constant<int, 8192>{});
+                    put(wv[3], std::integral_constant<int, 12288>{});
                 }
                 if (warp < p.B && lane < KB) {
                     // B operand: x' of batch column `warp` for slot `lane` (zero
