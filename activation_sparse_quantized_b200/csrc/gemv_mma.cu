@@ -22,8 +22,8 @@
 //    stages do not fit shared memory), a run's last block padded with zero
 //    rows.
 //  * 16 expanding warps; warp w expands slots w and w + 16 of every K-block.
-//    Its lanes read their own 16-byte columns of its rows into registers (4
-//    rows ahead) and store each code as the exact fp16 value q 2^-24 (2^-20
+//    Its lanes read their own 16-byte columns of its rows into registers (one
+//    K-block ahead) and store each code as the exact fp16 value q 2^-24 (2^-20
 //    for the high nibble of a byte): one AND per two codes, no zero point. A
 //    K-block's A operand (1024 outputs x its rows, M-major, 128-byte swizzle)
 //    and B operand (its rows x 16 batch columns of x' = x 2^S_b in fp16,
@@ -76,7 +76,7 @@ constexpr int kMBlocks = kTileN1 / 128;     // MMA M-blocks per tile
 __host__ __device__ constexpr int a_stage_bytes(int kb) { return kb * kTileN1 * 2; }
 __host__ __device__ constexpr int b_stage_bytes(int kb) { return kb * kMmaN * 2; }
 constexpr int kMaxStages = 4;               // operand stages (2..4, by shared memory)
-constexpr int kPfRows = 4;                  // rows of packed codes in flight per expanding lane
+constexpr int kPfRows = 2;                  // rows of packed codes in flight per expanding lane (one K-block)
 constexpr int kTmemCols = 512;              // two accumulator sets and the running totals
 // An accumulator set: the tile's 8 M-blocks and the row-sum block (below),
 // 16 columns each, 160 columns apart; the totals after both sets.
@@ -269,15 +269,7 @@ __device__ __forceinline__ void tmem_st16(uint32_t addr, const float *v)
                  : "memory");
 }
 
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d)
-{
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
-                 "r"(d)
-                 : "memory");
-}
-
-// The same at a compile-time offset from addr.
+// A 16-byte shared-memory store at a compile-time offset from addr.
 template <int OFF>
 __device__ __forceinline__ void st_shared_v4_at(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                                 uint32_t d)
