@@ -139,7 +139,7 @@ class ClockSampler:
             self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
             self.ok = True
-        except Exception as e:  # pragma: no cover - depends on the box
+        except Exception as e:  # pragma: no cover - NVML may be missing on the host
             self.err = str(e)
 
     def _sample(self):
